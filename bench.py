@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of blockwise causal varlen attention on B200.
+
+One step = the whole hot path on the packed zig-zag workload: zig-zag ring forward
+(planner, block forward with the online-softmax merge, finalise) and the ring
+backward fed the merged out/lse (Delta preprocess, block backward, dq conversion)
+over S = 16384 packed tokens (document lengths uniform in [512, 4096], multiples of
+2*cp), cp = 4 virtual ranks, 32 heads, head_dim 128, bf16 inputs.
+
+Metric: attention TFLOP/s of forward + backward, counting visible (q, k) pairs
+only: 4*D*H*pairs for the forward and 10*D*H*pairs for the backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cbv|reference] [--no-extra]
+
+With N > 1 (torchrun) every rank runs its own batch (different seed) on its own GPU:
+weak scaling, no data-path collective; the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "causal varlen attn TFLOP/s fwd+bwd (zig-zag ring, packed varlen)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["cbv", "reference"], default="cbv")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-extra", action="store_true", help="skip the other workloads' sub-benchmarks")
+    p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def profile_traffic(name: str):
+    """dram bytes per launch recorded in profiles/<name>.md ("dram_bytes_per_launch: N"), else None."""
+    path = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(path):
+        return None
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", open(path).read())
+    return float(m.group(1)) if m else None
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.lines: list[str] = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+def visible_pairs(cu, window=0):
+    from context_blockwise_causal_varlen_b200 import rank_pair_counts
+
+    return int(rank_pair_counts(cu, 1, "zigzag", window).sum())
+
+
+def make_ring_inputs(cu, H, D, seed, device):
+    from synth import torch_normal_bf16
+
+    S = int(cu[-1])
+    return [torch_normal_bf16((S, H, D), seed * 10 + i, device) for i in range(4)]  # q, k, v, dout
+
+
+def timed(fn, steps, warmup, stream_events=True):
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def extra_benchmarks(device, pk, pk_kind):
+    """The other workloads, one line each (not the headline)."""
+    import torch
+
+    import context_blockwise_causal_varlen_b200 as cbv
+    from synth import torch_normal_bf16
+    from synth.workloads import long_doc, paged_prefill, varlen_decode
+
+    res = {}
+    tf_peak = pk["bf16_tflops"]
+    # long single document, zig-zag and contiguous, full causal and sliding window
+    for layout, window in (("zigzag", 0), ("contiguous", 0), ("zigzag", 4096)):
+        w = long_doc(window=window)
+        q, k, v, do = make_ring_inputs(w.cu_seqlens, w.heads, w.head_dim, 7, device)
+        pairs = visible_pairs(w.cu_seqlens, window)
+        st = {}
+
+        def fwd():
+            st["o"], st["l"] = cbv.zigzag_ring_fwd(q, k, v, w.cu_seqlens, w.cp, window=window, layout=layout)
+
+        def bwd():
+            cbv.zigzag_ring_bwd(do, q, k, v, st["o"], st["l"], w.cu_seqlens, w.cp, window=window, layout=layout)
+
+        fwd()
+        t_f = timed(fwd, 5, 2)
+        t_b = timed(bwd, 5, 2)
+        f_fwd = 4 * w.head_dim * w.heads * pairs
+        f_bwd = 10 * w.head_dim * w.heads * pairs
+        key = f"long_doc_S65536_cp8_H16_{layout}" + (f"_W{window}" if window else "")
+        res[key] = {"fwd_tflops": f_fwd / t_f / 1e9, "bwd_tflops": f_bwd / t_b / 1e9,
+                    "fwd_bwd_tflops": (f_fwd + f_bwd) / (t_f + t_b) / 1e9,
+                    "fwd_bwd_frac": (f_fwd + f_bwd) / (t_f + t_b) / 1e9 / tf_peak, "ms": t_f + t_b}
+        del q, k, v, do, st
+        torch.cuda.empty_cache()
+    # paged KV-parallel prefill, round-robin shards
+    for window in (0, 8192):
+        w = paged_prefill(window=window)
+        q = torch_normal_bf16((w.hq, w.q_len, w.head_dim), 11, device)
+        kc = torch_normal_bf16((w.kv_len // w.block_size, w.hkv, w.block_size, w.head_dim), 12, device)
+        vc = torch_normal_bf16(kc.shape, 13, device)
+        perm = w.perm.astype(np.int64)
+        bt = torch.from_numpy(np.stack([perm[r::w.shards] for r in range(w.shards)]).astype(np.int32)).to(device)
+        fn = lambda: cbv.kvp_segmented_prefill(q, kc, vc, bt, cbv.KV_ROUND_ROBIN, w.seg_size, None,
+                                               w.global_q_offset, window, return_lse=False)
+        t = timed(fn, 10, 3)
+        qpos = w.global_q_offset + np.arange(w.q_len)
+        vis = np.minimum(qpos + 1, window) if window else qpos + 1
+        flops = 4 * w.head_dim * w.hq * int(vis.sum())
+        res[f"paged_prefill_S4096_KV32768_rr" + (f"_W{window}" if window else "")] = {
+            "tflops": flops / t / 1e9, "frac": flops / t / 1e9 / tf_peak, "ms": t}
+        del q, kc, vc
+        torch.cuda.empty_cache()
+    # one-query GQA varlen decode
+    w = varlen_decode()
+    cu_k = torch.from_numpy(w.cu_seqlens_k).to(device)
+    cu_q = torch.arange(w.num_seqs + 1, dtype=torch.int32, device=device)
+    tk = int(w.cu_seqlens_k[-1])
+    q = torch_normal_bf16((w.num_seqs, w.hq, w.head_dim), 21, device)
+    k = torch_normal_bf16((tk, w.hkv, w.head_dim), 22, device)
+    v = torch_normal_bf16((tk, w.hkv, w.head_dim), 23, device)
+    out = torch.empty_like(q)
+    ws = torch.empty(256, dtype=torch.uint8, device=device)
+    fn = lambda: cbv.varlen_decode(q, k, v, cu_q, cu_k, validate=False, out=out, workspace=ws)
+    t = timed(fn, 10, 3)
+    nbytes = 2 * tk * w.hkv * w.head_dim * 2 + 2 * q.numel() * 2 + 2 * cu_k.numel() * 4
+    res["varlen_decode_N8192_HQ32_HKV4"] = {"gbs": nbytes / t / 1e6, "frac": nbytes / t / 1e6 / pk["hbm_gbs"],
+                                            "ms": t, "bytes": nbytes}
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    # standalone merge at the packed workload's shapes
+    S, H, D = 16384, 32, 128
+    o = torch.randn((S, H, D), device=device)
+    l = torch.randn((H, S), device=device)
+    bo = torch.randn((S, H, D), device=device).to(torch.bfloat16)
+    bl = torch.randn((H, S), device=device)
+    t = timed(lambda: cbv.attn_merge(o, l, bo, bl), 20, 3)
+    nbytes = S * H * (D * 4 * 2 + D * 2 + 3 * 4)
+    res["merge_S16384_H32_D128"] = {"gbs": nbytes / t / 1e6, "frac": nbytes / t / 1e6 / pk["hbm_gbs"], "ms": t}
+    res["peak_kind"] = pk_kind
+    return res
+
+
+def cpu_baseline(cu, H, D, cp, budget_s=12.0):
+    """The oracle (ring forward + merged-lse backward, fp64) on a bounded sample of the workload."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import ring as R
+    from synth import normal_bf16, streams
+
+    d = int(np.argmax(np.diff(cu)))
+    L = int(cu[d + 1] - cu[d])
+    cu1 = np.array([0, L])
+    g = streams(99, 4)
+    flops = 0
+    heads = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and heads < H:
+        q, k, v, do = (normal_bf16(g[i], (L, 1, D)).astype(np.float64) for i in range(4))
+        o, l = R.ring_fwd(q, k, v, cu1, cp, D ** -0.5)
+        R.ring_bwd(do, q, k, v, o, l, cu1, cp, D ** -0.5)
+        flops += 14 * D * (L * (L + 1) // 2)
+        heads += 1
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle",
+            "sample": f"fp64 NumPy ring fwd+bwd of the longest document (L={L}, cp={cp}) for {heads} of {H} heads, "
+                      f"{dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The oracle, as it stands, on bounded samples of the same workload (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_info
+
+    from oracle import ring as R
+    from synth import normal_bf16, streams
+    from synth.workloads import packed_zigzag
+
+    w = packed_zigzag(args.seed)
+    cu = w.cu_seqlens
+    d = 0
+    L = int(cu[d + 1] - cu[d])
+    cu1 = np.array([0, L])
+    g = streams(99, 4)
+    q, k, v, do = (normal_bf16(g[i], (L, 1, w.head_dim)).astype(np.float64) for i in range(4))
+
+    def step():
+        o, l = R.ring_fwd(q, k, v, cu1, w.cp, w.head_dim ** -0.5)
+        R.ring_bwd(do, q, k, v, o, l, cu1, w.cp, w.head_dim ** -0.5)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    flops = 14 * w.head_dim * (L * (L + 1) // 2)
+    val = flops / dt / 1e12
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    sample = f"fp64 NumPy ring fwd+bwd of document 0 (L={L}, cp={w.cp}), one head per step"
+    line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "cp": w.cp, "heads": w.heads, "head_dim": w.head_dim,
+                       "l2": "inputs larger than L2 not applicable (CPU)"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import context_blockwise_causal_varlen_b200 as cbv
+    from synth.workloads import packed_zigzag
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    pk, pk_kind = peaks()
+
+    w = packed_zigzag(args.seed + rank)
+    cu = w.cu_seqlens
+    S, H, D, cp = w.total, w.heads, w.head_dim, w.cp
+    q, k, v, do = make_ring_inputs(cu, H, D, args.seed + rank, device)
+    pairs = visible_pairs(cu)
+    f_fwd, f_bwd = 4 * D * H * pairs, 10 * D * H * pairs
+    state = {}
+    ev = {"f0": [], "f1": [], "b1": []}
+
+    def step(record=False):
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            ev["f0"].append(e)
+        state["out"], state["lse"] = cbv.zigzag_ring_fwd(q, k, v, cu, cp)
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            ev["f1"].append(e)
+        state["grads"] = cbv.zigzag_ring_bwd(do, q, k, v, state["out"], state["lse"], cu, cp)
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            ev["b1"].append(e)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+        dist.barrier()
+    fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["f0"], ev["f1"])]))
+    bwd_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["f1"], ev["b1"])]))
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    ho = torch.empty_like(hq).pin_memory()
+    hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
+    dq_, dk_, dv_, do_ = (torch.empty_like(t) for t in (q, k, v, do))
+
+    def e2e_step():
+        for h, d in ((hq, q), (hk, k), (hv, v), (hdo, do_)):
+            d.copy_(h, non_blocking=True)
+        o, l = cbv.zigzag_ring_fwd(q, k, v, cu, cp)
+        gq, gk, gv = cbv.zigzag_ring_bwd(do_, q, k, v, o, l, cu, cp)
+        for h, d in ((ho, o), (hdq, gq), (hdk, gk), (hdv, gv)):
+            h.copy_(d, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, max(2, args.steps // 4), 2)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = sum(t.numel() * 2 for t in (q, k, v, do))
+    d2h = sum(t.numel() * 2 for t in (q, q, k, v))
+
+    total_flops = (f_fwd + f_bwd) * world
+    value = total_flops / (ms * 1e-3) / 1e12
+    if rank == 0:
+        # the dominant kernel: the block backward (10 of the 14 flops per pair)
+        dom_ms, dom_flops, dom_name = (bwd_ms, f_bwd, "bwd_kernel") if bwd_ms >= fwd_ms else (fwd_ms, f_fwd, "fwd_kernel")
+        achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "tokens": S, "docs": len(cu) - 1, "cp": cp, "heads": H, "head_dim": D,
+                       "layout": "zigzag", "visible_pairs_per_head": pairs,
+                       "l2": "inputs larger than L2 (q, k, v, dout 537 MB)", "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": profile_traffic(f"{dom_name}_packed_zigzag"),
+                         "kernel": dom_name, "peak_kind": f"{pk_kind} bf16 burst",
+                         "note": "duration = CUDA events around the API call on its stream (includes the call's "
+                                 "small helper kernels)"},
+            "phases_ms": {"fwd": fwd_ms, "bwd": bwd_ms},
+            "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * 4,
+            "clocks": clk,
+            "balance": {"zigzag_pairs_per_rank": cbv.rank_pair_counts(cu, cp, "zigzag").tolist(),
+                        "contiguous_pairs_per_rank": cbv.rank_pair_counts(cu, cp, "contiguous").tolist()},
+        }
+        if world == 1 and not args.no_cpu:
+            line["cpu_baseline"] = cpu_baseline(cu, H, D, cp)
+        if world == 1 and not args.no_extra:
+            line["extra"] = extra_benchmarks(device, pk, pk_kind)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

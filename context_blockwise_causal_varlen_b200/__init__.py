@@ -1,0 +1,431 @@
+"""Blockwise causal varlen attention on B200: Python binding of libcbv.so.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels (see ``include/cbv.h``).  PyTorch provides device memory and the
+current stream.  The binding fails loudly when ``libcbv.so`` is missing; there is
+no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcbv.so")
+ABI_VERSION = 1
+
+ZIGZAG, CONTIGUOUS = 0, 1
+KV_CONTIGUOUS, KV_ROUND_ROBIN = 0, 1
+SCHEDULE_FUSED, SCHEDULE_STEPWISE = 0, 1
+DTYPE_BF16, DTYPE_F32 = 0, 1
+
+STATUS = {
+    0: "OK", -1: "BAD_ARG", -2: "BAD_SHAPE", -3: "BAD_DTYPE", -4: "MISALIGNED", -5: "UNSUPPORTED_HEAD_DIM",
+    -6: "NOT_DIVISIBLE_2CP", -7: "NOT_CAUSAL", -8: "GQA_MISMATCH", -9: "BAD_CU_SEQLENS", -10: "Q_LEN_NOT_ONE",
+    -11: "WORKSPACE_TOO_SMALL", -12: "TIMEOUT", -13: "CUDA", -14: "VERSION",
+}
+
+
+class CbvError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"cbv error {STATUS.get(code, code)} ({code}): {message}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libcbv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m context_blockwise_causal_varlen_b200.build`")
+        _lib = ctypes.CDLL(LIB_PATH)
+        _declare(_lib)
+        if _lib.cbv_abi_version() != ABI_VERSION:
+            raise ImportError("libcbv.so ABI version mismatch")
+    return _lib
+
+
+# ----------------------------------------------------------------------------- C structs
+c_i32p = ctypes.POINTER(ctypes.c_int32)
+c_i64p = ctypes.POINTER(ctypes.c_int64)
+c_f32p = ctypes.POINTER(ctypes.c_float)
+
+
+class BlockFwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("num_docs", ctypes.c_int32),
+        ("cu_seqlens_q", c_i32p), ("cu_seqlens_k", c_i32p), ("q_pos_base", c_i32p), ("k_pos_base", c_i32p),
+        ("max_seqlen", ctypes.c_int32), ("scale", ctypes.c_float), ("causal", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("merge", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class RingArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("total", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("num_docs", ctypes.c_int32), ("cu_seqlens", c_i32p), ("max_seqlen", ctypes.c_int32),
+        ("cp", ctypes.c_int32), ("layout", ctypes.c_int32), ("scale", ctypes.c_float), ("causal", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("schedule", ctypes.c_int32),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
+        ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class BlockBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("dout", ctypes.c_void_p), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("num_docs", ctypes.c_int32),
+        ("cu_seqlens_q", c_i32p), ("cu_seqlens_k", c_i32p), ("q_pos_base", c_i32p), ("k_pos_base", c_i32p),
+        ("scale", ctypes.c_float), ("causal", ctypes.c_int32), ("window", ctypes.c_int32),
+        ("dq_acc", ctypes.c_void_p), ("dk_acc", ctypes.c_void_p), ("dv_acc", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class KvpArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("q_stride_head", ctypes.c_int64), ("q_stride_token", ctypes.c_int64),
+        ("q_len", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+        ("block_tables", ctypes.c_void_p), ("shards", ctypes.c_int32), ("blocks_per_shard", ctypes.c_int32),
+        ("kv_mode", ctypes.c_int32), ("seg_size", ctypes.c_int32), ("scale", ctypes.c_float),
+        ("global_q_offset", ctypes.c_int32), ("sliding_window", ctypes.c_int32),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("shard_out", ctypes.c_void_p),
+        ("shard_lse", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_k", ctypes.c_void_p),
+        ("num_seqs", ctypes.c_int32), ("total_q", ctypes.c_int64), ("total_k", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("validate", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+EXPORTS = [
+    "cbv_last_error_message", "cbv_abi_version", "cbv_read_status",
+    "cbv_local_cu_seqlens", "cbv_half_cu_seqlens", "cbv_get_half_index", "cbv_get_half_lse", "cbv_rank_tokens",
+    "cbv_rank_pair_counts", "cbv_ring_step",
+    "cbv_block_fwd_workspace_size", "cbv_attn_block_fwd", "cbv_attn_merge",
+    "cbv_zigzag_ring_fwd_workspace_size", "cbv_zigzag_ring_fwd", "cbv_zigzag_ring_bwd_workspace_size",
+    "cbv_zigzag_ring_bwd", "cbv_block_bwd_workspace_size", "cbv_attn_block_bwd",
+    "cbv_kvp_workspace_size", "cbv_kvp_segmented_prefill", "cbv_decode_workspace_size", "cbv_varlen_decode",
+]
+
+
+def _declare(L):
+    L.cbv_last_error_message.restype = ctypes.c_char_p
+    L.cbv_abi_version.restype = ctypes.c_int
+    L.cbv_read_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
+    L.cbv_local_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i32p]
+    L.cbv_half_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, c_i32p]
+    L.cbv_get_half_index.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, c_i32p, c_i64p]
+    L.cbv_get_half_lse.argtypes = [c_f32p, ctypes.c_int32, c_i32p, ctypes.c_int32, ctypes.c_int32, c_f32p]
+    L.cbv_rank_tokens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i32p]
+    L.cbv_rank_pair_counts.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i64p]
+    L.cbv_ring_step.argtypes = [ctypes.c_int32] * 4 + [c_i32p, c_i32p]
+    for name, st in (("block_fwd", BlockFwdArgs), ("zigzag_ring_fwd", RingArgs), ("zigzag_ring_bwd", RingArgs),
+                     ("block_bwd", BlockBwdArgs), ("kvp", KvpArgs), ("decode", DecodeArgs)):
+        f = getattr(L, f"cbv_{name}_workspace_size")
+        f.argtypes = [ctypes.POINTER(st)]
+        f.restype = ctypes.c_size_t
+    for name, st in (("cbv_attn_block_fwd", BlockFwdArgs), ("cbv_zigzag_ring_fwd", RingArgs),
+                     ("cbv_zigzag_ring_bwd", RingArgs), ("cbv_attn_block_bwd", BlockBwdArgs),
+                     ("cbv_kvp_segmented_prefill", KvpArgs), ("cbv_varlen_decode", DecodeArgs)):
+        getattr(L, name).argtypes = [ctypes.POINTER(st), ctypes.c_void_p]
+    L.cbv_attn_merge.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
+
+
+# ----------------------------------------------------------------------------- helpers
+def _check(rc: int):
+    if rc != 0:
+        raise CbvError(rc, lib().cbv_last_error_message().decode())
+
+
+def _host_i32(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.int32))
+
+
+def _p32(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(c_i32p)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise CbvError(-1, f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise CbvError(-3, f"{name} must be bfloat16, got {t.dtype}")
+    return t.contiguous()
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _header(st):
+    return dict(struct_size=ctypes.sizeof(st), abi_version=ABI_VERSION)
+
+
+def _scale(scale):
+    return 0.0 if scale is None else float(scale)
+
+
+def _layout(layout) -> int:
+    if isinstance(layout, str):
+        return {"zigzag": ZIGZAG, "contiguous": CONTIGUOUS}[layout]
+    return int(layout)
+
+
+def read_status(workspace: torch.Tensor) -> int:
+    """Device status word of the last call that used ``workspace`` (synchronises)."""
+    v = ctypes.c_int(0)
+    lib().cbv_read_status(_ptr(workspace), ctypes.byref(v), _stream(workspace.device))
+    return v.value
+
+
+# ----------------------------------------------------------------------------- planner (host)
+def local_cu_seqlens(cu_seqlens, cp: int, layout="zigzag") -> np.ndarray:
+    cu = _host_i32(cu_seqlens)
+    out = np.zeros_like(cu)
+    _check(lib().cbv_local_cu_seqlens(_p32(cu), len(cu) - 1, cp, _layout(layout), _p32(out)))
+    return out
+
+
+def half_cu_seqlens(cu_seqlens, cp: int) -> np.ndarray:
+    cu = _host_i32(cu_seqlens)
+    out = np.zeros_like(cu)
+    _check(lib().cbv_half_cu_seqlens(_p32(cu), len(cu) - 1, cp, _p32(out)))
+    return out
+
+
+def get_half_index(cu_local, front: bool) -> np.ndarray:
+    cu = _host_i32(cu_local)
+    n = ctypes.c_int64(0)
+    out = np.zeros(max(int(cu[-1]) // 2, 1), np.int32)
+    _check(lib().cbv_get_half_index(_p32(cu), len(cu) - 1, int(front), _p32(out), ctypes.byref(n)))
+    return out[: n.value]
+
+
+def get_half_lse(lse, cu_local, front: bool) -> np.ndarray:
+    lse = np.ascontiguousarray(np.asarray(lse, dtype=np.float32))
+    cu = _host_i32(cu_local)
+    out = np.zeros((lse.shape[0], int(cu[-1]) // 2), np.float32)
+    _check(lib().cbv_get_half_lse(lse.ctypes.data_as(c_f32p), lse.shape[0], _p32(cu), len(cu) - 1, int(front),
+                                  out.ctypes.data_as(c_f32p)))
+    return out
+
+
+def rank_tokens(cu_seqlens, cp: int, rank: int, layout="zigzag") -> np.ndarray:
+    cu = _host_i32(cu_seqlens)
+    out = np.zeros(max(int(cu[-1]) // cp, 1), np.int32)
+    _check(lib().cbv_rank_tokens(_p32(cu), len(cu) - 1, cp, rank, _layout(layout), _p32(out)))
+    return out[: int(cu[-1]) // cp]
+
+
+def rank_pair_counts(cu_seqlens, cp: int, layout="zigzag", window: int = 0) -> np.ndarray:
+    cu = _host_i32(cu_seqlens)
+    out = np.zeros(cp, np.int64)
+    _check(lib().cbv_rank_pair_counts(_p32(cu), len(cu) - 1, cp, _layout(layout), int(window),
+                                      out.ctypes.data_as(c_i64p)))
+    return out
+
+
+def ring_step(rank: int, step: int, cp: int, layout="zigzag") -> tuple[int, int]:
+    src, kind = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(lib().cbv_ring_step(rank, step, cp, _layout(layout), ctypes.byref(src), ctypes.byref(kind)))
+    return src.value, kind.value
+
+
+# ----------------------------------------------------------------------------- attention calls
+def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
+                    schedule: int = SCHEDULE_FUSED, max_seqlen: int = 0, out=None, lse=None, return_workspace=False):
+    """Ring forward over ``cp`` virtual ranks: ``(out [S,H,D] bf16, lse [H,S] f32)``."""
+    q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    S, H, D = q.shape
+    cu = _host_i32(cu_seqlens)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    a = RingArgs(**_header(RingArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), total=S, num_heads=H, num_kv_heads=k.shape[1],
+                 head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu), max_seqlen=max_seqlen, cp=cp,
+                 layout=_layout(layout), scale=_scale(scale), causal=1, window=int(window), schedule=int(schedule),
+                 out=_ptr(out), lse=_ptr(lse))
+    ws = _workspace(lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_zigzag_ring_fwd(ctypes.byref(a), _stream(q.device)))
+    return (out, lse, ws) if return_workspace else (out, lse)
+
+
+def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
+                    max_seqlen: int = 0, dq=None, dk=None, dv=None, return_workspace=False):
+    """Ring backward fed the merged out/lse: ``(dq, dk, dv)`` bf16."""
+    dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
+    S, H, D = q.shape
+    cu = _host_i32(cu_seqlens)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    a = RingArgs(**_header(RingArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), total=S, num_heads=H, num_kv_heads=k.shape[1],
+                 head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu), max_seqlen=max_seqlen, cp=cp,
+                 layout=_layout(layout), scale=_scale(scale), causal=1, window=int(window), schedule=0,
+                 out=_ptr(out), lse=_ptr(lse.contiguous()), dout=_ptr(dout), dq=_ptr(dq), dk=_ptr(dk), dv=_ptr(dv))
+    ws = _workspace(lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_zigzag_ring_bwd(ctypes.byref(a), _stream(q.device)))
+    return (dq, dk, dv, ws) if return_workspace else (dq, dk, dv)
+
+
+def attn_block_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int = 0, scale=None, causal: bool = True,
+                   window: int = 0, q_pos_base=None, k_pos_base=None, out=None, lse=None, merge: bool = False,
+                   out_dtype=torch.bfloat16):
+    """One varlen block: ``(out, lse)``; with ``merge=True`` merges into the running f32 ``(out, lse)`` in place."""
+    q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    Sq, H, D = q.shape
+    cq, ck = _host_i32(cu_seqlens_q), _host_i32(cu_seqlens_k)
+    qb = None if q_pos_base is None else _host_i32(q_pos_base)
+    kb = None if k_pos_base is None else _host_i32(k_pos_base)
+    if merge:
+        out_dtype = torch.float32
+        if out is None or lse is None:
+            raise CbvError(-1, "merge=True needs the running out (f32) and lse")
+    if out is None:
+        out = torch.empty((Sq, H, D), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((H, Sq), dtype=torch.float32, device=q.device)
+    a = BlockFwdArgs(**_header(BlockFwdArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), total_q=Sq, total_k=k.shape[0],
+                     num_heads=H, num_kv_heads=k.shape[1], head_dim=D, num_docs=len(cq) - 1, cu_seqlens_q=_p32(cq),
+                     cu_seqlens_k=_p32(ck), q_pos_base=_p32(qb), k_pos_base=_p32(kb), max_seqlen=int(max_seqlen),
+                     scale=_scale(scale), causal=int(bool(causal)), window=int(window), merge=int(bool(merge)),
+                     out_dtype=DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16, out=_ptr(out), lse=_ptr(lse))
+    ws = _workspace(lib().cbv_block_fwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_attn_block_fwd(ctypes.byref(a), _stream(q.device)))
+    return out, lse
+
+
+def attn_merge(out, lse, block_out, block_lse, return_weight: bool = False):
+    """In-place online-softmax merge of ``(block_out, block_lse)`` into the f32 running ``(out, lse)``."""
+    S, H, D = out.shape
+    w = torch.empty((H, S), dtype=torch.float32, device=out.device) if return_weight else None
+    dt = DTYPE_F32 if block_out.dtype == torch.float32 else DTYPE_BF16
+    _check(lib().cbv_attn_merge(_ptr(out), _ptr(lse), _ptr(block_out.contiguous()), dt, _ptr(block_lse.contiguous()),
+                                _ptr(w), S, H, D, _stream(out.device)))
+    return (out, lse, w) if return_weight else (out, lse)
+
+
+def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=None, causal: bool = True,
+                   window: int = 0, q_pos_base=None, k_pos_base=None, dq_acc=None, dk_acc=None, dv_acc=None):
+    """One block's backward fed the merged ``(out, lse)``; adds into f32 ``(dq_acc, dk_acc, dv_acc)``."""
+    dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
+    Sq, H, D = q.shape
+    Sk, Hkv, _ = k.shape
+    cq, ck = _host_i32(cu_seqlens_q), _host_i32(cu_seqlens_k)
+    qb = None if q_pos_base is None else _host_i32(q_pos_base)
+    kb = None if k_pos_base is None else _host_i32(k_pos_base)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq_acc = torch.zeros((Sq, H, D), **f32) if dq_acc is None else dq_acc
+    dk_acc = torch.zeros((Sk, Hkv, D), **f32) if dk_acc is None else dk_acc
+    dv_acc = torch.zeros((Sk, Hkv, D), **f32) if dv_acc is None else dv_acc
+    a = BlockBwdArgs(**_header(BlockBwdArgs), dout=_ptr(dout), q=_ptr(q), k=_ptr(k), v=_ptr(v), out=_ptr(out),
+                     lse=_ptr(lse.contiguous()), total_q=Sq, total_k=Sk, num_heads=H, num_kv_heads=Hkv, head_dim=D,
+                     num_docs=len(cq) - 1, cu_seqlens_q=_p32(cq), cu_seqlens_k=_p32(ck), q_pos_base=_p32(qb),
+                     k_pos_base=_p32(kb), scale=_scale(scale), causal=int(bool(causal)), window=int(window),
+                     dq_acc=_ptr(dq_acc), dk_acc=_ptr(dk_acc), dv_acc=_ptr(dv_acc))
+    ws = _workspace(lib().cbv_block_bwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_attn_block_bwd(ctypes.byref(a), _stream(q.device)))
+    return dq_acc, dk_acc, dv_acc
+
+
+def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_ROBIN, seg_size: int = 512,
+                          scale=None, global_q_offset: int = 0, sliding_window: int = 0, per_shard: bool = False,
+                          return_lse: bool = True):
+    """Paged KV-parallel prefill; q ``[HQ, S, D]`` -> ``out [HQ, S, D]`` (+ lse, + per-shard partials)."""
+    if not q.is_cuda or q.dtype != torch.bfloat16:
+        raise CbvError(-3, "q must be a CUDA bfloat16 tensor")
+    k_cache, v_cache = _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache")
+    HQ, S, D = q.shape
+    nb, HKV, bs, _ = k_cache.shape
+    bt = block_tables.to(device=q.device, dtype=torch.int32).contiguous()
+    R, bps = bt.shape
+    out = torch.empty((HQ, S, D), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((HQ, S), dtype=torch.float32, device=q.device) if return_lse else None
+    so = torch.empty((R, HQ, S, D), dtype=torch.float32, device=q.device) if per_shard else None
+    sl = torch.empty((R, HQ, S), dtype=torch.float32, device=q.device) if per_shard else None
+    a = KvpArgs(**_header(KvpArgs), q=_ptr(q), q_stride_head=q.stride(0), q_stride_token=q.stride(1), q_len=S,
+                num_heads=HQ, num_kv_heads=HKV, head_dim=D, k_cache=_ptr(k_cache), v_cache=_ptr(v_cache),
+                num_blocks=nb, block_size=bs, block_tables=_ptr(bt), shards=R, blocks_per_shard=bps,
+                kv_mode=int(kv_mode), seg_size=int(seg_size), scale=_scale(scale),
+                global_q_offset=int(global_q_offset), sliding_window=int(sliding_window), out=_ptr(out),
+                lse=_ptr(lse), shard_out=_ptr(so), shard_lse=_ptr(sl))
+    if q.stride(2) != 1:
+        raise CbvError(-4, "q's last dimension must be contiguous")
+    ws = _workspace(lib().cbv_kvp_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_kvp_segmented_prefill(ctypes.byref(a), _stream(q.device)))
+    res = [out]
+    if return_lse:
+        res.append(lse)
+    if per_shard:
+        res += [so, sl]
+    return tuple(res) if len(res) > 1 else out
+
+
+def varlen_decode(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, validate=None, out=None, workspace=None):
+    """One query per sequence, GQA, offsets read on the device: ``out [total_q, HQ, D]`` bf16."""
+    q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    if validate is None:
+        validate = not torch.cuda.is_current_stream_capturing()
+    cq = cu_seqlens_q.to(device=q.device, dtype=torch.int32).contiguous()
+    ck = cu_seqlens_k.to(device=q.device, dtype=torch.int32).contiguous()
+    out = torch.empty_like(q) if out is None else out
+    a = DecodeArgs(**_header(DecodeArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), out=_ptr(out), cu_seqlens_q=_ptr(cq),
+                   cu_seqlens_k=_ptr(ck), num_seqs=ck.numel() - 1, total_q=q.shape[0], total_k=k.shape[0],
+                   num_heads=q.shape[1], num_kv_heads=k.shape[1], head_dim=q.shape[2], scale=_scale(scale),
+                   validate=int(bool(validate)))
+    if cq.numel() != ck.numel():
+        raise CbvError(-9, "cu_seqlens_q and cu_seqlens_k sizes differ")
+    ws = _workspace(lib().cbv_decode_workspace_size(ctypes.byref(a)), q.device) if workspace is None else workspace
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_varlen_decode(ctypes.byref(a), _stream(q.device)))
+    return out

@@ -1,0 +1,772 @@
+// The C ABI of libcbv.so (include/cbv.h): argument checks, workspace layout,
+// tensor-map encoding and the launch sequence of every call.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/cbv.h"
+#include "kernels.h"
+#include "plan.h"
+#include "ptx.cuh"
+
+using namespace cbv;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(int err, const char* what) {
+  return fail(CBV_ERR_CUDA, "%s: %s", what, cudaGetErrorString((cudaError_t)err));
+}
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Bump allocator over the caller's workspace.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  }
+};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// rank-n tiled map; dims/strides in elements (strides for dims 1..n-1)
+int make_map(CUtensorMap* m, CUtensorMapDataType dt, int esize, int rank, const void* ptr, const uint64_t* dims,
+             const uint64_t* strides_el, const uint32_t* box, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return fail(CBV_ERR_CUDA, "cuTensorMapEncodeTiled is not available (driver too old or no GPU)");
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_el[i] * esize;
+  CUresult r = fn(m, dt, rank, const_cast<void*>(ptr), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CBV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return CBV_OK;
+}
+
+// token-major bf16 [T, H, D] (or any strides) as (D, H, T), box (64, 1, rows)
+int map_thd(CUtensorMap* m, const void* ptr, int64_t T, int H, int D, int64_t stride_t, int64_t stride_h, int rows) {
+  uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)std::max<int64_t>(T, 1)};
+  uint64_t st[2] = {(uint64_t)stride_h, (uint64_t)stride_t};
+  uint32_t box[3] = {64, 1, (uint32_t)rows};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3, ptr, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+float resolve_scale(float scale, int D) { return scale > 0.f ? scale : 1.0f / std::sqrt((float)D); }
+constexpr float kLog2e = 1.4426950408889634f;
+
+int check_header(uint32_t size, uint32_t expect, uint32_t ver) {
+  if (ver != CBV_ABI_VERSION) return fail(CBV_ERR_VERSION, "abi_version %u, library is %d", ver, CBV_ABI_VERSION);
+  if (size != expect) return fail(CBV_ERR_VERSION, "struct_size %u, library expects %u", size, expect);
+  return CBV_OK;
+}
+
+int check_heads(int H, int Hkv, int D) {
+  if (D != 64 && D != 128) return fail(CBV_ERR_UNSUPPORTED_HEAD_DIM, "head_dim %d (supported: 64, 128)", D);
+  if (H <= 0 || Hkv <= 0) return fail(CBV_ERR_BAD_SHAPE, "num_heads and num_kv_heads must be positive");
+  if (H % Hkv) return fail(CBV_ERR_GQA_MISMATCH, "GQA mismatch: %d q heads vs %d kv heads", H, Hkv);
+  return CBV_OK;
+}
+
+int check_cu(const int32_t* cu, int32_t num_docs, int64_t total, const char* what) {
+  std::string e = check_cu_seqlens(cu, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s: %s", what, e.c_str());
+  if ((int64_t)cu[num_docs] > total)
+    return fail(CBV_ERR_BAD_CU_SEQLENS, "%s: last offset %d exceeds the %lld rows", what, cu[num_docs], (long long)total);
+  return CBV_OK;
+}
+
+int check_max_seqlen(const int32_t* cu, int32_t num_docs, int32_t max_seqlen) {
+  if (max_seqlen <= 0) return CBV_OK;
+  for (int d = 0; d < num_docs; ++d)
+    if (cu[d + 1] - cu[d] > max_seqlen)
+      return fail(CBV_ERR_BAD_ARG, "max_seqlen %d is below document %d's length %d", max_seqlen, d, cu[d + 1] - cu[d]);
+  return CBV_OK;
+}
+
+int upload(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+  if (bytes == 0) return CBV_OK;
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
+  return e == cudaSuccess ? CBV_OK : cuda_fail(e, "uploading the schedule");
+}
+
+int zero_status(void* ws, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, s);
+  return e == cudaSuccess ? CBV_OK : cuda_fail(e, "clearing the status word");
+}
+
+struct PlanDev {
+  TileTask* tasks = nullptr;
+  Seg* segs = nullptr;
+};
+
+PlanDev carve_plan(Carve& c, const Plan& p) {
+  PlanDev d;
+  d.tasks = static_cast<TileTask*>(c.take(std::max<size_t>(1, p.tasks.size()) * sizeof(TileTask)));
+  d.segs = static_cast<Seg*>(c.take(std::max<size_t>(1, p.segs.size()) * sizeof(Seg)));
+  return d;
+}
+
+int upload_plan(const PlanDev& d, const Plan& p, cudaStream_t s) {
+  int rc = upload(d.tasks, p.tasks.data(), p.tasks.size() * sizeof(TileTask), s);
+  if (rc) return rc;
+  return upload(d.segs, p.segs.data(), p.segs.size() * sizeof(Seg), s);
+}
+
+int launch_rc(int e, const char* what) { return e == 0 ? CBV_OK : cuda_fail(e, what); }
+
+int grid_of(size_t tasks, int heads) {
+  const size_t g = tasks * (size_t)heads;
+  return g > (size_t)INT32_MAX ? -1 : (int)g;
+}
+
+// ------------------------------------------------------------------------ ring forward
+struct RingFwdLayout {
+  Plan fused;
+  std::vector<Plan> steps;
+  size_t bytes = 0;
+};
+
+int ring_common_checks(const cbv_ring_args* a) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_ring_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if (!a->causal) return fail(CBV_ERR_NOT_CAUSAL, "the ring layouts are causal only (zig-zag is meaningless otherwise)");
+  if (a->cp < 1) return fail(CBV_ERR_BAD_ARG, "cp must be >= 1");
+  if (a->layout != CBV_LAYOUT_ZIGZAG && a->layout != CBV_LAYOUT_CONTIGUOUS) return fail(CBV_ERR_BAD_ARG, "bad layout");
+  if ((rc = check_cu(a->cu_seqlens, a->num_docs, a->total, "cu_seqlens"))) return rc;
+  if (a->cu_seqlens[a->num_docs] != a->total)
+    return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens must end at total (%lld)", (long long)a->total);
+  if ((rc = check_max_seqlen(a->cu_seqlens, a->num_docs, a->max_seqlen))) return rc;
+  std::string e = check_divisible(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  if (a->schedule != CBV_SCHEDULE_FUSED && a->schedule != CBV_SCHEDULE_STEPWISE)
+    return fail(CBV_ERR_BAD_ARG, "bad schedule");
+  return CBV_OK;
+}
+
+RingFwdLayout ring_fwd_layout(const cbv_ring_args* a) {
+  RingFwdLayout L;
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  if (a->schedule == CBV_SCHEDULE_FUSED) {
+    L.fused = plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, -1, 128);
+    carve_plan(c, L.fused);
+  } else {
+    for (int s = 0; s < a->cp; ++s) {
+      L.steps.push_back(plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, s, 128));
+      carve_plan(c, L.steps.back());
+    }
+    c.take((size_t)a->total * a->num_heads * a->head_dim * sizeof(float));  // running out (fp32)
+  }
+  L.bytes = c.off;
+  return L;
+}
+
+FwdParams ring_fwd_params(const cbv_ring_args* a, int* rc) {
+  FwdParams p{};
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  *rc = map_thd(&p.tm_q, a->q, a->total, H, D, (int64_t)H * D, D, 128);
+  if (!*rc) *rc = map_thd(&p.tm_k, a->k, a->total, Hkv, D, (int64_t)Hkv * D, D, 128);
+  if (!*rc) *rc = map_thd(&p.tm_v, a->v, a->total, Hkv, D, (int64_t)Hkv * D, D, 128);
+  p.num_heads = H;
+  p.heads_per_kv = H / Hkv;
+  p.scale_log2 = resolve_scale(a->scale, D) * kLog2e;
+  p.window = a->window > 0 ? a->window : 0;
+  p.out_stride_t = (int64_t)H * D;
+  p.out_stride_h = D;
+  p.lse = a->lse;
+  p.lse_stride_h = a->total;
+  p.lse_stride_t = 1;
+  p.block_size = 1;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* cbv_last_error_message(void) { return g_err.c_str(); }
+int cbv_abi_version(void) { return CBV_ABI_VERSION; }
+
+int cbv_read_status(const void* workspace, int* status_out, void* stream) {
+  if (!workspace || !status_out) return fail(CBV_ERR_BAD_ARG, "NULL argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  *status_out = v;
+  if (v != 0) return fail(CBV_ERR_TIMEOUT, "a kernel gave up a wait (code 0x%x)", v);
+  return CBV_OK;
+}
+
+// ------------------------------------------------------------------------ planner exports
+int cbv_local_cu_seqlens(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t layout, int32_t* out) {
+  if (!out) return fail(CBV_ERR_BAD_ARG, "out is NULL");
+  std::string e = check_cu_seqlens(cu, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s", e.c_str());
+  e = check_divisible(cu, num_docs, cp, (Layout)layout);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  local_cu_seqlens(cu, num_docs, cp, out);
+  return CBV_OK;
+}
+
+int cbv_half_cu_seqlens(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t* out) {
+  if (!out) return fail(CBV_ERR_BAD_ARG, "out is NULL");
+  std::string e = check_cu_seqlens(cu, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s", e.c_str());
+  e = check_divisible(cu, num_docs, cp, kZigZag);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  half_cu_seqlens(cu, num_docs, cp, out);
+  return CBV_OK;
+}
+
+int cbv_get_half_index(const int32_t* cu_local, int32_t num_docs, int32_t front, int32_t* idx_out, int64_t* count_out) {
+  std::string e = check_cu_seqlens(cu_local, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s", e.c_str());
+  for (int d = 0; d < num_docs; ++d)
+    if ((cu_local[d + 1] - cu_local[d]) % 2) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "local document %d has odd length", d);
+  const int64_t n = get_half_index(cu_local, num_docs, front != 0, idx_out);
+  if (count_out) *count_out = n;
+  return CBV_OK;
+}
+
+int cbv_get_half_lse(const float* lse, int32_t num_heads, const int32_t* cu_local, int32_t num_docs, int32_t front,
+                     float* out) {
+  if (!lse || !out || num_heads < 0) return fail(CBV_ERR_BAD_ARG, "bad argument");
+  int64_t n = 0;
+  int rc = cbv_get_half_index(cu_local, num_docs, front, nullptr, &n);
+  if (rc) return rc;
+  std::vector<int32_t> idx(n);
+  get_half_index(cu_local, num_docs, front != 0, idx.data());
+  const int64_t S = cu_local[num_docs];
+  for (int h = 0; h < num_heads; ++h)
+    for (int64_t i = 0; i < n; ++i) out[h * n + i] = lse[h * S + idx[i]];
+  return CBV_OK;
+}
+
+int cbv_rank_tokens(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t rank, int32_t layout, int32_t* out) {
+  if (!out || rank < 0 || rank >= cp) return fail(CBV_ERR_BAD_ARG, "bad rank or NULL out");
+  std::string e = check_cu_seqlens(cu, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s", e.c_str());
+  e = check_divisible(cu, num_docs, cp, (Layout)layout);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  rank_tokens(cu, num_docs, cp, rank, (Layout)layout, out);
+  return CBV_OK;
+}
+
+int cbv_rank_pair_counts(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t layout, int32_t window,
+                         int64_t* counts_out) {
+  if (!counts_out) return fail(CBV_ERR_BAD_ARG, "counts_out is NULL");
+  std::string e = check_cu_seqlens(cu, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s", e.c_str());
+  e = check_divisible(cu, num_docs, cp, (Layout)layout);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  rank_pair_counts(cu, num_docs, cp, (Layout)layout, window, counts_out);
+  return CBV_OK;
+}
+
+int cbv_ring_step(int32_t rank, int32_t step, int32_t cp, int32_t layout, int32_t* src_out, int32_t* kind_out) {
+  if (!src_out || !kind_out || cp < 1 || rank < 0 || rank >= cp || step < 0 || step >= cp)
+    return fail(CBV_ERR_BAD_ARG, "bad argument");
+  ring_step(rank, step, cp, (Layout)layout, src_out, kind_out);
+  return CBV_OK;
+}
+
+// ------------------------------------------------------------------------ block forward
+static int block_fwd_checks(const cbv_block_fwd_args* a) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_block_fwd_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if ((rc = check_cu(a->cu_seqlens_q, a->num_docs, a->total_q, "cu_seqlens_q"))) return rc;
+  if ((rc = check_cu(a->cu_seqlens_k, a->num_docs, a->total_k, "cu_seqlens_k"))) return rc;
+  if ((rc = check_max_seqlen(a->cu_seqlens_q, a->num_docs, a->max_seqlen))) return rc;
+  if ((rc = check_max_seqlen(a->cu_seqlens_k, a->num_docs, a->max_seqlen))) return rc;
+  if (a->merge && a->out_dtype != CBV_DTYPE_F32) return fail(CBV_ERR_BAD_DTYPE, "merge = 1 needs an f32 out");
+  if (a->out_dtype != CBV_DTYPE_F32 && a->out_dtype != CBV_DTYPE_BF16) return fail(CBV_ERR_BAD_DTYPE, "bad out_dtype");
+  return CBV_OK;
+}
+
+size_t cbv_block_fwd_workspace_size(const cbv_block_fwd_args* a) {
+  if (block_fwd_checks(a)) return 0;
+  Plan p = plan_block_fwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs, a->causal != 0,
+                          a->window, a->num_heads, 128);
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  carve_plan(c, p);
+  return c.off;
+}
+
+int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
+  int rc = block_fwd_checks(a);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  Plan plan = plan_block_fwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs,
+                             a->causal != 0, a->window, H, 128);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, plan);
+  if (!a->workspace || a->workspace_bytes < c.off)
+    return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
+  FwdParams p{};
+  if ((rc = map_thd(&p.tm_q, a->q, a->total_q, H, D, (int64_t)H * D, D, 128))) return rc;
+  if ((rc = map_thd(&p.tm_k, a->k, a->total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  if ((rc = map_thd(&p.tm_v, a->v, a->total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)plan.tasks.size();
+  p.num_heads = H;
+  p.heads_per_kv = H / Hkv;
+  p.scale_log2 = resolve_scale(a->scale, D) * kLog2e;
+  p.window = a->window > 0 ? a->window : 0;
+  p.out = a->out;
+  p.out_stride_t = (int64_t)H * D;
+  p.out_stride_h = D;
+  p.lse = a->lse;
+  p.lse_stride_h = a->total_q;
+  p.lse_stride_t = 1;
+  p.out_mode = a->merge ? kOutMerge : (a->out_dtype == CBV_DTYPE_F32 ? kOutF32 : kOutBf16);
+  p.block_size = 1;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s))) return rc;
+  const int grid = grid_of(plan.tasks.size(), H);
+  if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
+  return launch_rc(launch_fwd(p, D, false, grid, s), "block forward launch");
+}
+
+// ------------------------------------------------------------------------ merge
+int cbv_attn_merge(float* out, float* lse, const void* block_out, int32_t block_out_dtype, const float* block_lse,
+                   float* weight_out, int64_t seqlen, int32_t num_heads, int32_t head_dim, void* stream) {
+  if (!out || !lse || !block_out || !block_lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (head_dim != 64 && head_dim != 128) return fail(CBV_ERR_UNSUPPORTED_HEAD_DIM, "head_dim %d", head_dim);
+  if (seqlen < 0 || num_heads <= 0) return fail(CBV_ERR_BAD_SHAPE, "bad shape");
+  if (block_out_dtype != CBV_DTYPE_BF16 && block_out_dtype != CBV_DTYPE_F32) return fail(CBV_ERR_BAD_DTYPE, "bad dtype");
+  if (!aligned16(out) || !aligned16(block_out)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  return launch_rc(launch_merge(out, lse, block_out, block_out_dtype == CBV_DTYPE_F32, block_lse, weight_out, seqlen,
+                                num_heads, head_dim, static_cast<cudaStream_t>(stream)),
+                   "merge launch");
+}
+
+// ------------------------------------------------------------------------ ring forward
+size_t cbv_zigzag_ring_fwd_workspace_size(const cbv_ring_args* a) {
+  if (ring_common_checks(a)) return 0;
+  return ring_fwd_layout(a).bytes;
+}
+
+int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
+  int rc = ring_common_checks(a);
+  if (rc) return rc;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RingFwdLayout L = ring_fwd_layout(a);
+  if (!a->workspace || a->workspace_bytes < L.bytes)
+    return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", L.bytes);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  FwdParams p = ring_fwd_params(a, &rc);
+  if (rc) return rc;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  const int D = a->head_dim, H = a->num_heads;
+  if (a->schedule == CBV_SCHEDULE_FUSED) {
+    PlanDev pd = carve_plan(c, L.fused);
+    if ((rc = upload_plan(pd, L.fused, s))) return rc;
+    p.tasks = pd.tasks;
+    p.segs = pd.segs;
+    p.num_tasks = (int)L.fused.tasks.size();
+    p.out = a->out;
+    p.out_mode = kOutBf16;
+    return launch_rc(launch_fwd(p, D, false, grid_of(L.fused.tasks.size(), H), s), "ring forward launch");
+  }
+  std::vector<PlanDev> pds;
+  for (auto& pl : L.steps) {
+    pds.push_back(carve_plan(c, pl));
+    if ((rc = upload_plan(pds.back(), pl, s))) return rc;
+  }
+  float* acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
+  for (int st = 0; st < a->cp; ++st) {
+    p.tasks = pds[st].tasks;
+    p.segs = pds[st].segs;
+    p.num_tasks = (int)L.steps[st].tasks.size();
+    p.out = acc;
+    p.out_mode = st == 0 ? kOutF32 : kOutMerge;
+    if ((rc = launch_rc(launch_fwd(p, D, false, grid_of(L.steps[st].tasks.size(), H), s), "ring step launch")))
+      return rc;
+  }
+  return launch_rc(launch_convert_bf16(acc, a->out, a->total * H * D, 1.f, s), "output conversion");
+}
+
+// ------------------------------------------------------------------------ paged KV-parallel prefill
+static int kvp_checks(const cbv_kvp_args* a) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_kvp_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if (a->q_len < 0 || a->shards < 1 || a->blocks_per_shard < 1 || a->num_blocks < 1)
+    return fail(CBV_ERR_BAD_SHAPE, "bad q_len / shards / blocks");
+  const int bs = a->block_size;
+  if (bs < 8 || bs > 128 || 128 % bs) return fail(CBV_ERR_BAD_ARG, "block_size must divide 128 and be >= 8");
+  if (a->seg_size <= 0 || a->seg_size % 128) return fail(CBV_ERR_BAD_ARG, "seg_size must be a positive multiple of 128");
+  if (a->kv_mode != CBV_KV_CONTIGUOUS && a->kv_mode != CBV_KV_ROUND_ROBIN) return fail(CBV_ERR_BAD_ARG, "bad kv_mode");
+  if (a->global_q_offset < 0) return fail(CBV_ERR_BAD_ARG, "global_q_offset must be >= 0");
+  if (!aligned16(a->q) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->out))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  if ((a->q_stride_token % 8) || (a->q_stride_head % 8)) return fail(CBV_ERR_MISALIGNED, "q strides must be multiples of 8 elements");
+  if ((a->shard_out == nullptr) != (a->shard_lse == nullptr)) return fail(CBV_ERR_BAD_ARG, "shard_out and shard_lse go together");
+  return CBV_OK;
+}
+
+static size_t kvp_layout(const cbv_kvp_args* a, Plan* plan_out) {
+  const int n_local = a->blocks_per_shard * a->block_size;
+  Plan plan = plan_kvp(a->q_len, a->num_heads, a->shards, n_local, a->seg_size, (KvMode)a->kv_mode, a->block_size,
+                       a->global_q_offset, a->sliding_window, a->shard_out != nullptr, 128);
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  carve_plan(c, plan);
+  const size_t rows = (size_t)a->num_heads * a->q_len;
+  if (!a->lse || a->shard_out) c.take(rows * sizeof(float));                // lse scratch / merged lse
+  if (a->shard_out) c.take(rows * a->head_dim * sizeof(float));             // merged fp32 out
+  if (plan_out) *plan_out = std::move(plan);
+  return c.off;
+}
+
+size_t cbv_kvp_workspace_size(const cbv_kvp_args* a) {
+  if (kvp_checks(a)) return 0;
+  return kvp_layout(a, nullptr);
+}
+
+int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
+  int rc = kvp_checks(a);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Plan plan;
+  const size_t need = kvp_layout(a, &plan);
+  if (!a->workspace || a->workspace_bytes < need) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", need);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, plan);
+  const size_t rows = (size_t)a->num_heads * a->q_len;
+  float* lse_scratch = (!a->lse || a->shard_out) ? static_cast<float*>(c.take(rows * sizeof(float))) : nullptr;
+  float* acc = a->shard_out ? static_cast<float*>(c.take(rows * a->head_dim * sizeof(float))) : nullptr;
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads, bs = a->block_size;
+  FwdParams p{};
+  if ((rc = map_thd(&p.tm_q, a->q, a->q_len, H, D, a->q_stride_token, a->q_stride_head, 128))) return rc;
+  {
+    uint64_t dims[4] = {(uint64_t)D, (uint64_t)bs, (uint64_t)Hkv, (uint64_t)a->num_blocks};
+    uint64_t st[3] = {(uint64_t)D, (uint64_t)bs * D, (uint64_t)Hkv * bs * D};
+    uint32_t box[4] = {64, (uint32_t)bs, 1, 1};
+    if ((rc = make_map(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 4, a->k_cache, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+    if ((rc = make_map(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 4, a->v_cache, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+  }
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)plan.tasks.size();
+  p.num_heads = H;
+  p.heads_per_kv = H / Hkv;
+  p.scale_log2 = resolve_scale(a->scale, D) * kLog2e;
+  p.window = a->sliding_window > 0 ? a->sliding_window : 0;
+  p.block_tables = a->block_tables;
+  p.blocks_per_shard = a->blocks_per_shard;
+  p.block_size = bs;
+  p.shards = a->shards;
+  p.kv_mode = a->kv_mode;
+  p.n_local = a->blocks_per_shard * bs;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s))) return rc;
+  const int grid = grid_of(plan.tasks.size(), H);
+  if (!a->shard_out) {
+    p.out = a->out;
+    p.out_mode = kOutBf16;
+    p.out_stride_t = D;
+    p.out_stride_h = (int64_t)a->q_len * D;
+    p.lse = a->lse ? a->lse : lse_scratch;
+    p.lse_stride_h = a->q_len;
+    p.lse_stride_t = 1;
+    return launch_rc(launch_fwd(p, D, true, grid, s), "prefill launch");
+  }
+  // per-shard partials, then an explicit online-softmax merge of the shards
+  p.out = a->shard_out;
+  p.out_mode = kOutF32;
+  p.out_stride_t = D;
+  p.out_stride_h = (int64_t)a->q_len * D;
+  p.out_shard_stride = (int64_t)H * a->q_len * D;
+  p.lse = a->shard_lse;
+  p.lse_stride_h = a->q_len;
+  p.lse_stride_t = 1;
+  p.lse_shard_stride = (int64_t)H * a->q_len;
+  if ((rc = launch_rc(launch_fwd(p, D, true, grid, s), "prefill launch"))) return rc;
+  cudaError_t e = cudaMemcpyAsync(acc, a->shard_out, rows * D * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(lse_scratch, a->shard_lse, rows * sizeof(float), cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copying shard 0");
+  for (int r = 1; r < a->shards; ++r) {
+    rc = launch_rc(launch_merge(acc, lse_scratch, a->shard_out + (size_t)r * rows * D, 1, a->shard_lse + (size_t)r * rows,
+                                nullptr, (int64_t)rows, 1, D, s),
+                   "shard merge");
+    if (rc) return rc;
+  }
+  if (a->lse) {
+    e = cudaMemcpyAsync(a->lse, lse_scratch, rows * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copying lse");
+  }
+  return launch_rc(launch_convert_bf16(acc, a->out, (int64_t)rows * D, 1.f, s), "output conversion");
+}
+
+// ------------------------------------------------------------------------ varlen decode
+size_t cbv_decode_workspace_size(const cbv_decode_args* a) {
+  (void)a;
+  return kStatusBytes;
+}
+
+int cbv_varlen_decode(const cbv_decode_args* a, void* stream) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_decode_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if (a->num_heads / a->num_kv_heads > 16) return fail(CBV_ERR_GQA_MISMATCH, "at most 16 q heads per kv head");
+  if (a->num_seqs < 0 || a->total_q < a->num_seqs || a->total_k < 0) return fail(CBV_ERR_BAD_SHAPE, "bad sizes");
+  if (!a->cu_seqlens_q || !a->cu_seqlens_k) return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens is NULL");
+  if (!a->workspace || a->workspace_bytes < kStatusBytes) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", kStatusBytes);
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->validate) {
+    std::vector<int32_t> cq(a->num_seqs + 1), ck(a->num_seqs + 1);
+    cudaError_t e = cudaMemcpyAsync(cq.data(), a->cu_seqlens_q, cq.size() * 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(ck.data(), a->cu_seqlens_k, ck.size() * 4, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading cu_seqlens");
+    for (int i = 0; i < a->num_seqs; ++i)
+      if (cq[i + 1] - cq[i] != 1)
+        return fail(CBV_ERR_Q_LEN_NOT_ONE, "sequence %d has %d query rows (one query per sequence only)", i, cq[i + 1] - cq[i]);
+    if (cq[0] < 0 || cq[a->num_seqs] > a->total_q) return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens_q out of range");
+    for (int i = 0; i < a->num_seqs; ++i)
+      if (ck[i + 1] < ck[i]) return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens_k must be non-decreasing");
+    if (ck[0] < 0 || ck[a->num_seqs] > a->total_k) return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens_k out of range");
+  }
+  const int D = a->head_dim, Hkv = a->num_kv_heads;
+  DecodeParams p{};
+  {
+    uint64_t dims[3] = {(uint64_t)D, (uint64_t)std::max<int64_t>(a->total_k, 1), (uint64_t)Hkv};
+    uint64_t st[2] = {(uint64_t)Hkv * D, (uint64_t)D};
+    const int hpc = Hkv % 4 == 0 ? 4 : (Hkv % 2 == 0 ? 2 : 1);
+    p.heads_per_cta = hpc;
+    uint32_t box[3] = {64, 32, (uint32_t)hpc};
+    if ((rc = make_map(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3, a->k, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+    if ((rc = make_map(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 3, a->v, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+  }
+  p.q = a->q;
+  p.out = a->out;
+  p.cu_q = a->cu_seqlens_q;
+  p.cu_k = a->cu_seqlens_k;
+  p.num_seqs = a->num_seqs;
+  p.hq = a->num_heads;
+  p.hkv = Hkv;
+  p.head_dim = D;
+  p.scale_log2 = resolve_scale(a->scale, D) * kLog2e;
+  p.status = static_cast<int*>(a->workspace);
+  if ((rc = zero_status(a->workspace, s))) return rc;
+  return launch_rc(launch_decode(p, s), "decode launch");
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------ backward
+namespace {
+
+int make_bwd_maps(BwdParams* p, const void* q, const void* dout, const void* k, const void* v, float* dq_acc,
+                  int64_t total_q, int64_t total_k, int H, int Hkv, int D) {
+  int rc;
+  if ((rc = map_thd(&p->tm_q, q, total_q, H, D, (int64_t)H * D, D, 64))) return rc;
+  if ((rc = map_thd(&p->tm_do, dout, total_q, H, D, (int64_t)H * D, D, 64))) return rc;
+  if ((rc = map_thd(&p->tm_k, k, total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  if ((rc = map_thd(&p->tm_v, v, total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)std::max<int64_t>(total_q, 1)};
+  uint64_t st[2] = {(uint64_t)D, (uint64_t)H * D};
+  uint32_t box[3] = {(uint32_t)D / 4, 1, 64};  // one warp's head-dim slice x 64 q rows
+  return make_map(&p->tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 3, dq_acc, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+struct BwdLayout {
+  Plan plan;
+  size_t bytes = 0;
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a) {
+  if (ring_common_checks(a)) return 0;
+  Plan plan = plan_ring_bwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_kv_heads, 128);
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  carve_plan(c, plan);
+  c.take((size_t)a->num_heads * a->total * sizeof(float));                 // Delta
+  c.take((size_t)a->total * a->num_heads * a->head_dim * sizeof(float));   // dq accumulator
+  return c.off;
+}
+
+int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
+  int rc = ring_common_checks(a);
+  if (rc) return rc;
+  if (!a->dout || !a->out || !a->lse || !a->dq || !a->dk || !a->dv) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) || !aligned16(a->dout) ||
+      !aligned16(a->dq) || !aligned16(a->dk) || !aligned16(a->dv))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  Plan plan = plan_ring_bwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, Hkv, 128);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, plan);
+  float* delta = static_cast<float*>(c.take((size_t)H * a->total * sizeof(float)));
+  float* dq_acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
+  if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
+  BwdParams p{};
+  if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, dq_acc, a->total, a->total, H, Hkv, D))) return rc;
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)plan.tasks.size();
+  p.num_heads = H;
+  p.num_kv_heads = Hkv;
+  p.heads_per_kv = H / Hkv;
+  p.scale = resolve_scale(a->scale, D);
+  p.scale_log2 = p.scale * kLog2e;
+  p.window = a->window > 0 ? a->window : 0;
+  p.lse = a->lse;
+  p.lse_stride_h = a->total;
+  p.delta = delta;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.dkv_stride_t = (int64_t)Hkv * D;
+  p.dkv_stride_h = D;
+  p.dkv_accumulate = 0;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->total, H, D, delta, dq_acc, s), "backward preprocess")))
+    return rc;
+  const int grid = grid_of(plan.tasks.size(), Hkv);
+  if ((rc = launch_rc(launch_bwd(p, D, grid, s), "backward launch"))) return rc;
+  return launch_rc(launch_convert_bf16(dq_acc, a->dq, a->total * H * D, 1.f, s), "dq conversion");
+}
+
+static int block_bwd_checks(const cbv_block_bwd_args* a) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_block_bwd_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if ((rc = check_cu(a->cu_seqlens_q, a->num_docs, a->total_q, "cu_seqlens_q"))) return rc;
+  if ((rc = check_cu(a->cu_seqlens_k, a->num_docs, a->total_k, "cu_seqlens_k"))) return rc;
+  if (!a->dout || !a->q || !a->k || !a->v || !a->out || !a->lse || !a->dq_acc || !a->dk_acc || !a->dv_acc)
+    return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) || !aligned16(a->dout) ||
+      !aligned16(a->dq_acc) || !aligned16(a->dk_acc) || !aligned16(a->dv_acc))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  return CBV_OK;
+}
+
+size_t cbv_block_bwd_workspace_size(const cbv_block_bwd_args* a) {
+  if (block_bwd_checks(a)) return 0;
+  Plan plan = plan_block_bwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs,
+                             a->causal != 0, a->window, a->num_kv_heads, 128);
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  carve_plan(c, plan);
+  c.take((size_t)a->num_heads * a->total_q * sizeof(float));
+  return c.off;
+}
+
+int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
+  int rc = block_bwd_checks(a);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  Plan plan = plan_block_bwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs,
+                             a->causal != 0, a->window, Hkv, 128);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, plan);
+  float* delta = static_cast<float*>(c.take((size_t)H * a->total_q * sizeof(float)));
+  if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
+  BwdParams p{};
+  if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, a->dq_acc, a->total_q, a->total_k, H, Hkv, D))) return rc;
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)plan.tasks.size();
+  p.num_heads = H;
+  p.num_kv_heads = Hkv;
+  p.heads_per_kv = H / Hkv;
+  p.scale = resolve_scale(a->scale, D);
+  p.scale_log2 = p.scale * kLog2e;
+  p.window = a->window > 0 ? a->window : 0;
+  p.lse = a->lse;
+  p.lse_stride_h = a->total_q;
+  p.delta = delta;
+  p.dk = a->dk_acc;
+  p.dv = a->dv_acc;
+  p.dkv_stride_t = (int64_t)Hkv * D;
+  p.dkv_stride_h = D;
+  p.dkv_accumulate = 1;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->total_q, H, D, delta, nullptr, s), "backward preprocess")))
+    return rc;
+  return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), Hkv), s), "backward launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,439 @@
+// Block backward on tcgen05, fed the MERGED softmax statistics.
+//
+// NeMo AutoModel, zigzag_ring_attention: _block_backward and
+// zigzag_ring_flash_attn_varlen_backward ("each block's flash backward is fed the
+// FINAL merged out/lse"); ulysses_attention._block0_backward.  With
+// P = exp(scale q k^T - lse) over a block's visible pairs and Delta = rowsum(dO * O):
+//   dV += P^T dO,  dP = dO V^T,  dS = P * (dP - Delta),  dQ += scale dS K,  dK += scale dS^T Q.
+//
+// One CTA owns a 128-key tile of one kv head and streams 64-row q tiles from every
+// segment (ring block) that sees it, for every q head of its GQA group, so dK and dV
+// accumulate in TMEM across all blocks and are written once (the ring's "K/V grads
+// travel back to their owner" becomes accumulation in place).  dQ^T = K^T dS^T is
+// formed per q tile in TMEM and added to an fp32 dq accumulator with a TMA bulk
+// reduce-add.
+//
+// Warps: 0 TMA producer (+ lse/Delta rows), 1 UMMA issuer (+ TMEM owner),
+// 2-5 P / dS (one key row per thread) and the dK/dV epilogue, 6-9 dQ readout.
+// TMEM columns: S^T [0,64), dP^T [64,128), dQ^T x2 [128,256), dV [256,256+D), dK [384,384+D).
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace cbv {
+
+namespace {
+
+constexpr int BN = 128;  // keys per CTA
+constexpr int BM = 64;   // q rows per streamed tile
+constexpr int kThreads = 320;
+
+struct QTile {
+  int32_t q_row;   // first q row
+  int32_t qpos0;   // its position
+  int32_t nvalid;  // valid rows
+  int32_t head;    // q head
+  int32_t causal;
+  int32_t need_mask;
+};
+
+struct QIter {
+  int32_t hs = 0, si = 0, j = 0, jn = 0;
+  Seg seg;
+};
+
+// Enumerates the q tiles (over the GQA group's q heads and all segments) that see
+// at least one key of the tile.  Every role runs its own copy.
+__device__ __forceinline__ bool next_qtile(const BwdParams& p, const TileTask& t, int kvh, QIter& it, QTile& r) {
+  const int32_t kp0 = t.pos0, kp1 = t.pos0 + t.rows - 1;
+  const int32_t W = p.window;
+  while (true) {
+    if (it.j >= it.jn) {
+      if (it.si >= t.nseg) {
+        it.hs++;
+        it.si = 0;
+        if (it.hs >= p.heads_per_kv) return false;
+      }
+      if (t.nseg == 0) return false;
+      it.seg = p.segs[t.seg0 + it.si];
+      it.si++;
+      const bool cz = (it.seg.flags & kSegCausal) || W > 0;
+      int32_t cmin = 0, cmax = it.seg.rows - 1;
+      if (cz) cmin = max(cmin, kp0 - it.seg.pos0);
+      if (W > 0) cmax = min(cmax, kp1 + W - 1 - it.seg.pos0);
+      if (cmax < cmin) {
+        it.j = it.jn = 0;
+        continue;
+      }
+      it.j = cmin / BM;
+      it.jn = cmax / BM + 1;
+    }
+    const int32_t j = it.j++;
+    const int32_t c0 = j * BM;
+    r.nvalid = min(BM, it.seg.rows - c0);
+    r.q_row = it.seg.row0 + c0;
+    r.qpos0 = it.seg.pos0 + c0;
+    r.head = kvh * p.heads_per_kv + it.hs;
+    r.causal = it.seg.flags & kSegCausal;
+    const bool cz = r.causal || W > 0;
+    const int32_t qa = r.qpos0, qb = r.qpos0 + r.nvalid - 1;
+    const bool all_vis = (r.nvalid == BM) && (t.rows == BN) && (!cz || qa >= kp1) && (W <= 0 || qb - kp0 < W);
+    r.need_mask = !all_vis;
+    return true;
+  }
+}
+
+template <int D>
+struct BwdSmem {
+  static constexpr uint32_t kKV = BN * D * 2;   // K or V tile (128 x D)
+  static constexpr uint32_t kQT = BM * D * 2;   // a q / dO tile (64 x D)
+  static constexpr uint32_t kPT = BN * BM * 2;  // P^T or dS^T (128 x 64)
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kKV;
+  static constexpr uint32_t kQ = kV + kKV;           // 2 stages
+  static constexpr uint32_t kDO = kQ + 2 * kQT;      // 2 stages
+  static constexpr uint32_t kPt = kDO + 2 * kQT;
+  static constexpr uint32_t kDSt = kPt + kPT;
+  static constexpr uint32_t kDQ = kDSt + kPT;        // fp32 staging [64][D]
+  static constexpr uint32_t kRow = kDQ + BM * D * 4;  // per stage: lse*log2e [64], Delta [64]
+  static constexpr uint32_t kBars = kRow + 2 * 2 * BM * 4;
+  static constexpr uint32_t kEnd = kBars + 256;
+  static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
+};
+
+enum BBar {
+  bKVFull = 0,
+  bQFull = 1,    // +stage
+  bQEmpty = 3,   // +stage
+  bSFull = 5,
+  bSFree = 6,
+  bPFull = 7,
+  bPtFree = 8,
+  bDQFull = 9,   // +buffer
+  bDQFree = 11,  // +buffer
+  bAccDone = 13,
+  bBNum = 14
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
+  using L = BwdSmem<D>;
+  constexpr int KH = D / 64;  // 64-column halves
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = sm + L::kK;
+  uint8_t* sV = sm + L::kV;
+  uint8_t* sQ = sm + L::kQ;
+  uint8_t* sDO = sm + L::kDO;
+  uint8_t* sPt = sm + L::kPt;
+  uint8_t* sDSt = sm + L::kDSt;
+  float* sDQ = reinterpret_cast<float*>(sm + L::kDQ);
+  float* sRow = reinterpret_cast<float*>(sm + L::kRow);  // [stage][lse2 64 | delta 64]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + bBNum);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int task_idx = blockIdx.x / p.num_kv_heads;
+  const int kvh = blockIdx.x % p.num_kv_heads;
+  const TileTask t = p.tasks[task_idx];
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[bKVFull], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[bQFull + s], 2);  // TMA bytes + the producer warp's lse/Delta stores
+      mbar_init(&bar[bQEmpty + s], 1);
+      mbar_init(&bar[bDQFull + s], 1);
+      mbar_init(&bar[bDQFree + s], 4);
+    }
+    mbar_init(&bar[bSFull], 1);
+    mbar_init(&bar[bSFree], 4);
+    mbar_init(&bar[bPFull], 4);
+    mbar_init(&bar[bPtFree], 1);
+    mbar_init(&bar[bAccDone], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDP = tmem + 64, tDQ0 = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_q);
+      mbar_arrive_expect_tx(&bar[bKVFull], 2 * L::kKV);
+      for (int h = 0; h < KH; ++h) {
+        tma_load_3d(sK + h * 16384, &p.tm_k, &bar[bKVFull], h * 64, kvh, t.row0);
+        tma_load_3d(sV + h * 16384, &p.tm_v, &bar[bKVFull], h * 64, kvh, t.row0);
+      }
+    }
+    QIter it;
+    QTile r;
+    int j = 0;
+    while (next_qtile(p, t, kvh, it, r)) {
+      const int st = j & 1;
+      if (!mbar_wait_warp(&bar[bQEmpty + st], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar[bQFull + st], 2 * L::kQT);
+        for (int h = 0; h < KH; ++h) {
+          tma_load_3d(sQ + st * L::kQT + h * 8192, &p.tm_q, &bar[bQFull + st], h * 64, r.head, r.q_row);
+          tma_load_3d(sDO + st * L::kQT + h * 8192, &p.tm_do, &bar[bQFull + st], h * 64, r.head, r.q_row);
+        }
+      }
+      float* row = sRow + st * 2 * BM;
+      const float* lse = p.lse + (int64_t)r.head * p.lse_stride_h;
+      const float* dl = p.delta + (int64_t)r.head * p.lse_stride_h;
+      for (int c = lane; c < BM; c += 32) {
+        const bool v = c < r.nvalid;
+        row[c] = v ? __ldg(&lse[r.q_row + c]) * kLog2e : INFINITY;
+        row[BM + c] = v ? __ldg(&dl[r.q_row + c]) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[bQFull + st]);
+      ++j;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_st = idesc_bf16(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
+      constexpr uint32_t id_kv = idesc_bf16(BN, D, false, true);     // dV, dK: 128 x D, K = 64
+      constexpr uint32_t id_dq = idesc_bf16(D, BM, true, true);      // dQ^T: D x 64, K = 128
+      const uint32_t k0 = smem_u32(sK), v0 = smem_u32(sV), q0 = smem_u32(sQ), do0 = smem_u32(sDO);
+      const uint32_t pt0 = smem_u32(sPt), ds0 = smem_u32(sDSt);
+      bool ok = mbar_wait(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
+      tc_fence_after();
+      auto issue_sdp = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&bar[bQFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait(&bar[bSFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t bo = st * L::kQT + (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_bf16_ss(tS, sdesc_sw128(k0 + ao, 16, 1024), sdesc_sw128(q0 + bo, 16, 1024), id_st, kk > 0);
+          umma_bf16_ss(tDP, sdesc_sw128(v0 + ao, 16, 1024), sdesc_sw128(do0 + bo, 16, 1024), id_st, kk > 0);
+        }
+        umma_commit(&bar[bSFull]);
+        return true;
+      };
+      QIter it;
+      QTile r;
+      int n = 0;
+      {
+        QIter c2;
+        QTile r2;
+        while (next_qtile(p, t, kvh, c2, r2)) ++n;
+      }
+      if (ok && n > 0) ok = issue_sdp(0);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j & 1;
+        if (j + 1 < n && !(ok = issue_sdp(j + 1))) break;
+        if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint64_t pa = sdesc_sw128(pt0 + kk * 32, 16, 1024);
+          const uint64_t da = sdesc_sw128(ds0 + kk * 32, 16, 1024);
+          const uint64_t ob = sdesc_sw128(do0 + st * L::kQT + kk * 2048, 8192, 1024);
+          const uint64_t qb = sdesc_sw128(q0 + st * L::kQT + kk * 2048, 8192, 1024);
+          umma_bf16_ss(tDV, pa, ob, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ss(tDK, da, qb, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (!mbar_wait(&bar[bDQFree + st], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t ka = sdesc_sw128(k0 + kk * 2048, 16384, 1024);
+          const uint64_t sb = sdesc_sw128(ds0 + kk * 2048, 16384, 1024);
+          umma_bf16_ss(tDQ0 + st * 64, ka, sb, id_dq, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar[bQEmpty + st]);
+        umma_commit(&bar[bPtFree]);
+        umma_commit(&bar[bDQFull + st]);
+      }
+      (void)it;
+      (void)r;
+      if (n > 0) umma_commit(&bar[bAccDone]);
+      else mbar_arrive(&bar[bAccDone]);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ P / dS (thread = key row)
+    const int quarter = warp & 3;
+    const int krow = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int32_t kpos = t.pos0 + krow;
+    const bool kvalid = krow < t.rows;
+    const int32_t W = p.window;
+    const float sl2 = p.scale_log2;
+    const uint32_t pt_row = smem_u32(sPt), ds_row = smem_u32(sDSt);
+    QIter it;
+    QTile r;
+    int j = 0;
+    bool ok = true;
+    while (next_qtile(p, t, kvh, it, r)) {
+      const int st = j & 1;
+      if (!mbar_wait_warp(&bar[bQFull + st], (j >> 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+      if (!mbar_wait_warp(&bar[bSFull], j & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+      tc_fence_after();
+      const float* row = sRow + st * 2 * BM;
+      uint32_t pp[BM / 2], pd[BM / 2];
+#pragma unroll
+      for (int hc = 0; hc < BM; hc += 32) {
+        uint32_t s[32], dp[32];
+        tmem_ld32(tS + lane_base + hc, s);
+        tmem_ld32(tDP + lane_base + hc, dp);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = hc + c + e;
+            bool vis = true;
+            if (r.need_mask) {
+              const int32_t qpos = r.qpos0 + col;
+              vis = kvalid && col < r.nvalid;
+              if (r.causal || W > 0) vis = vis && (kpos <= qpos);
+              if (W > 0) vis = vis && (qpos - kpos < W);
+            }
+            const float pe = vis ? ex2_approx(__uint_as_float(s[c + e]) * sl2 - row[col]) : 0.f;
+            pv[e] = pe;
+            dv[e] = pe * (__uint_as_float(dp[c + e]) - row[BM + col]);
+          }
+          pp[(hc + c) / 2] = pack_bf16x2(pv[0], pv[1]);
+          pd[(hc + c) / 2] = pack_bf16x2(dv[0], dv[1]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[bSFree]);
+      if (j > 0 && !mbar_wait_warp(&bar[bPtFree], (j - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        st_shared_v4(pt_row + sw128_offset(krow, ch), pp[ch * 4], pp[ch * 4 + 1], pp[ch * 4 + 2], pp[ch * 4 + 3]);
+        st_shared_v4(ds_row + sw128_offset(krow, ch), pd[ch * 4], pd[ch * 4 + 1], pd[ch * 4 + 2], pd[ch * 4 + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[bPFull]);
+      ++j;
+    }
+    // ---------------------------------------------------------------- dK / dV epilogue
+    if (ok && mbar_wait_warp(&bar[bAccDone], 0, p.status, kDevTimeoutEpilogue)) {
+      tc_fence_after();
+      const bool any = j > 0;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_base;
+        const float mul = which == 0 ? 1.f : p.scale;
+        void* dst_base = which == 0 ? p.dv : p.dk;
+        const int64_t off = (int64_t)(t.row0 + krow) * p.dkv_stride_t + (int64_t)kvh * p.dkv_stride_h;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tsrc + c, o);
+          tmem_ld_wait();
+          if (!kvalid) continue;
+          if (p.dkv_accumulate) {
+            if (!any) continue;
+            float* dst = reinterpret_cast<float*>(dst_base) + off + c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float4 a = *reinterpret_cast<float4*>(dst + e);
+              a.x += __uint_as_float(o[e]) * mul;
+              a.y += __uint_as_float(o[e + 1]) * mul;
+              a.z += __uint_as_float(o[e + 2]) * mul;
+              a.w += __uint_as_float(o[e + 3]) * mul;
+              *reinterpret_cast<float4*>(dst + e) = a;
+            }
+          } else {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(dst_base) + off + c;
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              float x[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) x[q] = any ? __uint_as_float(o[e + q]) * mul : 0.f;
+              uint4 v = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                                   pack_bf16x2(x[6], x[7]));
+              *reinterpret_cast<uint4*>(dst + e) = v;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ dQ readout (thread = head-dim row)
+    // Each warp owns D/4 head-dim rows and adds its [64 x D/4] slice with its own
+    // bulk reduce, so the four warps never wait on one another.
+    const int quarter = warp & 3;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    constexpr int DW = D / 4;  // head-dim rows per warp
+    // M = 128: lane l of quarter q holds d = 32q + l; M = 64: lanes 0-15 of quarter q hold d = 16q + l
+    const bool dvalid = lane < DW;
+    float* region = sDQ + quarter * (BM * DW);
+    QIter it;
+    QTile r;
+    int j = 0;
+    while (next_qtile(p, t, kvh, it, r)) {
+      const int st = j & 1;
+      if (!mbar_wait_warp(&bar[bDQFull + st], (j >> 1) & 1, p.status, kDevTimeoutEpilogue)) break;
+      tc_fence_after();
+      uint32_t v[BM];
+      tmem_ld32(tDQ0 + st * 64 + lane_base, v);
+      tmem_ld32(tDQ0 + st * 64 + lane_base + 32, v + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar[bDQFree + st]);
+        bulk_wait_group_read<0>();  // this warp's previous reduce has finished reading its region
+      }
+      __syncwarp();
+      if (dvalid) {
+#pragma unroll
+        for (int c = 0; c < BM; ++c) region[c * DW + lane] = __uint_as_float(v[c]) * p.scale;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row);
+        bulk_commit_group();
+      }
+      ++j;
+    }
+    if (lane == 0) bulk_wait_group<0>();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+int launch_bwd_t(const BwdParams& p, int grid, cudaStream_t stream) {
+  auto kern = bwd_kernel<D>;
+  const uint32_t smem = BwdSmem<D>::kDynamic;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return (int)e;
+  kern<<<grid, kThreads, smem, stream>>>(p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream) {
+  if (grid <= 0) return 0;
+  if (head_dim == 128) return launch_bwd_t<128>(p, grid, stream);
+  if (head_dim == 64) return launch_bwd_t<64>(p, grid, stream);
+  return (int)cudaErrorInvalidValue;
+}
+
+}  // namespace cbv

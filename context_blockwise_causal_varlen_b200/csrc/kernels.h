@@ -1,0 +1,91 @@
+// Kernel parameter blocks and launchers shared by the C ABI and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "plan.h"
+
+namespace cbv {
+
+// Output modes of the forward kernel's epilogue.
+enum OutMode : int32_t {
+  kOutBf16 = 0,   // write normalised out (bf16) and lse
+  kOutF32 = 1,    // write normalised out (fp32) and lse
+  kOutMerge = 2,  // merge into a running fp32 (out, lse) pair in place (online-softmax identity)
+};
+
+struct FwdParams {
+  CUtensorMap tm_q;  // (D, H, T) bf16, box (64, 1, 128), 128B swizzle
+  CUtensorMap tm_k;  // ring: (D, Hkv, T) box (64, 1, 128); paged: (D, bs, Hkv, pages) box (64, bs, 1, 1)
+  CUtensorMap tm_v;
+  const TileTask* tasks;
+  const Seg* segs;
+  int32_t num_tasks;
+  int32_t num_heads;
+  int32_t heads_per_kv;
+  float scale_log2;  // softmax scale * log2(e)
+  int32_t window;
+  void* out;
+  int64_t out_stride_t, out_stride_h;  // elements
+  float* lse;
+  int64_t lse_stride_h, lse_stride_t;  // elements
+  int32_t out_mode;
+  int64_t out_shard_stride, lse_shard_stride;  // per-shard outputs (task.aux = shard >= 0)
+  // paged KV
+  const int32_t* block_tables;  // [shards, blocks_per_shard]
+  int32_t blocks_per_shard, block_size, shards, kv_mode, n_local;
+  int* status;  // device status word (0 = ok)
+};
+
+struct BwdParams {
+  CUtensorMap tm_q;     // (D, H, T) bf16, box (64, 1, 64)
+  CUtensorMap tm_do;    // (D, H, T) bf16, box (64, 1, 64)
+  CUtensorMap tm_k;     // (D, Hkv, T) bf16, box (64, 1, 128)
+  CUtensorMap tm_v;
+  CUtensorMap tm_dq;    // (D, H, T) fp32, box (D, 1, 64), no swizzle (reduce-add target)
+  const TileTask* tasks;
+  const Seg* segs;
+  int32_t num_tasks;
+  int32_t num_heads, heads_per_kv, num_kv_heads;
+  float scale, scale_log2;
+  int32_t window;
+  const float* lse;    // [H, T] merged lse (natural log)
+  int64_t lse_stride_h;
+  const float* delta;  // [H, T] rowsum(dO * O)
+  // dk/dv outputs: bf16 (write) or fp32 (accumulate)
+  void* dk;
+  void* dv;
+  int64_t dkv_stride_t, dkv_stride_h;
+  int32_t dkv_accumulate;  // 0: write bf16; 1: add into fp32
+  int* status;
+};
+
+int launch_fwd(const FwdParams& p, int head_dim, bool paged, int grid, cudaStream_t stream);
+int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream);
+
+// Delta = rowsum(dout * out) per (token, head), written [H, T]; optionally zero dq_acc.
+int launch_bwd_preprocess(const void* dout, const void* out, int64_t total, int32_t heads, int32_t head_dim,
+                          float* delta, float* dq_acc, cudaStream_t stream);
+// fp32 [T, H, D] -> bf16, times `mul`.
+int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
+// Standalone merge of (block_out, block_lse) into a running fp32 (out, lse).
+int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
+                 float* weight_out, int64_t seqlen, int32_t heads, int32_t head_dim, cudaStream_t stream);
+// One-query varlen GQA decode.
+struct DecodeParams {
+  CUtensorMap tm_k;  // (D, Hkv, Tk) bf16, box (64, 1, 32), 128B swizzle
+  CUtensorMap tm_v;
+  const void* q;      // [Tq, HQ, D]
+  void* out;          // [Tq, HQ, D]
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int32_t num_seqs, hq, hkv, head_dim;
+  int32_t heads_per_cta;  // kv heads per CTA: 4, 2 or 1, dividing hkv (the TMA box never leaves the tensor)
+  float scale_log2;
+  int* status;
+};
+int launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+}  // namespace cbv

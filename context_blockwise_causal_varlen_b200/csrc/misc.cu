@@ -1,0 +1,156 @@
+// Memory-bound helper kernels: the standalone online-softmax merge, the backward
+// preprocess (Delta = rowsum(dO * O)) and the fp32 -> bf16 conversion.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace cbv {
+
+namespace {
+
+// One warp per (token, head) row; every lane owns D/32 consecutive elements.
+//
+// NeMo AutoModel, zigzag_ring_attention, update_out_and_lse (and ring_attention,
+// _update_out_and_lse): with w = sigmoid(block_lse - lse),
+//   out' = out - w (out - block_out),  lse' = lse - logsigmoid(lse - block_lse),
+// evaluated here as lse' = m + log(e^(lse-m) + e^(blse-m)), m = max(lse, blse), and
+// out' = out e^(lse-lse') + block_out e^(blse-lse'), which is the same quantity;
+// a side at -inf is the identity of the merge.
+template <int D, bool BF16_IN>
+__global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ out, float* __restrict__ lse,
+                                                    const void* __restrict__ block_out,
+                                                    const float* __restrict__ block_lse, float* __restrict__ weight,
+                                                    int64_t seqlen, int heads) {
+  constexpr int E = D / 32;
+  const int64_t rowid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (rowid >= seqlen * heads) return;
+  const int64_t tok = rowid / heads;
+  const int h = (int)(rowid % heads);
+  const int64_t li = (int64_t)h * seqlen + tok;
+  const float a = lse[li];
+  const float b = block_lse[li];
+  const float m = fmaxf(a, b);
+  float wa, wb, nl, w;
+  if (m == -INFINITY) {
+    wa = 1.f;
+    wb = 0.f;
+    nl = -INFINITY;
+    w = 0.f;
+  } else {
+    nl = m + __logf(__expf(a - m) + __expf(b - m));
+    wa = __expf(a - nl);
+    wb = __expf(b - nl);
+    w = wb;  // sigmoid(b - a) with the pre-merge lse
+  }
+  float* o = out + rowid * D + lane * E;
+  float x[E];
+  if constexpr (E == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(o);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  } else {
+    const float2 v = *reinterpret_cast<const float2*>(o);
+    x[0] = v.x; x[1] = v.y;
+  }
+  float y[E];
+  if (BF16_IN) {
+    const __nv_bfloat16* bo = reinterpret_cast<const __nv_bfloat16*>(block_out) + rowid * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) y[e] = __bfloat162float(bo[e]);
+  } else {
+    const float* bo = reinterpret_cast<const float*>(block_out) + rowid * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) y[e] = bo[e];
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = x[e] * wa + y[e] * wb;
+  if constexpr (E == 4) {
+    *reinterpret_cast<float4*>(o) = make_float4(x[0], x[1], x[2], x[3]);
+  } else {
+    *reinterpret_cast<float2*>(o) = make_float2(x[0], x[1]);
+  }
+  if (lane == 0) {
+    lse[li] = nl;
+    if (weight) weight[li] = w;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ dout,
+                                                    const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
+                                                    int64_t total, int heads) {
+  constexpr int E = D / 32;
+  const int64_t rowid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (rowid >= total * heads) return;
+  const __nv_bfloat16* a = dout + rowid * D + lane * E;
+  const __nv_bfloat16* b = out + rowid * D + lane * E;
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) s += __bfloat162float(a[e]) * __bfloat162float(b[e]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) {
+    const int64_t tok = rowid / heads;
+    const int h = (int)(rowid % heads);
+    delta[(int64_t)h * total + tok] = s;
+  }
+}
+
+__global__ void __launch_bounds__(256) convert_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
+                                                      int64_t n4, float mul) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = make_uint2(pack_bf16x2(v.x * mul, v.y * mul), pack_bf16x2(v.z * mul, v.w * mul));
+  }
+}
+
+}  // namespace
+
+int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
+                 float* weight_out, int64_t seqlen, int32_t heads, int32_t head_dim, cudaStream_t stream) {
+  const int64_t rows = seqlen * heads;
+  if (rows == 0) return 0;
+  const int64_t blocks = (rows + 7) / 8;
+  if (head_dim == 128) {
+    if (block_out_is_f32)
+      merge_kernel<128, false><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
+    else
+      merge_kernel<128, true><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
+  } else if (head_dim == 64) {
+    if (block_out_is_f32)
+      merge_kernel<64, false><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
+    else
+      merge_kernel<64, true><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
+  } else {
+    return (int)cudaErrorInvalidValue;
+  }
+  return (int)cudaGetLastError();
+}
+
+int launch_bwd_preprocess(const void* dout, const void* out, int64_t total, int32_t heads, int32_t head_dim,
+                          float* delta, float* dq_acc, cudaStream_t stream) {
+  const int64_t rows = total * heads;
+  if (rows == 0) return 0;
+  if (dq_acc) {
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)rows * head_dim * sizeof(float), stream);
+    if (e != cudaSuccess) return (int)e;
+  }
+  const int64_t blocks = (rows + 7) / 8;
+  auto d = reinterpret_cast<const __nv_bfloat16*>(dout);
+  auto o = reinterpret_cast<const __nv_bfloat16*>(out);
+  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, delta, total, heads);
+  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, delta, total, heads);
+  else return (int)cudaErrorInvalidValue;
+  return (int)cudaGetLastError();
+}
+
+int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream) {
+  if (n == 0) return 0;
+  const int64_t n4 = n / 4;  // n is a multiple of the head dim (64 or 128)
+  const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 148 * 16);
+  convert_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst), n4,
+                                             mul);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace cbv

@@ -1,0 +1,372 @@
+// Host planner (see plan.h).
+#include "plan.h"
+
+#include <algorithm>
+#include <cstdio>
+#include <map>
+#include <tuple>
+
+namespace cbv {
+
+namespace {
+
+int64_t sum_capped(int64_t a, int64_t b, int64_t window) {
+  // sum_{i=a}^{b-1} min(i + 1, window), window <= 0 meaning no cap
+  if (b <= a) return 0;
+  if (window <= 0) return (b * (b + 1) - a * (a + 1)) / 2;
+  int64_t s = 0;
+  int64_t lo = a, hi = std::min(b, window);  // i + 1 <= window  <=>  i < window
+  if (hi > lo) s += (hi * (hi + 1) - lo * (lo + 1)) / 2;
+  int64_t rest = b - std::max(a, window);
+  if (rest > 0) s += rest * window;
+  return s;
+}
+
+// visible (q, k) pairs between q positions [qp, qp+nq) and k positions [kp, kp+nk)
+int64_t visible_pairs(int64_t qp, int64_t nq, int64_t kp, int64_t nk, bool causal, int64_t window) {
+  int64_t total = 0;
+  for (int64_t i = 0; i < nq; ++i) {
+    int64_t q = qp + i;
+    int64_t lo = kp, hi = kp + nk - 1;
+    if (causal || window > 0) hi = std::min(hi, q);
+    if (window > 0) lo = std::max(lo, q - window + 1);
+    if (hi >= lo) total += hi - lo + 1;
+  }
+  return total;
+}
+
+int32_t weight(int64_t pairs) { return (int32_t)std::min<int64_t>(pairs / 256 + 1, INT32_MAX); }
+
+void sort_tasks(std::vector<TileTask>& t) {
+  std::stable_sort(t.begin(), t.end(), [](const TileTask& a, const TileTask& b) { return a.work > b.work; });
+}
+
+}  // namespace
+
+std::string check_cu_seqlens(const int32_t* cu, int32_t num_docs) {
+  if (num_docs < 0) return "num_docs must be >= 0";
+  if (cu == nullptr) return "cu_seqlens is NULL";
+  if (cu[0] != 0) return "cu_seqlens[0] must be 0";
+  for (int32_t d = 0; d < num_docs; ++d)
+    if (cu[d + 1] < cu[d]) return "cu_seqlens must be non-decreasing";
+  return "";
+}
+
+std::string check_divisible(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout) {
+  if (cp < 1) return "cp must be >= 1";
+  const int32_t n = layout == kZigZag ? 2 * cp : cp;
+  for (int32_t d = 0; d < num_docs; ++d)
+    if ((cu[d + 1] - cu[d]) % n) {
+      char buf[160];
+      snprintf(buf, sizeof buf, "document %d has length %d, not divisible by %d", d, cu[d + 1] - cu[d], n);
+      return buf;
+    }
+  return "";
+}
+
+void local_cu_seqlens(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t* out) {
+  for (int32_t d = 0; d <= num_docs; ++d) out[d] = cu[d] / cp;
+}
+
+void half_cu_seqlens(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t* out) {
+  for (int32_t d = 0; d <= num_docs; ++d) out[d] = cu[d] / (2 * cp);
+}
+
+int64_t get_half_index(const int32_t* cu_local, int32_t num_docs, bool front, int32_t* out) {
+  int64_t n = 0;
+  for (int32_t d = 0; d < num_docs; ++d) {
+    const int32_t a = cu_local[d], b = cu_local[d + 1], mid = a + (b - a) / 2;
+    const int32_t lo = front ? a : mid, hi = front ? mid : b;
+    for (int32_t i = lo; i < hi; ++i) {
+      if (out) out[n] = i;
+      ++n;
+    }
+  }
+  return n;
+}
+
+int64_t rank_tokens(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t rank, Layout layout, int32_t* out) {
+  int64_t n = 0;
+  auto emit = [&](int32_t a, int32_t b) {
+    for (int32_t i = a; i < b; ++i) {
+      if (out) out[n] = i;
+      ++n;
+    }
+  };
+  for (int32_t d = 0; d < num_docs; ++d) {
+    const int32_t g = cu[d], L = cu[d + 1] - cu[d];
+    if (layout == kZigZag) {
+      const int32_t c = L / (2 * cp);
+      emit(g + rank * c, g + (rank + 1) * c);
+      emit(g + (2 * cp - 1 - rank) * c, g + (2 * cp - rank) * c);
+    } else {
+      const int32_t c = L / cp;
+      emit(g + rank * c, g + (rank + 1) * c);
+    }
+  }
+  return n;
+}
+
+void rank_pair_counts(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int64_t* out) {
+  for (int32_t r = 0; r < cp; ++r) {
+    int64_t s = 0;
+    for (int32_t d = 0; d < num_docs; ++d) {
+      const int64_t L = cu[d + 1] - cu[d];
+      if (layout == kZigZag) {
+        const int64_t c = L / (2 * cp);
+        s += sum_capped(r * c, (r + 1) * c, window);
+        s += sum_capped((2 * cp - 1 - r) * c, (2 * cp - r) * c, window);
+      } else {
+        const int64_t c = L / cp;
+        s += sum_capped(r * c, (r + 1) * c, window);
+      }
+    }
+    out[r] = s;
+  }
+}
+
+void ring_step(int32_t rank, int32_t step, int32_t cp, Layout layout, int32_t* src, int32_t* kind) {
+  *src = ((rank - step) % cp + cp) % cp;
+  if (step == 0) {
+    *kind = kDiag;
+  } else if (layout == kZigZag) {
+    *kind = *src < rank ? kFrontK : kBackQ;
+  } else {
+    *kind = step <= rank ? kFull : kSkip;
+  }
+}
+
+std::vector<ChunkPair> ring_chunk_pairs(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout,
+                                        int32_t window, int32_t only_step) {
+  std::vector<ChunkPair> out;
+  for (int32_t r = 0; r < cp; ++r) {
+    for (int32_t s = 0; s < cp; ++s) {
+      if (only_step >= 0 && s != only_step) continue;
+      int32_t src, kind;
+      ring_step(r, s, cp, layout, &src, &kind);
+      if (kind == kSkip) continue;
+      for (int32_t d = 0; d < num_docs; ++d) {
+        const int32_t L = cu[d + 1] - cu[d];
+        const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+        const int32_t c = L / nchunk;
+        if (c == 0) continue;
+        std::vector<std::tuple<int32_t, int32_t, int32_t>> p;  // (q chunk, k chunk, causal)
+        if (layout == kZigZag) {
+          const int32_t f = r, b = 2 * cp - 1 - r, fs = src, bs = 2 * cp - 1 - src;
+          if (kind == kDiag) p = {{f, f, 1}, {b, f, 0}, {b, b, 1}};
+          else if (kind == kFrontK) p = {{f, fs, 0}, {b, fs, 0}};
+          else p = {{b, fs, 0}, {b, bs, 0}};
+        } else {
+          if (kind == kDiag) p = {{r, r, 1}};
+          else p = {{r, src, 0}};
+        }
+        for (auto& [x, y, causal] : p) {
+          // with a sliding window, drop chunk pairs that no query of x can see
+          if (window > 0 && x > y && (int64_t)(x - y - 1) * c + 1 >= window) continue;
+          out.push_back({d, r, s, x, y, causal});
+        }
+      }
+    }
+  }
+  return out;
+}
+
+Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t heads,
+                   int32_t only_step, int32_t tile_m) {
+  (void)heads;
+  Plan plan;
+  const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+  std::vector<ChunkPair> pairs = ring_chunk_pairs(cu, num_docs, cp, layout, window, only_step);
+  // group by (doc, q chunk), keeping ring order
+  std::map<std::pair<int32_t, int32_t>, std::vector<ChunkPair>> groups;
+  std::vector<std::pair<int32_t, int32_t>> order;
+  for (auto& p : pairs) {
+    auto key = std::make_pair(p.doc, p.q_chunk);
+    if (!groups.count(key)) order.push_back(key);
+    groups[key].push_back(p);
+  }
+  for (auto& key : order) {
+    const auto& g = groups[key];
+    const int32_t d = key.first, x = key.second;
+    const int32_t c = (cu[d + 1] - cu[d]) / nchunk;
+    const int32_t seg0 = (int32_t)plan.segs.size();
+    int32_t last_step = -1;
+    for (auto& p : g) {
+      Seg s;
+      s.row0 = cu[d] + p.k_chunk * c;
+      s.rows = c;
+      s.pos0 = s.row0;
+      s.flags = (p.causal ? kSegCausal : 0) | (p.step != last_step ? kSegBlockStart : 0);
+      last_step = p.step;
+      plan.segs.push_back(s);
+    }
+    const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    for (int32_t t0 = 0; t0 < c; t0 += tile_m) {
+      TileTask t{};
+      t.row0 = cu[d] + x * c + t0;
+      t.rows = std::min(tile_m, c - t0);
+      t.pos0 = t.row0;
+      t.seg0 = seg0;
+      t.nseg = nseg;
+      t.aux = -1;
+      int64_t w = 0;
+      for (int32_t i = 0; i < nseg; ++i) {
+        const Seg& s = plan.segs[seg0 + i];
+        w += visible_pairs(t.pos0, t.rows, s.pos0, s.rows, s.flags & kSegCausal, window);
+      }
+      t.work = weight(w);
+      plan.tasks.push_back(t);
+    }
+  }
+  sort_tasks(plan.tasks);
+  return plan;
+}
+
+Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t kv_heads,
+                   int32_t tile_n) {
+  (void)kv_heads;
+  Plan plan;
+  const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+  std::vector<ChunkPair> pairs = ring_chunk_pairs(cu, num_docs, cp, layout, window, -1);
+  std::map<std::pair<int32_t, int32_t>, std::vector<ChunkPair>> groups;
+  std::vector<std::pair<int32_t, int32_t>> order;
+  for (auto& p : pairs) {
+    auto key = std::make_pair(p.doc, p.k_chunk);
+    if (!groups.count(key)) order.push_back(key);
+    groups[key].push_back(p);
+  }
+  for (auto& key : order) {
+    const auto& g = groups[key];
+    const int32_t d = key.first, y = key.second;
+    const int32_t c = (cu[d + 1] - cu[d]) / nchunk;
+    const int32_t seg0 = (int32_t)plan.segs.size();
+    for (auto& p : g) {
+      Seg s;
+      s.row0 = cu[d] + p.q_chunk * c;
+      s.rows = c;
+      s.pos0 = s.row0;
+      s.flags = (p.causal ? kSegCausal : 0) | kSegBlockStart;
+      plan.segs.push_back(s);
+    }
+    const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    for (int32_t t0 = 0; t0 < c; t0 += tile_n) {
+      TileTask t{};
+      t.row0 = cu[d] + y * c + t0;
+      t.rows = std::min(tile_n, c - t0);
+      t.pos0 = t.row0;
+      t.seg0 = seg0;
+      t.nseg = nseg;
+      t.aux = -1;
+      int64_t w = 0;
+      for (int32_t i = 0; i < nseg; ++i) {
+        const Seg& s = plan.segs[seg0 + i];
+        w += visible_pairs(s.pos0, s.rows, t.pos0, t.rows, s.flags & kSegCausal, window);
+      }
+      t.work = weight(w);
+      plan.tasks.push_back(t);
+    }
+  }
+  sort_tasks(plan.tasks);
+  return plan;
+}
+
+Plan plan_block_fwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qbase, const int32_t* kbase,
+                    int32_t num_docs, bool causal, int32_t window, int32_t heads, int32_t tile_m) {
+  (void)heads;
+  Plan plan;
+  for (int32_t d = 0; d < num_docs; ++d) {
+    const int32_t lq = cu_q[d + 1] - cu_q[d], lk = cu_k[d + 1] - cu_k[d];
+    if (lq == 0) continue;
+    const int32_t qb = qbase ? qbase[d] : lk - lq;
+    const int32_t kb = kbase ? kbase[d] : 0;
+    const int32_t seg0 = (int32_t)plan.segs.size();
+    if (lk > 0) plan.segs.push_back(Seg{cu_k[d], lk, kb, (causal ? kSegCausal : 0) | kSegBlockStart});
+    const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    for (int32_t t0 = 0; t0 < lq; t0 += tile_m) {
+      TileTask t{};
+      t.row0 = cu_q[d] + t0;
+      t.rows = std::min(tile_m, lq - t0);
+      t.pos0 = qb + t0;
+      t.seg0 = seg0;
+      t.nseg = nseg;
+      t.aux = -1;
+      t.work = nseg ? weight(visible_pairs(t.pos0, t.rows, kb, lk, causal, window)) : 0;
+      plan.tasks.push_back(t);
+    }
+  }
+  sort_tasks(plan.tasks);
+  return plan;
+}
+
+Plan plan_block_bwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qbase, const int32_t* kbase,
+                    int32_t num_docs, bool causal, int32_t window, int32_t kv_heads, int32_t tile_n) {
+  (void)kv_heads;
+  Plan plan;
+  for (int32_t d = 0; d < num_docs; ++d) {
+    const int32_t lq = cu_q[d + 1] - cu_q[d], lk = cu_k[d + 1] - cu_k[d];
+    if (lk == 0) continue;
+    const int32_t qb = qbase ? qbase[d] : lk - lq;
+    const int32_t kb = kbase ? kbase[d] : 0;
+    const int32_t seg0 = (int32_t)plan.segs.size();
+    if (lq > 0) plan.segs.push_back(Seg{cu_q[d], lq, qb, (causal ? kSegCausal : 0) | kSegBlockStart});
+    const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    for (int32_t t0 = 0; t0 < lk; t0 += tile_n) {
+      TileTask t{};
+      t.row0 = cu_k[d] + t0;
+      t.rows = std::min(tile_n, lk - t0);
+      t.pos0 = kb + t0;
+      t.seg0 = seg0;
+      t.nseg = nseg;
+      t.aux = -1;
+      t.work = nseg ? weight(visible_pairs(qb, lq, t.pos0, t.rows, causal, window)) : 0;
+      plan.tasks.push_back(t);
+    }
+  }
+  sort_tasks(plan.tasks);
+  return plan;
+}
+
+Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int32_t seg_size, KvMode mode,
+              int32_t block_size, int32_t global_q_offset, int32_t window, bool per_shard, int32_t tile_m) {
+  (void)heads;
+  Plan plan;
+  const int64_t q_lo = global_q_offset, q_hi = (int64_t)global_q_offset + q_len - 1;
+  std::vector<int32_t> shard_seg0(shards), shard_nseg(shards);
+  for (int32_t r = 0; r < shards; ++r) {
+    shard_seg0[r] = (int32_t)plan.segs.size();
+    bool first = true;
+    for (int32_t s0 = 0; s0 < n_local; s0 += seg_size) {
+      const int32_t rows = std::min(seg_size, n_local - s0);
+      const int64_t kmin = kvp_position(r, s0, n_local, block_size, shards, mode);
+      const int64_t kmax = kvp_position(r, s0 + rows - 1, n_local, block_size, shards, mode);
+      // drop segments no query can see (causal: kmin > last q; window: kmax too old for the first q)
+      if (kmin > q_hi) continue;
+      if (window > 0 && q_lo - kmax >= window && q_hi - kmax >= window) continue;
+      plan.segs.push_back(Seg{s0, rows, 0, kSegCausal | (first ? kSegBlockStart : 0) | (r << kSegShardShift)});
+      first = false;
+    }
+    shard_nseg[r] = (int32_t)plan.segs.size() - shard_seg0[r];
+  }
+  for (int32_t t0 = 0; t0 < q_len; t0 += tile_m) {
+    const int32_t rows = std::min(tile_m, q_len - t0);
+    const int32_t pos0 = global_q_offset + t0;
+    for (int32_t r = 0; r < (per_shard ? shards : 1); ++r) {
+      TileTask t{};
+      t.row0 = t0;
+      t.rows = rows;
+      t.pos0 = pos0;
+      t.seg0 = per_shard ? shard_seg0[r] : 0;
+      t.nseg = per_shard ? shard_nseg[r] : (int32_t)plan.segs.size();
+      t.aux = per_shard ? r : -1;
+      // weight: visible keys of the tile (every key position below the tile is one page of some shard)
+      int64_t lo = window > 0 ? std::max<int64_t>(0, pos0 - window + 1) : 0;
+      int64_t span = (int64_t)pos0 + rows - lo;
+      t.work = weight((int64_t)rows * span / (per_shard ? shards : 1));
+      plan.tasks.push_back(t);
+    }
+  }
+  sort_tasks(plan.tasks);
+  return plan;
+}
+
+}  // namespace cbv

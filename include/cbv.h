@@ -1,0 +1,321 @@
+/*
+ * cbv.h - blockwise causal varlen attention on B200 (sm_100a): the C ABI of libcbv.so.
+ *
+ * What the library computes (sources are named by page title and section):
+ *   - NeMo AutoModel API, eagle.zigzag_ring_attention: zig-zag context parallelism
+ *     (module docstring), get_half_index / get_half_lse, _block_forward /
+ *     _block_backward, update_out_and_lse, zigzag_ring_flash_attn_varlen_forward /
+ *     _backward (the merged-lse backward);
+ *   - NeMo AutoModel API, eagle.ring_attention: the contiguous ring (module
+ *     docstring, ring_flash_attn_forward: step <= rank, causal only at step 0),
+ *     _update_out_and_lse (sigmoid-form merge), _fa_forward's (out, lse) contract;
+ *   - NKI library API, attention_kv_parallel_segmented_cte: KV-parallel segmented
+ *     prefill over a paged KV cache, contiguous or round-robin shards, sliding window;
+ *   - qsa_fa_fallback.py (SM121 recipe): one-query-per-sequence GQA varlen decode.
+ *
+ * Conventions shared by every call:
+ *   - Tensors are plain pointers.  "device" pointers are CUDA global memory of the
+ *     current device; "host" pointers are ordinary CPU memory read during the call
+ *     and not retained.  The caller owns all memory; the library allocates nothing
+ *     and keeps no state between calls.  Scratch memory comes from a caller-owned
+ *     device `workspace` whose size the matching *_workspace_size() call reports.
+ *   - bf16 means IEEE bfloat16 (torch.bfloat16); token-major layouts are
+ *     [tokens, heads, head_dim], contiguous.  lse is float32 [heads, tokens],
+ *     natural log.  head_dim is 64 or 128.
+ *   - Masks use positions.  In the ring and prefill calls a token's position is its
+ *     global row in natural packed order (prefill: global_q_offset + i for q).  A key
+ *     is visible when it is in the query's document and, if causal, kpos <= qpos;
+ *     with window = W > 0 also qpos - kpos < W (W keys including the query itself;
+ *     the NKI sliding_window integer, 0 = disabled).
+ *   - A query with no visible key gets out = 0 and lse = -inf.
+ *   - scale <= 0 selects head_dim^-0.5.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) unless stated otherwise, and returns CBV_OK (0) or a negative
+ *     cbv_status; cbv_last_error_message() then describes the failure.  Argument
+ *     errors are detected on the host before anything is launched.
+ *   - Kernels never wait without a bound: a stalled pipeline records a code in the
+ *     workspace status word and exits; cbv_read_status() returns CBV_ERR_TIMEOUT.
+ *   - Argument structs start with struct_size and abi_version so that fields are
+ *     never bound by position (the lesson of ring_attention's
+ *     require_flash_attn_version); a mismatch returns CBV_ERR_VERSION.
+ */
+#ifndef CBV_H
+#define CBV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CBV_ABI_VERSION 1
+
+typedef enum cbv_status {
+  CBV_OK = 0,
+  CBV_ERR_BAD_ARG = -1,
+  CBV_ERR_BAD_SHAPE = -2,
+  CBV_ERR_BAD_DTYPE = -3,
+  CBV_ERR_MISALIGNED = -4,
+  CBV_ERR_UNSUPPORTED_HEAD_DIM = -5,
+  CBV_ERR_NOT_DIVISIBLE_2CP = -6,
+  CBV_ERR_NOT_CAUSAL = -7,
+  CBV_ERR_GQA_MISMATCH = -8,
+  CBV_ERR_BAD_CU_SEQLENS = -9,
+  CBV_ERR_Q_LEN_NOT_ONE = -10,
+  CBV_ERR_WORKSPACE_TOO_SMALL = -11,
+  CBV_ERR_TIMEOUT = -12,
+  CBV_ERR_CUDA = -13,
+  CBV_ERR_VERSION = -14
+} cbv_status;
+
+typedef enum cbv_layout { CBV_LAYOUT_ZIGZAG = 0, CBV_LAYOUT_CONTIGUOUS = 1 } cbv_layout;
+typedef enum cbv_kv_mode { CBV_KV_CONTIGUOUS = 0, CBV_KV_ROUND_ROBIN = 1 } cbv_kv_mode;
+typedef enum cbv_dtype { CBV_DTYPE_BF16 = 0, CBV_DTYPE_F32 = 1 } cbv_dtype;
+typedef enum cbv_schedule {
+  /* one launch: each q tile visits every ring step's k/v block in ring order and
+     merges the block results on chip (log-sum-exp identity on the accumulator) */
+  CBV_SCHEDULE_FUSED = 0,
+  /* one launch per ring step; each launch merges its block into an fp32 running
+     (out, lse) pair in the workspace inside the kernel epilogue */
+  CBV_SCHEDULE_STEPWISE = 1
+} cbv_schedule;
+
+/* Text of the last error on this thread ("" if none).  Valid until the next call. */
+const char* cbv_last_error_message(void);
+int cbv_abi_version(void);
+
+/* Reads the device status word at the start of `workspace` (synchronises `stream`).
+   *status_out receives the raw kernel code (0 = ok).  Returns CBV_ERR_TIMEOUT if a
+   kernel gave up a wait, CBV_OK otherwise. */
+int cbv_read_status(const void* workspace, int* status_out, void* stream);
+
+/* ========================================================================= planner (host only)
+ * Integer, exact; all arrays are host memory.  cu_seqlens is GLOBAL, int32 [num_docs+1],
+ * natural packed order.  NeMo AutoModel zigzag_ring_attention: module docstring
+ * (2*cp chunks, rank r owns chunks r and 2cp-1-r), get_half_index, get_half_lse,
+ * _block_forward (halved cu_seqlens).  Errors: CBV_ERR_BAD_CU_SEQLENS (not starting
+ * at 0 or decreasing), CBV_ERR_NOT_DIVISIBLE_2CP, CBV_ERR_BAD_ARG. */
+
+/* out[d] = cu_global[d] / cp, int32 [num_docs+1]: every virtual rank's local cu_seqlens. */
+int cbv_local_cu_seqlens(const int32_t* cu_global, int32_t num_docs, int32_t cp, int32_t layout, int32_t* out);
+/* out[d] = cu_global[d] / (2 cp): cu_seqlens of the front or back halves (zig-zag only). */
+int cbv_half_cu_seqlens(const int32_t* cu_global, int32_t num_docs, int32_t cp, int32_t* out);
+/* Ascending local positions of the front (front != 0) or back half of every local
+   document, int32 [cu_local[num_docs] / 2]; *count_out receives the length. */
+int cbv_get_half_index(const int32_t* cu_local, int32_t num_docs, int32_t front, int32_t* idx_out,
+                       int64_t* count_out);
+/* Front or back half of a host float32 lse [num_heads, seqlen] (seqlen = cu_local[num_docs]),
+   per local document: out [num_heads, seqlen / 2]. */
+int cbv_get_half_lse(const float* lse, int32_t num_heads, const int32_t* cu_local, int32_t num_docs, int32_t front,
+                     float* out);
+/* Global rows of virtual rank `rank`'s tokens in local order, int32 [S / cp]. */
+int cbv_rank_tokens(const int32_t* cu_global, int32_t num_docs, int32_t cp, int32_t rank, int32_t layout,
+                    int32_t* out);
+/* Visible causal (q, k) pairs per virtual rank (the work each rank does), int64 [cp]. */
+int cbv_rank_pair_counts(const int32_t* cu_global, int32_t num_docs, int32_t cp, int32_t layout, int32_t window,
+                         int64_t* counts_out);
+/* Ring step schedule: the rank whose k/v reach `rank` at `step` (src = (rank-step) mod cp)
+   and the block kind: 0 diag (local q x local k, causal), 1 front-k (all local q x src's
+   front halves), 2 back-q (local back halves x all of src's k), 3 full (contiguous,
+   step <= rank), 4 skip (contiguous, step > rank). */
+int cbv_ring_step(int32_t rank, int32_t step, int32_t cp, int32_t layout, int32_t* src_out, int32_t* kind_out);
+
+/* ========================================================================= block forward
+ * One flash varlen block (zigzag_ring_attention._block_forward; ring_attention._fa_forward:
+ * returns (out[B,S,H,D], lse[B,H,S])).  Documents pair q rows [cu_q[d], cu_q[d+1]) with k
+ * rows [cu_k[d], cu_k[d+1]).  Positions: qpos = q_pos_base[d] + (i - cu_q[d]),
+ * kpos = k_pos_base[d] + (j - cu_k[d]); NULL bases mean k_pos_base = 0 and
+ * q_pos_base = L_k - L_q (bottom-right alignment).
+ * merge = 0: writes out (bf16 or f32, out_dtype) and lse.
+ * merge = 1: out must be f32; (out, lse) hold a running pair that is merged in place with
+ *            this block by the online-softmax identity (update_out_and_lse) in the kernel
+ *            epilogue.  Rows of the running pair outside this block are untouched. */
+typedef struct cbv_block_fwd_args {
+  uint32_t struct_size; /* sizeof(cbv_block_fwd_args) */
+  uint32_t abi_version; /* CBV_ABI_VERSION */
+  const void* q;        /* device bf16 [total_q, num_heads, head_dim] */
+  const void* k;        /* device bf16 [total_k, num_kv_heads, head_dim] */
+  const void* v;        /* device bf16 [total_k, num_kv_heads, head_dim] */
+  int64_t total_q, total_k;
+  int32_t num_heads, num_kv_heads, head_dim;
+  int32_t num_docs;
+  const int32_t* cu_seqlens_q; /* host int32 [num_docs+1] */
+  const int32_t* cu_seqlens_k; /* host int32 [num_docs+1] */
+  const int32_t* q_pos_base;   /* host int32 [num_docs] or NULL */
+  const int32_t* k_pos_base;   /* host int32 [num_docs] or NULL */
+  int32_t max_seqlen;          /* 0 or >= every document length (checked) */
+  float scale;
+  int32_t causal;
+  int32_t window;
+  int32_t merge;
+  int32_t out_dtype;           /* cbv_dtype of out when merge = 0 */
+  void* out;                   /* device [total_q, num_heads, head_dim] */
+  float* lse;                  /* device f32 [num_heads, total_q] */
+  void* workspace;             /* device, >= cbv_block_fwd_workspace_size() bytes, 256-byte aligned */
+  size_t workspace_bytes;
+} cbv_block_fwd_args;
+size_t cbv_block_fwd_workspace_size(const cbv_block_fwd_args* a);
+int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream);
+
+/* ========================================================================= merge
+ * In place: (out, lse) <- update_out_and_lse(out, lse, block_out, block_lse)
+ * (zigzag_ring_attention.update_out_and_lse; ring_attention._update_out_and_lse).
+ * out: device f32 [seqlen, num_heads, head_dim]; lse, block_lse: device f32 [num_heads, seqlen];
+ * block_out: device [seqlen, num_heads, head_dim] of block_out_dtype (bf16 or f32);
+ * weight_out: device f32 [num_heads, seqlen] or NULL, receives sigmoid(block_lse - lse)
+ * computed with the running lse before the merge.  A side at -inf is the identity. */
+int cbv_attn_merge(float* out, float* lse, const void* block_out, int32_t block_out_dtype, const float* block_lse,
+                   float* weight_out, int64_t seqlen, int32_t num_heads, int32_t head_dim, void* stream);
+
+/* ========================================================================= ring forward / backward
+ * Causal varlen attention of the whole packed batch computed the ring way
+ * (zigzag_ring_flash_attn_varlen_forward / _backward; ring_flash_attn_forward /
+ * _backward for layout = CBV_LAYOUT_CONTIGUOUS): the batch is split over cp VIRTUAL
+ * ranks on this GPU (zig-zag: rank r owns chunks r and 2cp-1-r of every document;
+ * contiguous: the r-th of cp pieces of every document); at step s rank r attends to the
+ * k/v of src = (r-s) mod cp with the block schedule of cbv_ring_step, and the block
+ * results are merged with the log-sum-exp identity.  There is no communication: the
+ * virtual ranks are address ranges in HBM.  q, k, v, out, dout, dq, dk, dv are in natural
+ * packed order; lse is [num_heads, total].
+ * Backward: every block is fed the MERGED out and lse (the merged-lse identity), dk/dv of
+ * a key tile accumulate across all blocks that see it, dq accumulates in fp32.
+ * Errors: causal = 0 -> CBV_ERR_NOT_CAUSAL (zig-zag is meaningless otherwise); a document
+ * length not divisible by 2cp (zig-zag) or cp (contiguous) -> CBV_ERR_NOT_DIVISIBLE_2CP. */
+typedef struct cbv_ring_args {
+  uint32_t struct_size; /* sizeof(cbv_ring_args) */
+  uint32_t abi_version; /* CBV_ABI_VERSION */
+  const void* q;        /* device bf16 [total, num_heads, head_dim] */
+  const void* k;        /* device bf16 [total, num_kv_heads, head_dim] */
+  const void* v;
+  int64_t total;
+  int32_t num_heads, num_kv_heads, head_dim;
+  int32_t num_docs;
+  const int32_t* cu_seqlens; /* host int32 [num_docs+1], GLOBAL */
+  int32_t max_seqlen;        /* 0 or >= every document length */
+  int32_t cp;                /* virtual ranks, >= 1 */
+  int32_t layout;            /* cbv_layout */
+  float scale;
+  int32_t causal;            /* must be 1 */
+  int32_t window;
+  int32_t schedule;          /* cbv_schedule (forward only) */
+  void* out;                 /* device bf16 [total, num_heads, head_dim]: forward output, backward input */
+  float* lse;                /* device f32 [num_heads, total]: forward output, backward input (merged) */
+  const void* dout;          /* backward: device bf16 [total, num_heads, head_dim] */
+  void* dq;                  /* backward: device bf16 outputs */
+  void* dk;
+  void* dv;
+  void* workspace;
+  size_t workspace_bytes;
+} cbv_ring_args;
+size_t cbv_zigzag_ring_fwd_workspace_size(const cbv_ring_args* a);
+int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream);
+size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a);
+int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream);
+
+/* ========================================================================= block backward
+ * One block's backward fed the MERGED softmax statistics (zigzag_ring_attention._block_backward;
+ * ulysses_attention._block0_backward): with P = exp(scale q k^T - lse) over the block's visible
+ * pairs, dV += P^T dO, dS = P (dO V^T - Delta), Delta = rowsum(dO * out), dQ += scale dS K,
+ * dK += scale dS^T Q.  dq_acc, dk_acc, dv_acc are device f32 accumulators that are ADDED
+ * to (token-major, like q and k).  Documents and positions as in cbv_attn_block_fwd. */
+typedef struct cbv_block_bwd_args {
+  uint32_t struct_size;
+  uint32_t abi_version;
+  const void* dout;    /* device bf16 [total_q, num_heads, head_dim] */
+  const void* q;       /* device bf16 [total_q, num_heads, head_dim] */
+  const void* k;       /* device bf16 [total_k, num_kv_heads, head_dim] */
+  const void* v;
+  const void* out;     /* device bf16 [total_q, num_heads, head_dim], the MERGED output */
+  const float* lse;    /* device f32 [num_heads, total_q], the MERGED lse */
+  int64_t total_q, total_k;
+  int32_t num_heads, num_kv_heads, head_dim;
+  int32_t num_docs;
+  const int32_t* cu_seqlens_q;  /* host */
+  const int32_t* cu_seqlens_k;  /* host */
+  const int32_t* q_pos_base;    /* host or NULL */
+  const int32_t* k_pos_base;    /* host or NULL */
+  float scale;
+  int32_t causal;
+  int32_t window;
+  float* dq_acc;       /* device f32 [total_q, num_heads, head_dim], += */
+  float* dk_acc;       /* device f32 [total_k, num_kv_heads, head_dim], += */
+  float* dv_acc;
+  void* workspace;
+  size_t workspace_bytes;
+} cbv_block_bwd_args;
+size_t cbv_block_bwd_workspace_size(const cbv_block_bwd_args* a);
+int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream);
+
+/* ========================================================================= paged KV-parallel prefill
+ * NKI attention_kv_parallel_segmented_cte: q token i (position global_q_offset + i) attends
+ * causally (plus optional sliding window) to the whole context, which is spread over
+ * `shards` KV shards of a paged cache.  Shard r reads its local tokens through row r of
+ * block_tables; local token t sits at global position r * n_local + t (CBV_KV_CONTIGUOUS,
+ * n_local = blocks_per_shard * block_size) or ((t / bs) * shards + r) * bs + t % bs
+ * (CBV_KV_ROUND_ROBIN: shard r holds global blocks r, r + shards, ...).  Every shard's KV
+ * is walked in segments of seg_size tokens and the partial results are merged by online
+ * softmax: across segments and shards on chip in one launch (shard_out == NULL), or per
+ * shard into shard_out / shard_lse for a later cbv_attn_merge (shard_out != NULL).
+ * GQA: q head h reads kv head h / (num_heads / num_kv_heads).
+ * Requirements: block_size divides 128 and is >= 8; seg_size is a multiple of 128. */
+typedef struct cbv_kvp_args {
+  uint32_t struct_size;
+  uint32_t abi_version;
+  const void* q;              /* device bf16, element (h, i, d) at q[h*q_stride_head + i*q_stride_token + d] */
+  int64_t q_stride_head, q_stride_token;  /* elements; [HQ, S, D] contiguous: S*D and D */
+  int32_t q_len, num_heads, num_kv_heads, head_dim;
+  const void* k_cache;        /* device bf16 [num_blocks, num_kv_heads, block_size, head_dim] */
+  const void* v_cache;
+  int32_t num_blocks, block_size;
+  const int32_t* block_tables; /* device int32 [shards, blocks_per_shard] of page ids */
+  int32_t shards, blocks_per_shard;
+  int32_t kv_mode;            /* cbv_kv_mode */
+  int32_t seg_size;
+  float scale;
+  int32_t global_q_offset;
+  int32_t sliding_window;     /* 0 = disabled */
+  void* out;                  /* device bf16 [num_heads, q_len, head_dim] (merged result) */
+  float* lse;                 /* device f32 [num_heads, q_len] or NULL */
+  float* shard_out;           /* NULL, or device f32 [shards, num_heads, q_len, head_dim] per-shard partials */
+  float* shard_lse;           /* with shard_out: device f32 [shards, num_heads, q_len] */
+  void* workspace;
+  size_t workspace_bytes;
+} cbv_kvp_args;
+size_t cbv_kvp_workspace_size(const cbv_kvp_args* a);
+int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream);
+
+/* ========================================================================= varlen decode
+ * qsa_fa_fallback.py, triton_varlen_attn_func: sequence s has exactly one query row
+ * cu_seqlens_q[s] and keys [cu_seqlens_k[s], cu_seqlens_k[s+1]); q head h reads kv head
+ * h / (num_heads / num_kv_heads); no mask; an empty key range writes zeros.  The offsets
+ * are DEVICE arrays read by the kernel, so their contents may change between CUDA-graph
+ * replays.  validate != 0 copies cu_seqlens_q to the host (synchronising the stream) and
+ * returns CBV_ERR_Q_LEN_NOT_ONE unless every sequence has one query row; pass 0 while
+ * capturing a graph.  The output row of sequence s is cu_seqlens_q[s].
+ * Requirements: num_heads / num_kv_heads <= 16. */
+typedef struct cbv_decode_args {
+  uint32_t struct_size;
+  uint32_t abi_version;
+  const void* q;              /* device bf16 [total_q, num_heads, head_dim] */
+  const void* k;              /* device bf16 [total_k, num_kv_heads, head_dim] */
+  const void* v;
+  void* out;                  /* device bf16 [total_q, num_heads, head_dim] */
+  const int32_t* cu_seqlens_q; /* device int32 [num_seqs+1] */
+  const int32_t* cu_seqlens_k; /* device int32 [num_seqs+1] */
+  int32_t num_seqs;
+  int64_t total_q, total_k;
+  int32_t num_heads, num_kv_heads, head_dim;
+  float scale;
+  int32_t validate;
+  void* workspace;            /* device, >= cbv_decode_workspace_size() bytes (status word) */
+  size_t workspace_bytes;
+} cbv_decode_args;
+size_t cbv_decode_workspace_size(const cbv_decode_args* a);
+int cbv_varlen_decode(const cbv_decode_args* a, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CBV_H */

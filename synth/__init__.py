@@ -101,3 +101,22 @@ def to_torch_bf16(x: np.ndarray, device="cpu"):
     bits = bf16_bits(np.asarray(x, dtype=np.float32))
     t = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
     return t.to(device)
+
+
+def torch_normal_bf16(shape, seed: int, device="cuda"):
+    """Standard normal float32 draws from torch's generator on ``device``, rounded to bfloat16.
+
+    For full-size workloads that are too large to draw on the host; tests that
+    check such inputs copy the rows they need back to the host.
+    """
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    step = 1 << 28
+    for i in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - i)
+        flat[i:i + n] = torch.randn(n, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return out

@@ -1,0 +1,170 @@
+"""The C ABI without a GPU: library loads, exports every declared symbol, struct
+layouts agree with a C compiler, the C++ planner matches the oracle planner bit for
+bit, and argument errors come back as status codes before any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+
+import context_blockwise_causal_varlen_b200 as cbv
+from oracle import planner as P
+from synth import cu_from_lengths, packed_doc_lengths, streams
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cbv.h")
+
+pytestmark = pytest.mark.skipif(not os.path.exists(cbv.LIB_PATH), reason="libcbv.so not built")
+
+
+def test_library_exports_every_declared_symbol():
+    names = set(re.findall(r"^(?:int|size_t|const char\*)\s+(cbv_\w+)\s*\(", open(HEADER).read(), re.M))
+    assert len(names) >= 20
+    L = cbv.lib()
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert set(cbv.EXPORTS) == names
+
+
+def test_struct_layouts_match_the_c_compiler():
+    structs = {"cbv_block_fwd_args": cbv.BlockFwdArgs, "cbv_ring_args": cbv.RingArgs,
+               "cbv_block_bwd_args": cbv.BlockBwdArgs, "cbv_kvp_args": cbv.KvpArgs, "cbv_decode_args": cbv.DecodeArgs}
+    src = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
+    for cname, st in structs.items():
+        src.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in st._fields_:
+            src.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    src.append("return 0;}")
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "l.c")
+        exe = os.path.join(d, "l")
+        open(c, "w").write("\n".join(src))
+        subprocess.run(["gcc", "-o", exe, c], check=True)
+        lines = subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n")
+    got = dict(line.split() for line in lines if line)
+    for cname, st in structs.items():
+        assert int(got[cname]) == ctypes.sizeof(st), cname
+        for f, _ in st._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(st, f).offset, f"{cname}.{f}"
+
+
+CUS = [[0, 96, 256], [0, 64], [0, 24, 32, 72], [0, 48, 144, 160], [0, 8, 8, 40]]
+
+
+@pytest.mark.parametrize("cu", CUS)
+@pytest.mark.parametrize("cp", [1, 2, 4])
+def test_planner_matches_oracle(cu, cp):
+    cu = np.array(cu)
+    for layout, name in ((cbv.ZIGZAG, P.ZIGZAG), (cbv.CONTIGUOUS, P.CONTIGUOUS)):
+        div = 2 * cp if layout == cbv.ZIGZAG else cp
+        if np.any(np.diff(cu) % div):
+            with pytest.raises(cbv.CbvError) as e:
+                cbv.local_cu_seqlens(cu, cp, layout)
+            assert e.value.status == "NOT_DIVISIBLE_2CP"
+            continue
+        assert np.array_equal(cbv.local_cu_seqlens(cu, cp, layout), P.local_cu_seqlens(cu, cp))
+        for r in range(cp):
+            assert np.array_equal(cbv.rank_tokens(cu, cp, r, layout), P.rank_tokens(cu, cp, r, name))
+        for w in (0, 5, 33):
+            assert np.array_equal(cbv.rank_pair_counts(cu, cp, layout, w), P.rank_pair_counts(cu, cp, name, w))
+        if layout == cbv.ZIGZAG:
+            assert np.array_equal(cbv.half_cu_seqlens(cu, cp), P.half_cu_seqlens(cu, cp))
+            cl = P.local_cu_seqlens(cu, cp)
+            for front in (True, False):
+                assert np.array_equal(cbv.get_half_index(cl, front), P.get_half_index(cl, front))
+                lse = np.random.default_rng(0).standard_normal((3, int(cl[-1]))).astype(np.float32)
+                assert np.array_equal(cbv.get_half_lse(lse, cl, front), P.get_half_lse(lse, cl, front))
+        for r in range(cp):
+            for s in range(cp):
+                src, kind = cbv.ring_step(r, s, cp, layout)
+                osrc, okind = (P.zigzag_step if layout == cbv.ZIGZAG else P.contiguous_step)(r, s, cp)
+                names = {0: "diag", 1: "front_k", 2: "back_q", 3: "full", 4: "skip"}
+                assert (src, names[kind]) == (osrc, okind)
+
+
+def test_planner_on_the_packed_workload_and_long_doc():
+    for seed in range(5):
+        cu = cu_from_lengths(packed_doc_lengths(streams(seed, 6)[4], 16384, 512, 4096, 8))
+        for layout, name in ((cbv.ZIGZAG, P.ZIGZAG), (cbv.CONTIGUOUS, P.CONTIGUOUS)):
+            assert np.array_equal(cbv.rank_pair_counts(cu, 4, layout), P.rank_pair_counts(cu, 4, name))
+        zz = cbv.rank_pair_counts(cu, 4, cbv.ZIGZAG)
+        per_doc_equal = True
+        for d in range(len(cu) - 1):
+            one = cbv.rank_pair_counts(cu[d:d + 2] - cu[d], 4, cbv.ZIGZAG)
+            per_doc_equal &= bool(np.all(one == one[0]))
+        assert per_doc_equal and np.all(zz == zz[0])
+    cu = np.array([0, 65536])
+    assert np.all(cbv.rank_pair_counts(cu, 8, cbv.ZIGZAG) == 268439552)
+    ct = cbv.rank_pair_counts(cu, 8, cbv.CONTIGUOUS)
+    assert ct[0] == 33558528 and ct[-1] == 503320576
+    w = cbv.rank_pair_counts(cu, 8, cbv.ZIGZAG, 4096)
+    assert w.sum() == 260048896 == P.rank_pair_counts(cu, 8, P.ZIGZAG, 4096).sum()
+
+
+def _ring_args(**kw):
+    cu = kw.pop("cu", np.array([0, 96, 256], np.int32))
+    a = cbv.RingArgs(struct_size=ctypes.sizeof(cbv.RingArgs), abi_version=cbv.ABI_VERSION, total=int(cu[-1]),
+                     num_heads=2, num_kv_heads=2, head_dim=64, num_docs=len(cu) - 1,
+                     cu_seqlens=cu.ctypes.data_as(cbv.c_i32p), cp=2, causal=1)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, cu
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("causal", 0, "NOT_CAUSAL"),
+    ("head_dim", 96, "UNSUPPORTED_HEAD_DIM"),
+    ("num_kv_heads", 3, "GQA_MISMATCH"),
+    ("cp", 0, "BAD_ARG"),
+    ("cp", 5, "NOT_DIVISIBLE_2CP"),
+    ("abi_version", 7, "VERSION"),
+    ("struct_size", 8, "VERSION"),
+    ("total", 300, "BAD_CU_SEQLENS"),
+    ("max_seqlen", 100, "BAD_ARG"),
+    ("schedule", 9, "BAD_ARG"),
+])
+def test_ring_argument_errors_are_reported_before_any_launch(field, value, status):
+    a, cu = _ring_args(**{field: value})
+    rc = cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None)
+    assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
+    assert cbv.lib().cbv_last_error_message()
+    assert cbv.lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a)) == 0
+
+
+def test_bad_cu_seqlens_rejected():
+    a, cu = _ring_args(cu=np.array([0, 100, 96, 256], np.int32))
+    assert cbv.STATUS[cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None)] == "BAD_CU_SEQLENS"
+    a, cu = _ring_args(cu=np.array([4, 96, 256], np.int32))
+    assert cbv.STATUS[cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None)] == "BAD_CU_SEQLENS"
+
+
+def test_workspace_sizes_are_reported():
+    a, cu = _ring_args()
+    n_fwd = cbv.lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a))
+    assert n_fwd >= 256 and n_fwd % 256 == 0
+    a.schedule = cbv.SCHEDULE_STEPWISE
+    assert cbv.lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a)) >= 256 * 2 * 64 * 4
+    n_bwd = cbv.lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(a))
+    assert n_bwd >= 256 * 2 * 64 * 4 + 2 * 256 * 4
+
+
+def test_decode_rejects_bad_gqa_and_head_dim():
+    a = cbv.DecodeArgs(struct_size=ctypes.sizeof(cbv.DecodeArgs), abi_version=cbv.ABI_VERSION, num_seqs=1, total_q=1,
+                       total_k=1, num_heads=32, num_kv_heads=1, head_dim=128)
+    assert cbv.STATUS[cbv.lib().cbv_varlen_decode(ctypes.byref(a), None)] == "GQA_MISMATCH"
+    a.num_kv_heads, a.num_heads = 4, 30
+    assert cbv.STATUS[cbv.lib().cbv_varlen_decode(ctypes.byref(a), None)] == "GQA_MISMATCH"
+    a.num_heads, a.head_dim = 32, 80
+    assert cbv.STATUS[cbv.lib().cbv_varlen_decode(ctypes.byref(a), None)] == "UNSUPPORTED_HEAD_DIM"
+
+
+def test_kvp_rejects_bad_block_and_segment_sizes():
+    a = cbv.KvpArgs(struct_size=ctypes.sizeof(cbv.KvpArgs), abi_version=cbv.ABI_VERSION, q_len=16, num_heads=4,
+                    num_kv_heads=2, head_dim=128, num_blocks=8, block_size=24, shards=2, blocks_per_shard=4,
+                    seg_size=512)
+    assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"
+    a.block_size, a.seg_size = 32, 100
+    assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"

@@ -1,0 +1,103 @@
+"""Paged KV-parallel prefill and varlen decode on the GPU against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import context_blockwise_causal_varlen_b200 as cbv
+from oracle import decode as DEC
+from oracle import paged as PG
+from synth import block_permutation, cu_from_lengths, streams
+from tests.gpu_util import check_lse, check_out, dev, f64, gen, host, sync
+
+pytestmark = pytest.mark.gpu
+
+
+def _paged(seed, R, bps, bs, hq, hkv, D, S):
+    nb = R * bps
+    q, kc, vc = gen(seed, (hq, S, D), (nb, hkv, bs, D), (nb, hkv, bs, D))
+    perm = block_permutation(streams(seed + 100, 1)[0], nb)
+    return q, kc, vc, perm
+
+
+@pytest.mark.parametrize("mode", [PG.ROUND_ROBIN, PG.CONTIGUOUS])
+@pytest.mark.parametrize("window,seg", [(0, 128), (300, 256), (700, 128)])
+def test_kvp_prefill_matches_oracle(mode, window, seg):
+    R, bps, bs, hq, hkv, D, S = 4, 8, 32, 8, 2, 128, 300
+    q, kc, vc, perm = _paged(20, R, bps, bs, hq, hkv, D, S)
+    bt = PG.shard_block_tables(perm, R, mode)
+    gqo = R * bps * bs - S - 17
+    K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, mode)
+    ro, rl = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=window)
+    kv_mode = cbv.KV_ROUND_ROBIN if mode == PG.ROUND_ROBIN else cbv.KV_CONTIGUOUS
+    out, lse = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), kv_mode=kv_mode, seg_size=seg,
+                                         scale=0.1, global_q_offset=gqo, sliding_window=window)
+    sync()
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+
+
+def test_kvp_per_shard_partials_and_their_merge():
+    R, bps, bs, hq, hkv, D, S = 4, 4, 32, 4, 1, 128, 200
+    q, kc, vc, perm = _paged(21, R, bps, bs, hq, hkv, D, S)
+    bt = PG.shard_block_tables(perm, R, PG.ROUND_ROBIN)
+    gqo = 300
+    (ro, rl), shards = PG.prefill_segmented(f64(q), f64(kc), f64(vc), bt, bs, 128, 0.1, gqo, window=0,
+                                            mode=PG.ROUND_ROBIN, return_shards=True)
+    out, lse, so, sl = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), seg_size=128,
+                                                 scale=0.1, global_q_offset=gqo, per_shard=True)
+    sync()
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+    for r in range(R):
+        check_out(host(so[r]), shards[r][0], what=f"shard {r} out")
+        check_lse(host(sl[r]), shards[r][1], what=f"shard {r} lse")
+
+
+def test_kvp_segment_size_does_not_change_the_result():
+    R, bps, bs, hq, hkv, D, S = 2, 16, 16, 4, 2, 64, 256
+    q, kc, vc, perm = _paged(22, R, bps, bs, hq, hkv, D, S)
+    bt = torch.from_numpy(PG.shard_block_tables(perm, R, PG.ROUND_ROBIN))
+    a = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), bt, seg_size=128, global_q_offset=256)
+    b = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), bt, seg_size=256, global_q_offset=256)
+    sync()
+    assert torch.allclose(a[0].float(), b[0].float(), atol=1e-2)
+    assert torch.allclose(a[1], b[1], atol=1e-4)
+
+
+@pytest.mark.parametrize("hq,hkv,D", [(32, 4, 128), (8, 8, 128), (16, 2, 64), (12, 3, 128)])
+def test_decode_matches_oracle(hq, hkv, D):
+    lengths = np.concatenate([[0, 1, 2, 31, 32, 33, 64, 65], streams(30, 1)[0].integers(1, 700, 40)])
+    n = len(lengths)
+    cu_k = cu_from_lengths(lengths)
+    q, k, v = gen(31, (n, hq, D), (int(cu_k[-1]), hkv, D), (int(cu_k[-1]), hkv, D))
+    cu_q = np.arange(n + 1, dtype=np.int32)
+    ref = DEC.varlen_decode(f64(q), f64(k), f64(v), cu_q, cu_k, 0.1)
+    out = cbv.varlen_decode(dev(q), dev(k), dev(v), torch.from_numpy(cu_q), torch.from_numpy(cu_k), scale=0.1)
+    sync()
+    check_out(host(out), ref)
+    assert np.all(host(out)[0] == 0)  # empty key range -> zeros
+
+
+def test_decode_reads_offsets_on_device():
+    # change cu_seqlens_k contents in place (no host round trip) and run again
+    hq, hkv, D = 8, 2, 128
+    lengths = np.array([5, 100, 0, 77])
+    cu_k = cu_from_lengths(lengths)
+    q, k, v = gen(32, (4, hq, D), (400, hkv, D), (400, hkv, D))
+    cu_q = torch.arange(5, dtype=torch.int32, device="cuda")
+    ck = torch.from_numpy(cu_k).cuda()
+    out = torch.empty((4, hq, D), dtype=torch.bfloat16, device="cuda")
+    cbv.varlen_decode(dev(q), dev(k), dev(v), cu_q, ck, scale=0.1, validate=False, out=out)
+    new = cu_from_lengths([50, 0, 200, 1])
+    ck.copy_(torch.from_numpy(new))
+    cbv.varlen_decode(dev(q), dev(k), dev(v), cu_q, ck, scale=0.1, validate=False, out=out)
+    sync()
+    ref = DEC.varlen_decode(f64(q), f64(k), f64(v), np.arange(5), new, 0.1)
+    check_out(host(out), ref)
+
+
+def test_decode_rejects_more_than_one_query_per_sequence():
+    q, k, v = gen(33, (4, 8, 128), (10, 2, 128), (10, 2, 128))
+    with pytest.raises(cbv.CbvError) as e:
+        cbv.varlen_decode(dev(q), dev(k), dev(v), torch.tensor([0, 1, 3, 4]), torch.tensor([0, 3, 6, 10]))
+    assert e.value.status == "Q_LEN_NOT_ONE"
