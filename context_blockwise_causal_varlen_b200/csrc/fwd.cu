@@ -269,7 +269,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const int32_t qpos = t.pos0 + row;
     const float sl2 = p.scale_log2;
     const int32_t W = p.window;
-    float m = -INFINITY, l = 0.f;
+    // l: exact fp32 row sum (for lse); lr: sum of the bf16-rounded P the PV product uses,
+    // which normalises out so the weights applied to V sum to one exactly
+    float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
     TileIter it;
     TileRef r;
@@ -321,19 +323,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         rescale_o = (m != -INFINITY);
       }
       const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-      float rowsum = 0.f;
+      float rowsum = 0.f, rowsum_r = 0.f;
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
         const float p0 = ex2_approx(__uint_as_float(s[c]) - msub);
         const float p1 = ex2_approx(__uint_as_float(s[c + 1]) - msub);
         const uint32_t pb = pack_bf16x2(p0, p1);
-        // the row sum adds the bf16 values the PV product uses, so the weights
-        // applied to V are normalised exactly (a dominant key keeps its value)
-        rowsum += __uint_as_float(pb << 16) + __uint_as_float(pb & 0xffff0000u);
+        rowsum += p0 + p1;
+        rowsum_r += __uint_as_float(pb << 16) + __uint_as_float(pb & 0xffff0000u);
         pk[c / 2] = pb;
       }
       l = l * alpha + rowsum;
+      lr = lr * alpha + rowsum_r;
       m = m_use;
       // PV of the previous tile must be done before O is rescaled and P is overwritten
       if (i > 0 && !mbar_wait_warp(&bar[bPVDone], (i - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
@@ -367,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (ok && mbar_wait_warp(&bar[bODone], 0, p.status, kDevTimeoutEpilogue)) {
       tc_fence_after();
       const bool has = (l > 0.f) && (m != -INFINITY);
-      const float inv_l = has ? 1.f / l : 0.f;
+      const float inv_l = (has && lr > 0.f) ? 1.f / lr : 0.f;
       const float lse_b = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
       const bool valid = row < t.rows;
       const int64_t orow = (int64_t)(t.row0 + row);
