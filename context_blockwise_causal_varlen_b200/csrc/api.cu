@@ -635,8 +635,18 @@ int make_bwd_maps(BwdParams* p, const void* q, const void* dout, const void* k, 
   if ((rc = map_thd(&p->tm_v, v, total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
   uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)std::max<int64_t>(total_q, 1)};
   uint64_t st[2] = {(uint64_t)D, (uint64_t)H * D};
-  uint32_t box[3] = {(uint32_t)D / 4, 1, 64};  // one warp's head-dim slice x 64 q rows
+  uint32_t box[3] = {(uint32_t)D / 4, 1, 32};  // one warp's head-dim slice x 32 q rows
   return make_map(&p->tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 3, dq_acc, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+int64_t pad4(int64_t t) { return (t + 3) / 4 * 4; }
+
+// [H, t_pad] fp32 rows (lse * log2e or Delta) as a 2-D map, box of 68 rows
+int make_row_map(CUtensorMap* m, const float* rows, int64_t t_pad, int H) {
+  uint64_t dims[2] = {(uint64_t)std::max<int64_t>(t_pad, 4), (uint64_t)H};
+  uint64_t st[1] = {(uint64_t)t_pad};
+  uint32_t box[2] = {68, 1};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2, rows, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 struct BwdLayout {
@@ -654,7 +664,8 @@ size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a) {
   Carve c(nullptr);
   c.take(kStatusBytes);
   carve_plan(c, plan);
-  c.take((size_t)a->num_heads * a->total * sizeof(float));                 // Delta
+  c.take((size_t)a->num_heads * pad4(a->total) * sizeof(float));           // Delta
+  c.take((size_t)a->num_heads * pad4(a->total) * sizeof(float));           // lse * log2e
   c.take((size_t)a->total * a->num_heads * a->head_dim * sizeof(float));   // dq accumulator
   return c.off;
 }
@@ -672,7 +683,9 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   Carve c(a->workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, plan);
-  float* delta = static_cast<float*>(c.take((size_t)H * a->total * sizeof(float)));
+  const int64_t tp = pad4(a->total);
+  float* delta = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
+  float* lse2 = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
   float* dq_acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   BwdParams p{};
@@ -686,9 +699,8 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   p.scale = resolve_scale(a->scale, D);
   p.scale_log2 = p.scale * kLog2e;
   p.window = a->window > 0 ? a->window : 0;
-  p.lse = a->lse;
-  p.lse_stride_h = a->total;
-  p.delta = delta;
+  if ((rc = make_row_map(&p.tm_lse, lse2, tp, H))) return rc;
+  if ((rc = make_row_map(&p.tm_delta, delta, tp, H))) return rc;
   p.dk = a->dk;
   p.dv = a->dv;
   p.dkv_stride_t = (int64_t)Hkv * D;
@@ -697,7 +709,8 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->total, H, D, delta, dq_acc, s), "backward preprocess")))
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, delta, lse2, dq_acc, s),
+                      "backward preprocess")))
     return rc;
   const int grid = grid_of(plan.tasks.size(), Hkv);
   if ((rc = launch_rc(launch_bwd(p, D, grid, s), "backward launch"))) return rc;
@@ -726,7 +739,8 @@ size_t cbv_block_bwd_workspace_size(const cbv_block_bwd_args* a) {
   Carve c(nullptr);
   c.take(kStatusBytes);
   carve_plan(c, plan);
-  c.take((size_t)a->num_heads * a->total_q * sizeof(float));
+  c.take((size_t)a->num_heads * pad4(a->total_q) * sizeof(float));
+  c.take((size_t)a->num_heads * pad4(a->total_q) * sizeof(float));
   return c.off;
 }
 
@@ -740,7 +754,9 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   Carve c(a->workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, plan);
-  float* delta = static_cast<float*>(c.take((size_t)H * a->total_q * sizeof(float)));
+  const int64_t tp = pad4(a->total_q);
+  float* delta = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
+  float* lse2 = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   BwdParams p{};
   if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, a->dq_acc, a->total_q, a->total_k, H, Hkv, D))) return rc;
@@ -753,9 +769,8 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.scale = resolve_scale(a->scale, D);
   p.scale_log2 = p.scale * kLog2e;
   p.window = a->window > 0 ? a->window : 0;
-  p.lse = a->lse;
-  p.lse_stride_h = a->total_q;
-  p.delta = delta;
+  if ((rc = make_row_map(&p.tm_lse, lse2, tp, H))) return rc;
+  if ((rc = make_row_map(&p.tm_delta, delta, tp, H))) return rc;
   p.dk = a->dk_acc;
   p.dv = a->dv_acc;
   p.dkv_stride_t = (int64_t)Hkv * D;
@@ -764,7 +779,8 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->total_q, H, D, delta, nullptr, s), "backward preprocess")))
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, delta, lse2, nullptr, s),
+                      "backward preprocess")))
     return rc;
   return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), Hkv), s), "backward launch");
 }

@@ -13,8 +13,9 @@
 // formed per q tile in TMEM and added to an fp32 dq accumulator with a TMA bulk
 // reduce-add.
 //
-// Warps: 0 TMA producer (+ lse/Delta rows), 1 UMMA issuer (+ TMEM owner),
-// 2-5 P / dS (one key row per thread) and the dK/dV epilogue, 6-9 dQ readout.
+// Warps: 0 TMA producer (q, dO, lse*log2e and Delta rows of a 3-stage ring),
+// 1 UMMA issuer (+ TMEM owner), 2-9 P / dS in two warpgroups that split the 64
+// q columns (one key row per thread) and then the dV / dK epilogue, 10-13 dQ readout.
 // TMEM columns: S^T [0,64), dP^T [64,128), dQ^T x2 [128,256), dV [256,256+D), dK [384,384+D).
 #include "kernels.h"
 #include "ptx.cuh"
@@ -25,7 +26,10 @@ namespace {
 
 constexpr int BN = 128;  // keys per CTA
 constexpr int BM = 64;   // q rows per streamed tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
+constexpr int NS = 3;     // q / dO / row stages
+constexpr int kRowBox = BM + 4;  // lse/Delta box: 68 floats from a 16-byte aligned start
+constexpr int kRowSlot = 96;     // floats per row buffer: 384 bytes keeps every TMA destination 128-byte aligned
 
 struct QTile {
   int32_t q_row;   // first q row
@@ -87,34 +91,35 @@ struct BwdSmem {
   static constexpr uint32_t kKV = BN * D * 2;   // K or V tile (128 x D)
   static constexpr uint32_t kQT = BM * D * 2;   // a q / dO tile (64 x D)
   static constexpr uint32_t kPT = BN * BM * 2;  // P^T or dS^T (128 x 64)
+  static constexpr uint32_t kRowBytes = kRowBox * 4;  // bytes one row box delivers
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kKV;
-  static constexpr uint32_t kQ = kV + kKV;           // 2 stages
-  static constexpr uint32_t kDO = kQ + 2 * kQT;      // 2 stages
-  static constexpr uint32_t kPt = kDO + 2 * kQT;
+  static constexpr uint32_t kQ = kV + kKV;            // NS stages
+  static constexpr uint32_t kDO = kQ + NS * kQT;      // NS stages
+  static constexpr uint32_t kPt = kDO + NS * kQT;
   static constexpr uint32_t kDSt = kPt + kPT;
-  static constexpr uint32_t kDQ = kDSt + kPT;        // fp32 staging [64][D]
-  static constexpr uint32_t kRow = kDQ + BM * D * 4;  // per stage: lse*log2e [64], Delta [64]
-  static constexpr uint32_t kBars = kRow + 2 * 2 * BM * 4;
-  static constexpr uint32_t kEnd = kBars + 256;
+  static constexpr uint32_t kDQ = kDSt + kPT;             // fp32 staging: 4 warps x [32][D/4]
+  static constexpr uint32_t kRow = kDQ + (BM / 2) * D * 4;  // per stage: lse*log2e and Delta slots
+  static constexpr uint32_t kBars = kRow + NS * 2 * kRowSlot * 4;
+  static constexpr uint32_t kEnd = kBars + 128;
   static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
+  static_assert(kDynamic <= 232448, "shared memory budget");
 };
 
 enum BBar {
   bKVFull = 0,
-  bQFull = 1,    // +stage
-  bQEmpty = 3,   // +stage
-  bSFull = 5,
-  bSFree = 6,
-  bPFull = 7,
-  bPtFree = 8,
-  bDQFull = 9,   // +buffer
-  bDQFree = 11,  // +buffer
-  bAccDone = 13,
-  bBNum = 14
+  bQFull = 1,    // +stage (NS)
+  bQEmpty = 4,   // +stage (NS)
+  bSFull = 7,
+  bSFree = 8,
+  bPFull = 9,
+  bPtFree = 10,
+  bDQFull = 11,  // +buffer (2)
+  bDQFree = 13,  // +buffer (2)
+  bAccDone = 15,
+  bBNum = 16
 };
 
-constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
@@ -129,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* sPt = sm + L::kPt;
   uint8_t* sDSt = sm + L::kDSt;
   float* sDQ = reinterpret_cast<float*>(sm + L::kDQ);
-  float* sRow = reinterpret_cast<float*>(sm + L::kRow);  // [stage][lse2 64 | delta 64]
+  float* sRow = reinterpret_cast<float*>(sm + L::kRow);  // [stage][lse*log2e 68 | Delta 68]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + bBNum);
 
@@ -141,15 +146,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bar[bKVFull], 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[bQFull + s], 2);  // TMA bytes + the producer warp's lse/Delta stores
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar[bQFull + s], 1);
       mbar_init(&bar[bQEmpty + s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[bDQFull + s], 1);
       mbar_init(&bar[bDQFree + s], 4);
     }
     mbar_init(&bar[bSFull], 1);
-    mbar_init(&bar[bSFree], 4);
-    mbar_init(&bar[bPFull], 4);
+    mbar_init(&bar[bSFree], 8);
+    mbar_init(&bar[bPFull], 8);
     mbar_init(&bar[bPtFree], 1);
     mbar_init(&bar[bAccDone], 1);
     fence_mbar_init();
@@ -174,30 +181,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tma_load_3d(sV + h * 16384, &p.tm_v, &bar[bKVFull], h * 64, kvh, t.row0);
       }
     }
-    QIter it;
-    QTile r;
-    int j = 0;
-    while (next_qtile(p, t, kvh, it, r)) {
-      const int st = j & 1;
-      if (!mbar_wait_warp(&bar[bQEmpty + st], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar[bQFull + st], 2 * L::kQT);
+    if (lane == 0) {
+      QIter it;
+      QTile r;
+      int j = 0;
+      while (next_qtile(p, t, kvh, it, r)) {
+        const int st = j % NS;
+        if (!mbar_wait(&bar[bQEmpty + st], ((j / NS) & 1) ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
+        uint64_t* full = &bar[bQFull + st];
+        mbar_arrive_expect_tx(full, 2 * L::kQT + 2 * L::kRowBytes);
         for (int h = 0; h < KH; ++h) {
-          tma_load_3d(sQ + st * L::kQT + h * 8192, &p.tm_q, &bar[bQFull + st], h * 64, r.head, r.q_row);
-          tma_load_3d(sDO + st * L::kQT + h * 8192, &p.tm_do, &bar[bQFull + st], h * 64, r.head, r.q_row);
+          tma_load_3d(sQ + st * L::kQT + h * 8192, &p.tm_q, full, h * 64, r.head, r.q_row);
+          tma_load_3d(sDO + st * L::kQT + h * 8192, &p.tm_do, full, h * 64, r.head, r.q_row);
         }
+        float* row = sRow + st * 2 * kRowSlot;
+        const int x = r.q_row & ~3;  // 16-byte aligned start; the softmax indexes from q_row & 3
+        tma_load_2d(row, &p.tm_lse, full, x, r.head);
+        tma_load_2d(row + kRowSlot, &p.tm_delta, full, x, r.head);
+        ++j;
       }
-      float* row = sRow + st * 2 * BM;
-      const float* lse = p.lse + (int64_t)r.head * p.lse_stride_h;
-      const float* dl = p.delta + (int64_t)r.head * p.lse_stride_h;
-      for (int c = lane; c < BM; c += 32) {
-        const bool v = c < r.nvalid;
-        row[c] = v ? __ldg(&lse[r.q_row + c]) * kLog2e : INFINITY;
-        row[BM + c] = v ? __ldg(&dl[r.q_row + c]) : 0.f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[bQFull + st]);
-      ++j;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ UMMA issuer
@@ -210,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       bool ok = mbar_wait(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_sdp = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&bar[bQFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
+        const int st = j % NS;
+        if (!mbar_wait(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutMma)) return false;
         if (!mbar_wait(&bar[bSFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) return false;
         tc_fence_after();
 #pragma unroll
@@ -234,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
       if (ok && n > 0) ok = issue_sdp(0);
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j & 1;
+        const int st = j % NS;
+        const int db = j & 1;  // dQ^T TMEM buffer
         if (j + 1 < n && !(ok = issue_sdp(j + 1))) break;
         if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
@@ -247,25 +250,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           umma_bf16_ss(tDV, pa, ob, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
           umma_bf16_ss(tDK, da, qb, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        if (!mbar_wait(&bar[bDQFree + st], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait(&bar[bDQFree + db], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t ka = sdesc_sw128(k0 + kk * 2048, 16384, 1024);
           const uint64_t sb = sdesc_sw128(ds0 + kk * 2048, 16384, 1024);
-          umma_bf16_ss(tDQ0 + st * 64, ka, sb, id_dq, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tDQ0 + db * 64, ka, sb, id_dq, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bar[bQEmpty + st]);
         umma_commit(&bar[bPtFree]);
-        umma_commit(&bar[bDQFull + st]);
+        umma_commit(&bar[bDQFull + db]);
       }
       (void)it;
       (void)r;
       if (n > 0) umma_commit(&bar[bAccDone]);
       else mbar_arrive(&bar[bAccDone]);
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // ------------------------------------------------------------------ P / dS (thread = key row)
+    // warpgroup wg handles q columns [32 wg, 32 wg + 32) of every tile
+    const int wg = (warp - 2) >> 2;
+    const int c0 = wg * 32;
     const int quarter = warp & 3;
     const int krow = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -279,24 +285,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     int j = 0;
     bool ok = true;
     while (next_qtile(p, t, kvh, it, r)) {
-      const int st = j & 1;
-      if (!mbar_wait_warp(&bar[bQFull + st], (j >> 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+      const int st = j % NS;
+      if (!mbar_wait_warp(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
       if (!mbar_wait_warp(&bar[bSFull], j & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
       tc_fence_after();
-      const float* row = sRow + st * 2 * BM;
-      uint32_t pp[BM / 2], pd[BM / 2];
-#pragma unroll
-      for (int hc = 0; hc < BM; hc += 32) {
+      const float* lrow = sRow + st * 2 * kRowSlot + (r.q_row & 3) + c0;
+      const float* drow = lrow + kRowSlot;
+      uint32_t pp[16], pd[16];
+      {
         uint32_t s[32], dp[32];
-        tmem_ld32(tS + lane_base + hc, s);
-        tmem_ld32(tDP + lane_base + hc, dp);
+        tmem_ld32(tS + lane_base + c0, s);
+        tmem_ld32(tDP + lane_base + c0, dp);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           float pv[2], dv[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int col = hc + c + e;
+            const int col = c0 + c + e;
             bool vis = true;
             if (r.need_mask) {
               const int32_t qpos = r.qpos0 + col;
@@ -304,12 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
               if (r.causal || W > 0) vis = vis && (kpos <= qpos);
               if (W > 0) vis = vis && (qpos - kpos < W);
             }
-            const float pe = vis ? ex2_approx(__uint_as_float(s[c + e]) * sl2 - row[col]) : 0.f;
+            const float pe = vis ? ex2_approx(fmaf(__uint_as_float(s[c + e]), sl2, -lrow[c + e])) : 0.f;
             pv[e] = pe;
-            dv[e] = pe * (__uint_as_float(dp[c + e]) - row[BM + col]);
+            // rows past the segment hold whatever the row buffer holds: keep them out of dS
+            dv[e] = vis ? pe * (__uint_as_float(dp[c + e]) - drow[c + e]) : 0.f;
           }
-          pp[(hc + c) / 2] = pack_bf16x2(pv[0], pv[1]);
-          pd[(hc + c) / 2] = pack_bf16x2(dv[0], dv[1]);
+          pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
+          pd[c / 2] = pack_bf16x2(dv[0], dv[1]);
         }
       }
       tc_fence_before();
@@ -317,9 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       if (lane == 0) mbar_arrive(&bar[bSFree]);
       if (j > 0 && !mbar_wait_warp(&bar[bPtFree], (j - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        st_shared_v4(pt_row + sw128_offset(krow, ch), pp[ch * 4], pp[ch * 4 + 1], pp[ch * 4 + 2], pp[ch * 4 + 3]);
-        st_shared_v4(ds_row + sw128_offset(krow, ch), pd[ch * 4], pd[ch * 4 + 1], pd[ch * 4 + 2], pd[ch * 4 + 3]);
+      for (int ch = 0; ch < 4; ++ch) {
+        const int chunk = (c0 >> 3) + ch;
+        st_shared_v4(pt_row + sw128_offset(krow, chunk), pp[ch * 4], pp[ch * 4 + 1], pp[ch * 4 + 2], pp[ch * 4 + 3]);
+        st_shared_v4(ds_row + sw128_offset(krow, chunk), pd[ch * 4], pd[ch * 4 + 1], pd[ch * 4 + 2], pd[ch * 4 + 3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -330,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     if (ok && mbar_wait_warp(&bar[bAccDone], 0, p.status, kDevTimeoutEpilogue)) {
       tc_fence_after();
       const bool any = j > 0;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
+      {
+        const int which = wg;  // warpgroup 0: dV, warpgroup 1: dK
         const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_base;
         const float mul = which == 0 ? 1.f : p.scale;
         void* dst_base = which == 0 ? p.dv : p.dk;
@@ -371,14 +379,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------------ dQ readout (thread = head-dim row)
-    // Each warp owns D/4 head-dim rows and adds its [64 x D/4] slice with its own
-    // bulk reduce, so the four warps never wait on one another.
+    // Each warp owns D/4 head-dim rows and adds its [32 x D/4] slices (two per q tile)
+    // with its own bulk reduces, so the four warps never wait on one another.
     const int quarter = warp & 3;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     constexpr int DW = D / 4;  // head-dim rows per warp
     // M = 128: lane l of quarter q holds d = 32q + l; M = 64: lanes 0-15 of quarter q hold d = 16q + l
     const bool dvalid = lane < DW;
-    float* region = sDQ + quarter * (BM * DW);
+    float* region = sDQ + quarter * ((BM / 2) * DW);
     QIter it;
     QTile r;
     int j = 0;
@@ -392,20 +400,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar[bDQFree + st]);
-        bulk_wait_group_read<0>();  // this warp's previous reduce has finished reading its region
-      }
-      __syncwarp();
-      if (dvalid) {
+      if (lane == 0) mbar_arrive(&bar[bDQFree + st]);
 #pragma unroll
-        for (int c = 0; c < BM; ++c) region[c * DW + lane] = __uint_as_float(v[c]) * p.scale;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row);
-        bulk_commit_group();
+      for (int hf = 0; hf < 2; ++hf) {
+        if (lane == 0) bulk_wait_group_read<0>();  // this warp's previous reduce has read its region
+        __syncwarp();
+        if (dvalid) {
+#pragma unroll
+          for (int c = 0; c < BM / 2; ++c) region[c * DW + lane] = __uint_as_float(v[hf * 32 + c]) * p.scale;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row + hf * 32);
+          bulk_commit_group();
+        }
       }
       ++j;
     }

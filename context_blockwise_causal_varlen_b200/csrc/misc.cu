@@ -74,10 +74,13 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ out, flo
   }
 }
 
+// Backward preprocess: Delta_i = <dO_i, O_i> with the merged (bf16) output, and the
+// merged lse in log2 units, both laid out [H, t_pad] for the backward's row loads.
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ dout,
-                                                    const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
-                                                    int64_t total, int heads) {
+                                                    const __nv_bfloat16* __restrict__ out,
+                                                    const float* __restrict__ lse, float* __restrict__ delta,
+                                                    float* __restrict__ lse2, int64_t total, int64_t t_pad, int heads) {
   constexpr int E = D / 32;
   const int64_t rowid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -92,7 +95,8 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
   if (lane == 0) {
     const int64_t tok = rowid / heads;
     const int h = (int)(rowid % heads);
-    delta[(int64_t)h * total + tok] = s;
+    delta[(int64_t)h * t_pad + tok] = s;
+    lse2[(int64_t)h * t_pad + tok] = lse[(int64_t)h * total + tok] * 1.4426950408889634f;
   }
 }
 
@@ -127,8 +131,9 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
   return (int)cudaGetLastError();
 }
 
-int launch_bwd_preprocess(const void* dout, const void* out, int64_t total, int32_t heads, int32_t head_dim,
-                          float* delta, float* dq_acc, cudaStream_t stream) {
+int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
+                          int32_t heads, int32_t head_dim, float* delta, float* lse2, float* dq_acc,
+                          cudaStream_t stream) {
   const int64_t rows = total * heads;
   if (rows == 0) return 0;
   if (dq_acc) {
@@ -138,8 +143,8 @@ int launch_bwd_preprocess(const void* dout, const void* out, int64_t total, int3
   const int64_t blocks = (rows + 7) / 8;
   auto d = reinterpret_cast<const __nv_bfloat16*>(dout);
   auto o = reinterpret_cast<const __nv_bfloat16*>(out);
-  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, delta, total, heads);
-  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, delta, total, heads);
+  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, delta, lse2, total, t_pad, heads);
+  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, delta, lse2, total, t_pad, heads);
   else return (int)cudaErrorInvalidValue;
   return (int)cudaGetLastError();
 }
