@@ -140,6 +140,7 @@ EXPORTS = [
     "cbv_zigzag_ring_fwd_workspace_size", "cbv_zigzag_ring_fwd", "cbv_zigzag_ring_bwd_workspace_size",
     "cbv_zigzag_ring_bwd", "cbv_block_bwd_workspace_size", "cbv_attn_block_bwd",
     "cbv_kvp_workspace_size", "cbv_kvp_segmented_prefill", "cbv_decode_workspace_size", "cbv_varlen_decode",
+    "cbv_noalloc_scratch_bytes", "cbv_zigzag_ring_fwd_noalloc",
 ]
 
 
@@ -163,6 +164,8 @@ def _declare(L):
                      ("cbv_zigzag_ring_bwd", RingArgs), ("cbv_attn_block_bwd", BlockBwdArgs),
                      ("cbv_kvp_segmented_prefill", KvpArgs), ("cbv_varlen_decode", DecodeArgs)):
         getattr(L, name).argtypes = [ctypes.POINTER(st), ctypes.c_void_p]
+    L.cbv_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    L.cbv_zigzag_ring_fwd_noalloc.argtypes = [ctypes.POINTER(RingArgs), ctypes.c_void_p]
     L.cbv_attn_merge.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
 

@@ -225,6 +225,11 @@ FwdParams ring_fwd_params(const cbv_ring_args* a, int* rc) {
 
 }  // namespace
 
+namespace cbv {
+// Sets the text cbv_last_error_message() returns (for entry points in other files).
+void set_last_error(const char* msg) { g_err = msg; }
+}  // namespace cbv
+
 extern "C" {
 
 const char* cbv_last_error_message(void) { return g_err.c_str(); }

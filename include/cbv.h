@@ -18,7 +18,8 @@
  *     current device; "host" pointers are ordinary CPU memory read during the call
  *     and not retained.  The caller owns all memory; the library allocates nothing
  *     and keeps no state between calls.  Scratch memory comes from a caller-owned
- *     device `workspace` whose size the matching *_workspace_size() call reports.
+ *     device `workspace` whose size the matching *_workspace_size() call reports
+ *     (cbv_zigzag_ring_fwd_noalloc, at the end, is the one call with built-in scratch).
  *   - bf16 means IEEE bfloat16 (torch.bfloat16); token-major layouts are
  *     [tokens, heads, head_dim], contiguous.  lse is float32 [heads, tokens],
  *     natural log.  head_dim is 64 or 128.
@@ -313,6 +314,30 @@ typedef struct cbv_decode_args {
 } cbv_decode_args;
 size_t cbv_decode_workspace_size(const cbv_decode_args* a);
 int cbv_varlen_decode(const cbv_decode_args* a, void* stream);
+
+/* ========================================================================= ring forward without allocation
+ * The pages have no counterpart for this call; it serves callers that cannot allocate.
+ * cbv_zigzag_ring_fwd takes its scratch (status word and tile schedule) from a workspace the
+ * caller allocates.  Callers that cannot call cudaMalloc where they run attention (an
+ * allocation-free serving loop with a memory budget fixed at start-up, a runtime that owns all
+ * device memory through its own allocator, a plain C host with no device allocator) can use
+ * this variant instead: it computes exactly what cbv_zigzag_ring_fwd computes with the fused
+ * schedule, but its scratch is a fixed array of cbv_noalloc_scratch_bytes() bytes (1 MiB)
+ * compiled into the library, which every GPU that loads the library holds until the process
+ * exits.  a->workspace and a->workspace_bytes are ignored; inputs and outputs are still the
+ * caller's.  It calls no cudaMalloc, cudaFree or allocating library routine.
+ * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ * - Every call, from any thread or stream, shares the one array, and each call overwrites what
+ *   the last one left there: calls that overlap on the GPU race.  Serialise them (one stream,
+ *   or events between streams).
+ * - A problem whose scratch would exceed the array (cbv_zigzag_ring_fwd_workspace_size()
+ *   larger than cbv_noalloc_scratch_bytes(), e.g. the stepwise schedule, which keeps an fp32
+ *   running output) returns CBV_ERR_WORKSPACE_TOO_SMALL with a message; nothing is launched.
+ * - Argument errors are those of cbv_zigzag_ring_fwd.
+ * - cbv_read_status() cannot reach the array; a kernel timeout shows up as wrong output only. */
+size_t cbv_noalloc_scratch_bytes(void);
+int cbv_zigzag_ring_fwd_noalloc(const cbv_ring_args* a, void* stream);
 
 #ifdef __cplusplus
 }
