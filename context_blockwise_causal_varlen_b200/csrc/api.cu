@@ -191,11 +191,13 @@ RingFwdLayout ring_fwd_layout(const cbv_ring_args* a) {
   Carve c(nullptr);
   c.take(kStatusBytes);
   if (a->schedule == CBV_SCHEDULE_FUSED) {
-    L.fused = plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, -1, 128);
+    L.fused = plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, -1, 128,
+                            true);
     carve_plan(c, L.fused);
   } else {
     for (int s = 0; s < a->cp; ++s) {
-      L.steps.push_back(plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, s, 128));
+      L.steps.push_back(
+          plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, s, 128, false));
       carve_plan(c, L.steps.back());
     }
     c.take((size_t)a->total * a->num_heads * a->head_dim * sizeof(float));  // running out (fp32)
@@ -381,7 +383,7 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  const int grid = grid_of(plan.tasks.size(), H);
+  const int grid = grid_of(plan.tasks.size(), 1);
   if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
   return launch_rc(launch_fwd(p, D, false, grid, s), "block forward launch");
 }
@@ -429,7 +431,7 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
     p.num_tasks = (int)L.fused.tasks.size();
     p.out = a->out;
     p.out_mode = kOutBf16;
-    return launch_rc(launch_fwd(p, D, false, grid_of(L.fused.tasks.size(), H), s), "ring forward launch");
+    return launch_rc(launch_fwd(p, D, false, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch");
   }
   std::vector<PlanDev> pds;
   for (auto& pl : L.steps) {
@@ -443,7 +445,7 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
     p.num_tasks = (int)L.steps[st].tasks.size();
     p.out = acc;
     p.out_mode = st == 0 ? kOutF32 : kOutMerge;
-    if ((rc = launch_rc(launch_fwd(p, D, false, grid_of(L.steps[st].tasks.size(), H), s), "ring step launch")))
+    if ((rc = launch_rc(launch_fwd(p, D, false, grid_of(L.steps[st].tasks.size(), 1), s), "ring step launch")))
       return rc;
   }
   return launch_rc(launch_convert_bf16(acc, a->out, a->total * H * D, 1.f, s), "output conversion");
@@ -529,7 +531,7 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  const int grid = grid_of(plan.tasks.size(), H);
+  const int grid = grid_of(plan.tasks.size(), 1);
   if (!a->shard_out) {
     p.out = a->out;
     p.out_mode = kOutBf16;
@@ -717,7 +719,7 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, delta, lse2, dq_acc, s),
                       "backward preprocess")))
     return rc;
-  const int grid = grid_of(plan.tasks.size(), Hkv);
+  const int grid = grid_of(plan.tasks.size(), 1);
   if ((rc = launch_rc(launch_bwd(p, D, grid, s), "backward launch"))) return rc;
   return launch_rc(launch_convert_bf16(dq_acc, a->dq, a->total * H * D, 1.f, s), "dq conversion");
 }
@@ -787,7 +789,7 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, delta, lse2, nullptr, s),
                       "backward preprocess")))
     return rc;
-  return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), Hkv), s), "backward launch");
+  return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch");
 }
 
 }  // extern "C"

@@ -140,9 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int task_idx = blockIdx.x / p.num_kv_heads;
-  const int kvh = blockIdx.x % p.num_kv_heads;
-  const TileTask t = p.tasks[task_idx];
+  const TileTask t = p.tasks[blockIdx.x];
+  const int kvh = t.head;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar[bKVFull], 1);
@@ -297,19 +296,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tmem_ld32(tS + lane_base + c0, s);
         tmem_ld32(tDP + lane_base + c0, dp);
         tmem_ld_wait();
+        // this key row sees the q columns [lo, hi] (positions are linear in the column)
+        int32_t lo = 0, hi = BM - 1;
+        if (r.need_mask) {
+          hi = kvalid ? r.nvalid - 1 : -1;
+          if (r.causal || W > 0) lo = max(lo, kpos - r.qpos0);
+          if (W > 0) hi = min(hi, kpos + W - 1 - r.qpos0);
+        }
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
           float pv[2], dv[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int col = c0 + c + e;
-            bool vis = true;
-            if (r.need_mask) {
-              const int32_t qpos = r.qpos0 + col;
-              vis = kvalid && col < r.nvalid;
-              if (r.causal || W > 0) vis = vis && (kpos <= qpos);
-              if (W > 0) vis = vis && (qpos - kpos < W);
-            }
+            const bool vis = col >= lo && col <= hi;
             const float pe = vis ? ex2_approx(fmaf(__uint_as_float(s[c + e]), sl2, -lrow[c + e])) : 0.f;
             pv[e] = pe;
             // rows past the segment hold whatever the row buffer holds: keep them out of dS

@@ -143,10 +143,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int task_idx = blockIdx.x / p.num_heads;
-  const int head = blockIdx.x % p.num_heads;
+  const TileTask t = p.tasks[blockIdx.x];
+  const int head = t.head;
   const int kvh = head / p.heads_per_kv;
-  const TileTask t = p.tasks[task_idx];
 
   if (threadIdx.x == 0) {
     mbar_init(&bar[bQFull], 1);
@@ -290,15 +289,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       if (lane == 0) mbar_arrive(&bar[bSFree + sb]);
 
       float mx = -INFINITY;
-      if (r.need_mask) {
+      if (r.need_mask && (!PAGED || p.kv_mode == kKvContiguous)) {
+        // positions are linear in the column: the visible columns of this row are [lo, hi]
+        int32_t hi = r.nvalid - 1, lo = 0;
+        if (r.causal || W > 0) hi = min(hi, qpos - r.kpos0);
+        if (W > 0) lo = max(lo, qpos - W + 1 - r.kpos0);
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
-          int32_t kpos;
-          if (!PAGED || p.kv_mode == kKvContiguous) {
-            kpos = r.kpos0 + c;
-          } else {
-            kpos = r.kpos0 + (c / p.block_size) * p.shards * p.block_size + (c % p.block_size);
-          }
+          const float v = (c >= lo && c <= hi) ? __uint_as_float(s[c]) * sl2 : -INFINITY;
+          s[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else if (r.need_mask) {
+        // round-robin pages: position = page base + offset inside the page
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int32_t kpos = r.kpos0 + (c / p.block_size) * p.shards * p.block_size + (c % p.block_size);
           bool vis = c < r.nvalid;
           if (r.causal || W > 0) vis = vis && (kpos <= qpos);
           if (W > 0) vis = vis && (qpos - kpos < W);

@@ -37,8 +37,55 @@ int64_t visible_pairs(int64_t qp, int64_t nq, int64_t kp, int64_t nk, bool causa
 
 int32_t weight(int64_t pairs) { return (int32_t)std::min<int64_t>(pairs / 256 + 1, INT32_MAX); }
 
-void sort_tasks(std::vector<TileTask>& t) {
-  std::stable_sort(t.begin(), t.end(), [](const TileTask& a, const TileTask& b) { return a.work > b.work; });
+// Replace segs[first..] by their union as runs of adjacent rows, in position order.
+// A run is causal if any of its parts is (the causal test is a no-op on parts that
+// lie wholly before the tile, so applying it to the whole run changes nothing).
+void coalesce_tail(std::vector<Seg>& segs, size_t first) {
+  std::vector<Seg> part(segs.begin() + first, segs.end());
+  std::sort(part.begin(), part.end(), [](const Seg& a, const Seg& b) { return a.row0 < b.row0; });
+  segs.resize(first);
+  for (const Seg& s : part) {
+    if (segs.size() > first) {
+      Seg& t = segs.back();
+      if (t.row0 + t.rows == s.row0 && t.pos0 + t.rows == s.pos0) {
+        t.rows += s.rows;
+        t.flags |= (s.flags & kSegCausal);
+        continue;
+      }
+    }
+    segs.push_back(s);
+  }
+  if (segs.size() > first) segs[first].flags |= kSegBlockStart;
+}
+
+// Expands every tile (whose `head` field holds its group, e.g. its document) into one
+// task per head, ordered so that tasks sharing operands run side by side: groups by
+// descending total work, inside a group head by head (heads of one GQA group are
+// adjacent), inside a head tiles by descending work.  Consecutive CTAs then reuse the
+// same k/v (forward) or q/dO and dq rows (backward) from L2, and the largest pieces
+// start first.
+void expand_heads(std::vector<TileTask>& tiles, int32_t heads) {
+  std::map<int32_t, std::vector<TileTask>> groups;
+  std::map<int32_t, int64_t> total;
+  for (const TileTask& t : tiles) {
+    groups[t.head].push_back(t);
+    total[t.head] += t.work;
+  }
+  std::vector<int32_t> order;
+  for (auto& kv : groups) order.push_back(kv.first);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return total[a] > total[b]; });
+  std::vector<TileTask> out;
+  out.reserve(tiles.size() * (size_t)heads);
+  for (int32_t g : order) {
+    auto& v = groups[g];
+    std::stable_sort(v.begin(), v.end(), [](const TileTask& a, const TileTask& b) { return a.work > b.work; });
+    for (int32_t h = 0; h < heads; ++h)
+      for (TileTask t : v) {
+        t.head = h;
+        out.push_back(t);
+      }
+  }
+  tiles.swap(out);
 }
 
 }  // namespace
@@ -172,8 +219,7 @@ std::vector<ChunkPair> ring_chunk_pairs(const int32_t* cu, int32_t num_docs, int
 }
 
 Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t heads,
-                   int32_t only_step, int32_t tile_m) {
-  (void)heads;
+                   int32_t only_step, int32_t tile_m, bool coalesce) {
   Plan plan;
   const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
   std::vector<ChunkPair> pairs = ring_chunk_pairs(cu, num_docs, cp, layout, window, only_step);
@@ -200,6 +246,7 @@ Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       last_step = p.step;
       plan.segs.push_back(s);
     }
+    if (coalesce) coalesce_tail(plan.segs, seg0);
     const int32_t nseg = (int32_t)plan.segs.size() - seg0;
     for (int32_t t0 = 0; t0 < c; t0 += tile_m) {
       TileTask t{};
@@ -209,6 +256,7 @@ Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       t.seg0 = seg0;
       t.nseg = nseg;
       t.aux = -1;
+      t.head = d;
       int64_t w = 0;
       for (int32_t i = 0; i < nseg; ++i) {
         const Seg& s = plan.segs[seg0 + i];
@@ -218,13 +266,12 @@ Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       plan.tasks.push_back(t);
     }
   }
-  sort_tasks(plan.tasks);
+  expand_heads(plan.tasks, heads);
   return plan;
 }
 
 Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t kv_heads,
                    int32_t tile_n) {
-  (void)kv_heads;
   Plan plan;
   const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
   std::vector<ChunkPair> pairs = ring_chunk_pairs(cu, num_docs, cp, layout, window, -1);
@@ -248,6 +295,7 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       s.flags = (p.causal ? kSegCausal : 0) | kSegBlockStart;
       plan.segs.push_back(s);
     }
+    coalesce_tail(plan.segs, seg0);
     const int32_t nseg = (int32_t)plan.segs.size() - seg0;
     for (int32_t t0 = 0; t0 < c; t0 += tile_n) {
       TileTask t{};
@@ -257,6 +305,7 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       t.seg0 = seg0;
       t.nseg = nseg;
       t.aux = -1;
+      t.head = d;
       int64_t w = 0;
       for (int32_t i = 0; i < nseg; ++i) {
         const Seg& s = plan.segs[seg0 + i];
@@ -266,13 +315,12 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       plan.tasks.push_back(t);
     }
   }
-  sort_tasks(plan.tasks);
+  expand_heads(plan.tasks, kv_heads);
   return plan;
 }
 
 Plan plan_block_fwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qbase, const int32_t* kbase,
                     int32_t num_docs, bool causal, int32_t window, int32_t heads, int32_t tile_m) {
-  (void)heads;
   Plan plan;
   for (int32_t d = 0; d < num_docs; ++d) {
     const int32_t lq = cu_q[d + 1] - cu_q[d], lk = cu_k[d + 1] - cu_k[d];
@@ -290,17 +338,17 @@ Plan plan_block_fwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qba
       t.seg0 = seg0;
       t.nseg = nseg;
       t.aux = -1;
+      t.head = d;
       t.work = nseg ? weight(visible_pairs(t.pos0, t.rows, kb, lk, causal, window)) : 0;
       plan.tasks.push_back(t);
     }
   }
-  sort_tasks(plan.tasks);
+  expand_heads(plan.tasks, heads);
   return plan;
 }
 
 Plan plan_block_bwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qbase, const int32_t* kbase,
                     int32_t num_docs, bool causal, int32_t window, int32_t kv_heads, int32_t tile_n) {
-  (void)kv_heads;
   Plan plan;
   for (int32_t d = 0; d < num_docs; ++d) {
     const int32_t lq = cu_q[d + 1] - cu_q[d], lk = cu_k[d + 1] - cu_k[d];
@@ -318,17 +366,17 @@ Plan plan_block_bwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qba
       t.seg0 = seg0;
       t.nseg = nseg;
       t.aux = -1;
+      t.head = d;
       t.work = nseg ? weight(visible_pairs(qb, lq, t.pos0, t.rows, causal, window)) : 0;
       plan.tasks.push_back(t);
     }
   }
-  sort_tasks(plan.tasks);
+  expand_heads(plan.tasks, kv_heads);
   return plan;
 }
 
 Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int32_t seg_size, KvMode mode,
               int32_t block_size, int32_t global_q_offset, int32_t window, bool per_shard, int32_t tile_m) {
-  (void)heads;
   Plan plan;
   const int64_t q_lo = global_q_offset, q_hi = (int64_t)global_q_offset + q_len - 1;
   std::vector<int32_t> shard_seg0(shards), shard_nseg(shards);
@@ -358,6 +406,7 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
       t.seg0 = per_shard ? shard_seg0[r] : 0;
       t.nseg = per_shard ? shard_nseg[r] : (int32_t)plan.segs.size();
       t.aux = per_shard ? r : -1;
+      t.head = 0;
       // weight: visible keys of the tile (every key position below the tile is one page of some shard)
       int64_t lo = window > 0 ? std::max<int64_t>(0, pos0 - window + 1) : 0;
       int64_t span = (int64_t)pos0 + rows - lo;
@@ -365,7 +414,7 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
       plan.tasks.push_back(t);
     }
   }
-  sort_tasks(plan.tasks);
+  expand_heads(plan.tasks, heads);
   return plan;
 }
 

@@ -25,7 +25,7 @@ struct TileTask {
   int32_t seg0;  // first streamed segment of this tile
   int32_t nseg;  // number of streamed segments
   int32_t aux;   // paged prefill: shard of the single-shard variant (-1 = all shards)
-  int32_t head;  // head index (q head in the forward, kv head in the backward)
+  int32_t head;  // head (q head in the forward, kv head in the backward); one task per tile and head
   int32_t work;  // estimated visible pairs / 256 (scheduling weight)
 };
 
@@ -72,12 +72,15 @@ struct Plan {
   std::vector<Seg> segs;
 };
 
-// Forward over the ring: one task per 128-row q tile per head, segments = the k chunks
-// of every block the tile's chunk meets, in ring-step order (only_step >= 0: that step only).
+// Forward over the ring: one task per 128-row q tile (inside one chunk, i.e. one virtual
+// rank's rows) per head; segments = the k chunks of every block the tile's chunk meets, in
+// ring-step order (only_step >= 0: that step only).  With `coalesce`, chunks that sit next
+// to each other in memory are visited as one run, in position order: the same (q, k) pairs,
+// merged on chip in a different order, with fewer ragged k tiles.
 Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t heads,
-                   int32_t only_step, int32_t tile_m);
+                   int32_t only_step, int32_t tile_m, bool coalesce);
 // Backward over the ring: one task per 128-row k tile per kv head, segments = the q chunks
-// that meet the tile's chunk (all blocks), in ring order.
+// that meet the tile's chunk (all blocks), coalesced into runs of adjacent rows.
 Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t kv_heads,
                    int32_t tile_n);
 // One varlen block with explicit per-document positions.
