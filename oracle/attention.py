@@ -293,3 +293,85 @@ def brute_force_attention(q, k, v, qpos, kpos, qdoc, kdoc, scale, causal, window
                 for t in range(dv):
                     out[i][h][t] += p * float(v[j][kh][t])
     return np.asarray(out), np.asarray(lse)
+
+
+# --------------------------------------------------------------------------- subsets (large inputs)
+
+def _row_stats(q, k, v, qpos, kpos, qdoc, kdoc, i, h, kh, scale, causal, window, lse_i):
+    """Visible key indices, P row and scores of one query row against all keys."""
+    m = visible(qpos[i:i + 1], kpos, qdoc[i:i + 1], kdoc, causal, window)[0]
+    j = np.nonzero(m)[0]
+    s = scale * (k[j, kh] @ q[i, h])
+    p = np.exp(s - lse_i) if np.isfinite(lse_i) else np.zeros_like(s)
+    return j, p
+
+
+def attention_grad_rows(dout, q, k, v, out, lse, cu_q, cu_k, scale, rows, heads, causal=True, window=0,
+                        qpos=None, kpos=None):
+    """``dq`` of the given query rows and heads (``[len(rows), len(heads), D]``).
+
+    The same definition as :func:`attention_bwd`, evaluated row by row:
+    ``dq_i = scale * sum_j P_ij (<dO_i, v_j> - Delta_i) k_j`` with
+    ``P_ij = exp(scale <q_i, k_j> - lse_i)`` and ``Delta_i = <dO_i, out_i>``.
+    ``out`` and ``lse`` are needed only at the given rows.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    nq, hq, d = q.shape
+    nk, hkv, _ = k.shape
+    if qpos is None or kpos is None:
+        dq_, dk_ = default_positions(cu_q, cu_k)
+        qpos = dq_ if qpos is None else qpos
+        kpos = dk_ if kpos is None else kpos
+    qdoc, kdoc = doc_ids(cu_q, nq), doc_ids(cu_k, nk)
+    res = np.zeros((len(rows), len(heads), d))
+    for a, i in enumerate(rows):
+        for b, h in enumerate(heads):
+            kh = _kv_head(h, hq, hkv)
+            do = np.asarray(dout[i, h], np.float64)
+            j, p = _row_stats(q, k, v, np.asarray(qpos), np.asarray(kpos), qdoc, kdoc, i, h, kh, scale, causal,
+                              window, float(lse[h, i]))
+            delta = float(do @ np.asarray(out[i, h], np.float64))
+            ds = p * (v[j, kh] @ do - delta)
+            res[a, b] = scale * (ds @ k[j, kh])
+    return res
+
+
+def attention_grad_cols(dout, q, k, v, out, lse, cu_q, cu_k, scale, cols, heads, causal=True, window=0,
+                        qpos=None, kpos=None):
+    """``(dk, dv)`` of the given key rows for the given q heads' contributions.
+
+    ``dv_j = sum_i P_ij dO_i`` and ``dk_j = scale * sum_i P_ij (<dO_i, v_j> - Delta_i) q_i``
+    over every query row i that sees key j; ``out``/``lse`` must be exact at those rows.
+    Returns arrays ``[len(cols), len(heads), D]`` (one entry per q head; a kv head's
+    gradient is the sum over its q heads).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    nq, hq, d = q.shape
+    nk, hkv, _ = k.shape
+    if qpos is None or kpos is None:
+        dq_, dk_ = default_positions(cu_q, cu_k)
+        qpos = dq_ if qpos is None else qpos
+        kpos = dk_ if kpos is None else kpos
+    qpos, kpos = np.asarray(qpos), np.asarray(kpos)
+    qdoc, kdoc = doc_ids(cu_q, nq), doc_ids(cu_k, nk)
+    dk = np.zeros((len(cols), len(heads), d))
+    dv = np.zeros((len(cols), len(heads), d))
+    for a, j in enumerate(cols):
+        m = visible(qpos, kpos[j:j + 1], qdoc, kdoc[j:j + 1], causal, window)[:, 0]
+        i = np.nonzero(m)[0]
+        for b, h in enumerate(heads):
+            kh = _kv_head(h, hq, hkv)
+            l = np.asarray(lse[h, i], np.float64)
+            fin = np.isfinite(l)
+            s = scale * (q[i, h] @ k[j, kh])
+            p = np.where(fin, np.exp(s - np.where(fin, l, 0.0)), 0.0)
+            do = np.asarray(dout[i, h], np.float64)
+            delta = (do * np.asarray(out[i, h], np.float64)).sum(axis=1)
+            ds = p * (do @ v[j, kh] - delta)
+            dv[a, b] = p @ do
+            dk[a, b] = scale * (ds @ q[i, h])
+    return dk, dv

@@ -210,3 +210,19 @@ def test_rows_subset_matches_full():
     so, sl = A.attention_fwd(q, k, v, cu, cu, 0.3, causal=True, rows=rows)
     np.testing.assert_allclose(so[rows], fo[rows], atol=1e-14)
     np.testing.assert_allclose(sl[:, rows], fl[:, rows], atol=1e-14)
+
+
+def test_row_and_column_gradient_subsets_match_the_full_backward():
+    cu = cu_from_lengths([40, 56])
+    q, k, v, do = _inputs(14, 96, 4, 2, 8)
+    out, lse = A.attention_fwd(q, k, v, cu, cu, 0.3, causal=True, window=17)
+    dq, dk, dv = A.attention_bwd(do, q, k, v, out, lse, cu, cu, 0.3, causal=True, window=17)
+    rows, heads = [0, 5, 39, 40, 95], [0, 3]
+    gq = A.attention_grad_rows(do, q, k, v, out, lse, cu, cu, 0.3, rows, heads, causal=True, window=17)
+    np.testing.assert_allclose(gq, dq[np.ix_(rows, heads)], atol=1e-12)
+    cols = [0, 20, 39, 40, 90]
+    gk, gv = A.attention_grad_cols(do, q, k, v, out, lse, cu, cu, 0.3, cols, [0, 1, 2, 3], causal=True, window=17)
+    # kv head h gathers q heads 2h and 2h+1
+    for kh in range(2):
+        np.testing.assert_allclose(gk[:, 2 * kh] + gk[:, 2 * kh + 1], dk[cols, kh], atol=1e-12)
+        np.testing.assert_allclose(gv[:, 2 * kh] + gv[:, 2 * kh + 1], dv[cols, kh], atol=1e-12)
