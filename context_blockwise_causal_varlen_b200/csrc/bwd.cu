@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   using L = BwdSmem<D>;
   constexpr int KH = D / 64;  // 64-column halves
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = align_smem_1024(smem_raw);
   uint8_t* sK = sm + L::kK;
   uint8_t* sV = sm + L::kV;
   uint8_t* sQ = sm + L::kQ;
@@ -206,8 +206,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       constexpr uint32_t id_st = idesc_bf16(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
       constexpr uint32_t id_kv = idesc_bf16(BN, D, false, true);     // dV, dK: 128 x D, K = 64
       constexpr uint32_t id_dq = idesc_bf16(D, BM, true, true);      // dQ^T: D x 64, K = 128
-      const uint32_t k0 = smem_u32(sK), v0 = smem_u32(sV), q0 = smem_u32(sQ), do0 = smem_u32(sDO);
-      const uint32_t pt0 = smem_u32(sPt), ds0 = smem_u32(sDSt);
+      // base descriptors, built once; per-instruction offsets are compile-time constants
+      const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);        // K as K-major A (S^T)
+      const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);        // V as K-major A (dP^T)
+      const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);    // K^T as MN-major A (dQ^T)
+      const uint64_t dPt = sdesc_sw128(smem_u32(sPt), 16, 1024);        // P^T, K-major A (dV)
+      const uint64_t dDSt = sdesc_sw128(smem_u32(sDSt), 16, 1024);      // dS^T, K-major A (dK)
+      const uint64_t dDSt_mn = sdesc_sw128(smem_u32(sDSt), 16384, 1024);  // dS^T, MN-major B (dQ^T)
+      // stage s of q / dO sits s * kQT bytes after stage 0
+      const uint64_t dQ_k = sdesc_sw128(smem_u32(sQ), 16, 1024);       // q as K-major B (S^T)
+      const uint64_t dO_k = sdesc_sw128(smem_u32(sDO), 16, 1024);      // dO as K-major B (dP^T)
+      const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 8192, 1024);    // q as MN-major B (dK)
+      const uint64_t dO_mn = sdesc_sw128(smem_u32(sDO), 8192, 1024);   // dO as MN-major B (dV)
       bool ok = mbar_wait(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_sdp = [&](int j) -> bool {
@@ -215,12 +225,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!mbar_wait(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutMma)) return false;
         if (!mbar_wait(&bar[bSFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) return false;
         tc_fence_after();
+        const uint64_t bq = sdesc_add(dQ_k, st * L::kQT), bo = sdesc_add(dO_k, st * L::kQT);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t bo = st * L::kQT + (kk >> 2) * 8192 + (kk & 3) * 32;
-          umma_bf16_ss(tS, sdesc_sw128(k0 + ao, 16, 1024), sdesc_sw128(q0 + bo, 16, 1024), id_st, kk > 0);
-          umma_bf16_ss(tDP, sdesc_sw128(v0 + ao, 16, 1024), sdesc_sw128(do0 + bo, 16, 1024), id_st, kk > 0);
+          const uint32_t bb = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_bf16_ss(tS, sdesc_add(dK_k, ao), sdesc_add(bq, bb), id_st, kk > 0);
+          umma_bf16_ss(tDP, sdesc_add(dV_k, ao), sdesc_add(bo, bb), id_st, kk > 0);
         }
         umma_commit(&bar[bSFull]);
         return true;
@@ -240,23 +251,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (j + 1 < n && !(ok = issue_sdp(j + 1))) break;
         if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
+        const uint64_t omn = sdesc_add(dO_mn, st * L::kQT), qmn = sdesc_add(dQ_mn, st * L::kQT);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint64_t pa = sdesc_sw128(pt0 + kk * 32, 16, 1024);
-          const uint64_t da = sdesc_sw128(ds0 + kk * 32, 16, 1024);
-          const uint64_t ob = sdesc_sw128(do0 + st * L::kQT + kk * 2048, 8192, 1024);
-          const uint64_t qb = sdesc_sw128(q0 + st * L::kQT + kk * 2048, 8192, 1024);
-          umma_bf16_ss(tDV, pa, ob, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_bf16_ss(tDK, da, qb, id_kv, (j > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16_ss(tDV, sdesc_add(dPt, kk * 32), sdesc_add(omn, kk * 2048), id_kv, acc);
+          umma_bf16_ss(tDK, sdesc_add(dDSt, kk * 32), sdesc_add(qmn, kk * 2048), id_kv, acc);
         }
         if (!mbar_wait(&bar[bDQFree + db], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t tdq = tDQ0 + db * 64;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t ka = sdesc_sw128(k0 + kk * 2048, 16384, 1024);
-          const uint64_t sb = sdesc_sw128(ds0 + kk * 2048, 16384, 1024);
-          umma_bf16_ss(tDQ0 + db * 64, ka, sb, id_dq, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ss(tdq, sdesc_add(dK_mn, kk * 2048), sdesc_add(dDSt_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
         umma_commit(&bar[bQEmpty + st]);
         umma_commit(&bar[bPtFree]);
         umma_commit(&bar[bDQFull + db]);

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   constexpr int KS = D / 16;  // k16 steps over the head dim
   constexpr int ND = D / 8;   // n8 blocks over the head dim
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = align_smem_1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint64_t* empty = full + kDecStages;
 

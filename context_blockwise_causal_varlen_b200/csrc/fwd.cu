@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   using L = FwdSmem<D>;
   constexpr int QH = D / 64;  // 64-column halves of a D-wide tile
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = align_smem_1024(smem_raw);
   uint8_t* sQ = sm + L::kQ;
   uint8_t* sK = sm + L::kK;
   uint8_t* sV = sm + L::kV;
@@ -217,7 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
-      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV), p0 = smem_u32(sP);
+      // base descriptors, built once; per-instruction offsets are compile-time constants
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);      // stage s at + s * kTileBytes
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
       bool ok = mbar_wait(&bar[bQFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_pv = [&](int j) -> bool {
@@ -225,12 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) return false;
         if (!mbar_wait(&bar[bVFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
         tc_fence_after();
+        const uint64_t dv = sdesc_add(dV0, st * L::kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(p0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(v0 + st * L::kTileBytes + kk * 2048, 16384, 1024);
-          umma_bf16_ss(tO, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ss(tO, sdesc_add(dP, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(dv, kk * 2048), idesc_o,
+                       (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bar[bVEmpty + st]);
         umma_commit(&bar[bPVDone]);
         return true;
@@ -244,12 +247,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (!mbar_wait(&bar[bKFull + st], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
         if (!mbar_wait(&bar[bSFree + st], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
+        const uint64_t dk = sdesc_add(dK0, st * L::kTileBytes);
+        const uint32_t ts = tS0 + st * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(q0 + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k0 + st * L::kTileBytes + off, 16, 1024);
-          umma_bf16_ss(tS0 + st * 128, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(ts, sdesc_add(dQ, off), sdesc_add(dk, off), idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bar[bKEmpty + st]);
         umma_commit(&bar[bSFull + st]);

@@ -29,6 +29,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory base rounded up to 1024 bytes (128B-swizzle atoms and TMA
+// destinations need it).  Pointer arithmetic on the extern __shared__ array keeps the
+// shared address space visible to the compiler, so accesses compile to shared loads
+// and stores rather than generic ones.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -195,6 +203,11 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= (uint64_t)2 << 61;  // SWIZZLE_128B
   return d;
 }
+
+// Descriptor of the same layout `bytes` further on: the start address is a 14-bit
+// field in 16-byte units at the bottom of the descriptor, and shared-memory
+// addresses stay below 256 KB, so adding never carries out of the field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
 
 __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
