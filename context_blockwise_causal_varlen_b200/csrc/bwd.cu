@@ -303,32 +303,42 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tmem_ld32(tS + lane_base + c0, s);
         tmem_ld32(tDP + lane_base + c0, dp);
         tmem_ld_wait();
-        // this key row sees the q columns [lo, hi] (positions are linear in the column)
-        int32_t lo = 0, hi = BM - 1;
-        if (r.need_mask) {
-          hi = kvalid ? r.nvalid - 1 : -1;
+        // S^T / dP^T are in registers: release the TMEM buffers so the next tile's
+        // S^T and dP^T can be computed while this one is being turned into P and dS
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[bSFree]);
+        if (!r.need_mask) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -lrow[c]));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -lrow[c + 1]));
+            pp[c / 2] = pack_bf16x2(p0, p1);
+            pd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - drow[c]),
+                                    p1 * (__uint_as_float(dp[c + 1]) - drow[c + 1]));
+          }
+        } else {
+          // this key row sees the q columns [lo, hi] (positions are linear in the column)
+          int32_t hi = kvalid ? r.nvalid - 1 : -1, lo = 0;
           if (r.causal || W > 0) lo = max(lo, kpos - r.qpos0);
           if (W > 0) hi = min(hi, kpos + W - 1 - r.qpos0);
-        }
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float pv[2], dv[2];
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], dv[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = c0 + c + e;
-            const bool vis = col >= lo && col <= hi;
-            const float pe = vis ? ex2_approx(fmaf(__uint_as_float(s[c + e]), sl2, -lrow[c + e])) : 0.f;
-            pv[e] = pe;
-            // rows past the segment hold whatever the row buffer holds: keep them out of dS
-            dv[e] = vis ? pe * (__uint_as_float(dp[c + e]) - drow[c + e]) : 0.f;
+            for (int e = 0; e < 2; ++e) {
+              const int col = c0 + c + e;
+              const bool vis = col >= lo && col <= hi;
+              const float pe = vis ? ex2_approx(fmaf(__uint_as_float(s[c + e]), sl2, -lrow[c + e])) : 0.f;
+              pv[e] = pe;
+              // rows past the segment hold whatever the row buffer holds: keep them out of dS
+              dv[e] = vis ? pe * (__uint_as_float(dp[c + e]) - drow[c + e]) : 0.f;
+            }
+            pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
+            pd[c / 2] = pack_bf16x2(dv[0], dv[1]);
           }
-          pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
-          pd[c / 2] = pack_bf16x2(dv[0], dv[1]);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[bSFree]);
       if (j > 0 && !mbar_wait_warp(&bar[bPtFree], (j - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
