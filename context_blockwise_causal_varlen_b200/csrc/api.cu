@@ -36,6 +36,7 @@ int cuda_fail(int err, const char* what) {
 }
 
 constexpr size_t kAlign = 256;
+constexpr int32_t kPairRows = 256;  // q rows per forward task: two 128-row tiles
 constexpr size_t kStatusBytes = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -191,13 +192,14 @@ RingFwdLayout ring_fwd_layout(const cbv_ring_args* a) {
   Carve c(nullptr);
   c.take(kStatusBytes);
   if (a->schedule == CBV_SCHEDULE_FUSED) {
-    L.fused = plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, -1, 128,
-                            true);
+    L.fused = plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, -1,
+                            kPairRows, true);
     carve_plan(c, L.fused);
   } else {
     for (int s = 0; s < a->cp; ++s) {
       L.steps.push_back(
-          plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, s, 128, false));
+          plan_ring_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, s, kPairRows,
+                        false));
       carve_plan(c, L.steps.back());
     }
     c.take((size_t)a->total * a->num_heads * a->head_dim * sizeof(float));  // running out (fp32)
@@ -340,7 +342,7 @@ static int block_fwd_checks(const cbv_block_fwd_args* a) {
 size_t cbv_block_fwd_workspace_size(const cbv_block_fwd_args* a) {
   if (block_fwd_checks(a)) return 0;
   Plan p = plan_block_fwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs, a->causal != 0,
-                          a->window, a->num_heads, 128);
+                          a->window, a->num_heads, kPairRows);
   Carve c(nullptr);
   c.take(kStatusBytes);
   carve_plan(c, p);
@@ -355,7 +357,7 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
     return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   Plan plan = plan_block_fwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs,
-                             a->causal != 0, a->window, H, 128);
+                             a->causal != 0, a->window, H, kPairRows);
   Carve c(a->workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, plan);
@@ -385,7 +387,7 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   if ((rc = upload_plan(pd, plan, s))) return rc;
   const int grid = grid_of(plan.tasks.size(), 1);
   if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
-  return launch_rc(launch_fwd(p, D, false, grid, s), "block forward launch");
+  return launch_rc(launch_fwd_pingpong(p, D, grid, s), "block forward launch");
 }
 
 // ------------------------------------------------------------------------ merge
@@ -431,7 +433,7 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
     p.num_tasks = (int)L.fused.tasks.size();
     p.out = a->out;
     p.out_mode = kOutBf16;
-    return launch_rc(launch_fwd(p, D, false, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch");
+    return launch_rc(launch_fwd_pingpong(p, D, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch");
   }
   std::vector<PlanDev> pds;
   for (auto& pl : L.steps) {
@@ -445,7 +447,7 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
     p.num_tasks = (int)L.steps[st].tasks.size();
     p.out = acc;
     p.out_mode = st == 0 ? kOutF32 : kOutMerge;
-    if ((rc = launch_rc(launch_fwd(p, D, false, grid_of(L.steps[st].tasks.size(), 1), s), "ring step launch")))
+    if ((rc = launch_rc(launch_fwd_pingpong(p, D, grid_of(L.steps[st].tasks.size(), 1), s), "ring step launch")))
       return rc;
   }
   return launch_rc(launch_convert_bf16(acc, a->out, a->total * H * D, 1.f, s), "output conversion");

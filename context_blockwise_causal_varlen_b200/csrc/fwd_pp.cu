@@ -1,0 +1,424 @@
+// Block forward on tcgen05, two q tiles per CTA ("ping-pong").
+//
+// Same operation as fwd.cu (the per-block flash forward of the NeMo AutoModel
+// zig-zag ring page, _block_forward, with the blocks of a tile merged by the
+// online-softmax identity, update_out_and_lse, on chip), organised so that the
+// tensor core never waits for one softmax: a CTA owns two 128-row q tiles A and B
+// of the same head that stream the same k/v tiles.  While warpgroup A turns S_A
+// into P_A, the tensor core computes S_B or PV_B, and the other way round.
+//
+// P never leaves TMEM: the softmax writes P (bf16, two per 32-bit column) over the
+// S columns it has just read, and PV takes its A operand from TMEM.
+//
+// Warps: 0 TMA producer, 1 UMMA issuer (+ TMEM owner), 2-5 softmax / epilogue of
+// tile A, 6-9 softmax / epilogue of tile B.  TMEM columns: S_A (and P_A) [0,128),
+// S_B (and P_B) [128,256), O_A [256, 256+D), O_B [256+D, 256+2D).
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace cbv {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int kThreads = 320;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: keep a stale max while it is within 2^8
+
+struct KTile {
+  int32_t k_row, kpos0, nvalid, causal;
+};
+
+struct KIter {
+  int32_t si = 0, j = 0, jn = 0;
+  Seg seg;
+};
+
+// k tiles that at least one row of q positions [qp0, qp1] can see (non-paged).
+__device__ __forceinline__ bool next_ktile(const FwdParams& p, const TileTask& t, int32_t qp0, int32_t qp1,
+                                           KIter& it, KTile& r) {
+  const int32_t W = p.window;
+  while (true) {
+    if (it.j >= it.jn) {
+      if (it.si >= t.nseg) return false;
+      it.seg = p.segs[t.seg0 + it.si];
+      it.si++;
+      const bool cz = (it.seg.flags & kSegCausal) || W > 0;
+      int32_t cmax = it.seg.rows - 1, cmin = 0;
+      if (cz) cmax = min(cmax, qp1 - it.seg.pos0);
+      if (W > 0) cmin = max(0, qp0 - W + 1 - it.seg.pos0);
+      if (cmax < cmin) {
+        it.j = it.jn = 0;
+        continue;
+      }
+      it.j = cmin / BN;
+      it.jn = cmax / BN + 1;
+    }
+    const int32_t c0 = it.j++ * BN;
+    r.nvalid = min(BN, it.seg.rows - c0);
+    r.k_row = it.seg.row0 + c0;
+    r.kpos0 = it.seg.pos0 + c0;
+    r.causal = it.seg.flags & kSegCausal;
+    return true;
+  }
+}
+
+template <int D>
+struct PPSmem {
+  static constexpr uint32_t kTile = BM * D * 2;  // a 128 x D bf16 tile
+  static constexpr uint32_t kQ = 0;              // Q_A, Q_B
+  static constexpr uint32_t kK = kQ + 2 * kTile; // 2 stages
+  static constexpr uint32_t kV = kK + 2 * kTile; // 2 stages
+  static constexpr uint32_t kBars = kV + 2 * kTile;
+  static constexpr uint32_t kEnd = kBars + 256;
+  static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
+  static_assert(kDynamic <= 232448, "shared memory budget");
+};
+
+enum PBar {
+  pQFull = 0,
+  pKFull = 1,    // +stage
+  pVFull = 3,    // +stage
+  pKEmpty = 5,   // +stage
+  pVEmpty = 7,   // +stage
+  pSFull = 9,    // +tile
+  pPFull = 11,   // +tile
+  pPVDone = 13,  // +tile
+  pODone = 15,
+  pNum = 16
+};
+
+// tcgen05.mma with the A operand (P) in tensor memory
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_constant__ FwdParams p) {
+  using L = PPSmem<D>;
+  constexpr int QH = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = align_smem_1024(smem_raw);
+  uint8_t* sQ = sm + L::kQ;
+  uint8_t* sK = sm + L::kK;
+  uint8_t* sV = sm + L::kV;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + pNum);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const TileTask t = p.tasks[blockIdx.x];
+  const int head = t.head;
+  const int kvh = head / p.heads_per_kv;
+  const bool has_b = t.rows > BM;
+  const int32_t qp0 = t.pos0, qp1 = t.pos0 + t.rows - 1;  // union of the two tiles
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[pQFull], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[pKFull + s], 1);
+      mbar_init(&bar[pVFull + s], 1);
+      mbar_init(&bar[pKEmpty + s], 1);
+      mbar_init(&bar[pVEmpty + s], 1);
+      mbar_init(&bar[pSFull + s], 1);
+      mbar_init(&bar[pPFull + s], 4);
+      mbar_init(&bar[pPVDone + s], 1);
+    }
+    mbar_init(&bar[pODone], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_q);
+      tma_prefetch_desc(&p.tm_k);
+      tma_prefetch_desc(&p.tm_v);
+      mbar_arrive_expect_tx(&bar[pQFull], (has_b ? 2 : 1) * L::kTile);
+      for (int x = 0; x < (has_b ? 2 : 1); ++x)
+        for (int h = 0; h < QH; ++h)
+          tma_load_3d(sQ + x * L::kTile + h * 16384, &p.tm_q, &bar[pQFull], h * 64, head, t.row0 + x * BM);
+      KIter it;
+      KTile r;
+      int i = 0;
+      while (next_ktile(p, t, qp0, qp1, it, r)) {
+        const int st = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        if (!mbar_wait(&bar[pKEmpty + st], ph ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
+        mbar_arrive_expect_tx(&bar[pKFull + st], L::kTile);
+        for (int h = 0; h < QH; ++h)
+          tma_load_3d(sK + st * L::kTile + h * 16384, &p.tm_k, &bar[pKFull + st], h * 64, kvh, r.k_row);
+        if (!mbar_wait(&bar[pVEmpty + st], ph ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
+        mbar_arrive_expect_tx(&bar[pVFull + st], L::kTile);
+        for (int h = 0; h < QH; ++h)
+          tma_load_3d(sV + st * L::kTile + h * 16384, &p.tm_v, &bar[pVFull + st], h * 64, kvh, r.k_row);
+        ++i;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
+      const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);      // tile x at + x * kTile
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);      // stage s at + s * kTile
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
+      int n = 0;
+      {
+        KIter c;
+        KTile r;
+        while (next_ktile(p, t, qp0, qp1, c, r)) ++n;
+      }
+      const int ntile = has_b ? 2 : 1;
+      bool ok = mbar_wait(&bar[pQFull], 0, p.status, kDevTimeoutMma);
+      tc_fence_after();
+      auto issue_s = [&](int x, int i) {
+        const uint64_t dq = sdesc_add(dQ0, x * L::kTile), dk = sdesc_add(dK0, (i & 1) * L::kTile);
+        const uint32_t ts = tmem + x * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16_ss(ts, sdesc_add(dq, off), sdesc_add(dk, off), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar[pSFull + x]);
+      };
+      auto issue_pv = [&](int x, int i) {
+        const uint64_t dv = sdesc_add(dV0, (i & 1) * L::kTile);
+        const uint32_t tp = tmem + x * 128, to = tmem + 256 + x * D;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts(to, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bar[pPVDone + x]);
+      };
+      if (ok && n > 0) {
+        ok = mbar_wait(&bar[pKFull], 0, p.status, kDevTimeoutMma);
+        tc_fence_after();
+        if (ok) {
+          for (int x = 0; x < ntile; ++x) issue_s(x, 0);
+          umma_commit(&bar[pKEmpty]);
+        }
+      }
+      for (int i = 0; ok && i < n; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        for (int x = 0; x < ntile && ok; ++x) {
+          if (!mbar_wait(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(x, i);
+          if (i + 1 < n) {
+            const int st1 = (i + 1) & 1;
+            if (!mbar_wait(&bar[pKFull + st1], ((i + 1) >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            // P_x(i) lives in the columns S_x(i+1) will overwrite: let PV_x(i) finish reading it first
+            if (!mbar_wait(&bar[pPVDone + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(x, i + 1);
+            if (x == ntile - 1) umma_commit(&bar[pKEmpty + st1]);
+          }
+        }
+        if (ok) umma_commit(&bar[pVEmpty + st]);
+      }
+      if (n > 0) umma_commit(&bar[pODone]);
+      else mbar_arrive(&bar[pODone]);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue (warps 2..9)
+    const int x = (warp - 2) >> 2;  // tile: 0 = A, 1 = B
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + x * 128 + lane_base;
+    const uint32_t tO = tmem + 256 + x * D + lane_base;
+    const int trow = x * BM + row;  // row within the pair
+    const int32_t qpos = t.pos0 + trow;
+    const int32_t xq0 = t.pos0 + x * BM, xq1 = min(t.pos0 + t.rows - 1, xq0 + BM - 1);
+    const float sl2 = p.scale_log2;
+    const int32_t W = p.window;
+    float m = -INFINITY, l = 0.f, lr = 0.f;
+    bool ok = true;
+    int i = 0;
+    if (x == 0 || has_b) {
+      KIter it;
+      KTile r;
+      while (next_ktile(p, t, qp0, qp1, it, r)) {
+        if (!mbar_wait_warp(&bar[pSFull + x], i & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t s[BN];
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) tmem_ld32(tS + c, s + c);
+        tmem_ld_wait();
+        // this tile's rows see the columns [lo, hi] of this k tile
+        const bool cz = r.causal || W > 0;
+        const int32_t kmin = r.kpos0, kmax = r.kpos0 + r.nvalid - 1;
+        const bool need_mask = !((r.nvalid == BN) && (!cz || kmax <= xq0) && (W <= 0 || xq1 - kmin < W));
+        float mx = -INFINITY;
+        if (need_mask) {
+          int32_t hi = r.nvalid - 1, lo = 0;
+          if (cz) hi = min(hi, qpos - r.kpos0);
+          if (W > 0) lo = max(lo, qpos - W + 1 - r.kpos0);
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const float v = (c >= lo && c <= hi) ? __uint_as_float(s[c]) * sl2 : -INFINITY;
+            s[c] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const float v = __uint_as_float(s[c]) * sl2;
+            s[c] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        }
+        float m_use = m, alpha = 1.f;
+        bool rescale_o = false;
+        if (mx > m + kRescaleThreshold) {
+          m_use = mx;
+          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - mx);
+          rescale_o = (m != -INFINITY);
+        }
+        const float msub = (m_use == -INFINITY) ? 0.f : m_use;
+        float rowsum = 0.f, rowsum_r = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2_approx(__uint_as_float(s[c]) - msub);
+          const float p1 = ex2_approx(__uint_as_float(s[c + 1]) - msub);
+          const uint32_t pb = pack_bf16x2(p0, p1);
+          rowsum += p0 + p1;
+          rowsum_r += __uint_as_float(pb << 16) + __uint_as_float(pb & 0xffff0000u);
+          pk[c / 2] = pb;
+        }
+        l = l * alpha + rowsum;
+        lr = lr * alpha + rowsum_r;
+        m = m_use;
+        // PV of the previous k tile must be done: O is rescaled and P overwrites its input
+        if (i > 0 && !mbar_wait_warp(&bar[pPVDone + x], (i - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c, o);
+          }
+        }
+        tmem_st32(tS, pk);
+        tmem_st32(tS + 32, pk + 32);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[pPFull + x]);
+        ++i;
+      }
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && (x == 0 || has_b) && mbar_wait_warp(&bar[pODone], 0, p.status, kDevTimeoutEpilogue)) {
+      tc_fence_after();
+      const bool has = (l > 0.f) && (m != -INFINITY);
+      const float inv_l = (has && lr > 0.f) ? 1.f / lr : 0.f;
+      const float lse_b = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
+      const bool valid = trow < t.rows;
+      const int64_t orow = (int64_t)(t.row0 + trow);
+      float* lse_ptr = p.lse + (int64_t)head * p.lse_stride_h + orow * p.lse_stride_t;
+      float wa = 0.f, wb = 1.f, lse_new = lse_b;
+      if (p.out_mode == kOutMerge && valid) {
+        const float lse_a = *lse_ptr;
+        const float mm = fmaxf(lse_a, lse_b);
+        if (mm == -INFINITY) {
+          wa = 1.f;
+          wb = 0.f;
+          lse_new = -INFINITY;
+        } else {
+          lse_new = mm + __logf(__expf(lse_a - mm) + __expf(lse_b - mm));
+          wa = __expf(lse_a - lse_new);
+          wb = __expf(lse_b - lse_new);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+        tmem_ld_wait();
+        if (!valid) continue;
+        if (!has) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (p.out_mode == kOutBf16) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.out_stride_t +
+                               (int64_t)head * p.out_stride_h + c;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + e) = v;
+          }
+        } else {
+          float* dst = reinterpret_cast<float*>(p.out) + orow * p.out_stride_t + (int64_t)head * p.out_stride_h + c;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float4 v;
+            v.x = __uint_as_float(o[e + 0]) * inv_l;
+            v.y = __uint_as_float(o[e + 1]) * inv_l;
+            v.z = __uint_as_float(o[e + 2]) * inv_l;
+            v.w = __uint_as_float(o[e + 3]) * inv_l;
+            if (p.out_mode == kOutMerge) {
+              const float4 a = *reinterpret_cast<const float4*>(dst + e);
+              v.x = a.x * wa + v.x * wb;
+              v.y = a.y * wa + v.y * wb;
+              v.z = a.z * wa + v.z * wb;
+              v.w = a.w * wa + v.w * wb;
+            }
+            *reinterpret_cast<float4*>(dst + e) = v;
+          }
+        }
+      }
+      if (valid) *lse_ptr = lse_new;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int D>
+int launch_pp_t(const FwdParams& p, int grid, cudaStream_t stream) {
+  auto kern = fwd_pp_kernel<D>;
+  const uint32_t smem = PPSmem<D>::kDynamic;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return (int)e;
+  kern<<<grid, kThreads, smem, stream>>>(p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_fwd_pingpong(const FwdParams& p, int head_dim, int grid, cudaStream_t stream) {
+  if (grid <= 0) return 0;
+  if (head_dim == 128) return launch_pp_t<128>(p, grid, stream);
+  if (head_dim == 64) return launch_pp_t<64>(p, grid, stream);
+  return (int)cudaErrorInvalidValue;
+}
+
+}  // namespace cbv
