@@ -16,7 +16,10 @@
 // Warps: 0 TMA producer (q, dO, lse*log2e and Delta rows of a 3-stage ring),
 // 1 UMMA issuer (+ TMEM owner), 2-9 P / dS in two warpgroups that split the 64
 // q columns (one key row per thread) and then the dV / dK epilogue, 10-13 dQ readout.
-// TMEM columns: S^T [0,64), dP^T [64,128), dQ^T x2 [128,256), dV [256,256+D), dK [384,384+D).
+// TMEM columns: S^T [0,64), dP^T [64,128), dQ^T [128,192), V [192, 192+D/2), dV [256,256+D),
+// dK [384,384+D).  V sits in TMEM (copied once from shared memory) as the A operand of
+// dP^T = V dO^T, so that product reads only dO from shared memory: the five UMMAs of a
+// q tile are limited by shared-memory bandwidth, and this one then needs a third of it.
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -114,10 +117,11 @@ enum BBar {
   bSFree = 8,
   bPFull = 9,
   bPtFree = 10,
-  bDQFull = 11,  // +buffer (2)
-  bDQFree = 13,  // +buffer (2)
-  bAccDone = 15,
-  bBNum = 16
+  bDQFull = 11,
+  bDQFree = 12,
+  bVTmem = 13,
+  bAccDone = 14,
+  bBNum = 15
 };
 
 
@@ -149,10 +153,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_init(&bar[bQFull + s], 1);
       mbar_init(&bar[bQEmpty + s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[bDQFull + s], 1);
-      mbar_init(&bar[bDQFree + s], 4);
-    }
+    mbar_init(&bar[bDQFull], 1);
+    mbar_init(&bar[bDQFree], 4);
+    mbar_init(&bar[bVTmem], 4);
     mbar_init(&bar[bSFull], 1);
     mbar_init(&bar[bSFree], 8);
     mbar_init(&bar[bPFull], 8);
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 64, tDQ0 = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+  const uint32_t tS = tmem, tDP = tmem + 64, tDQ = tmem + 128, tV = tmem + 192, tDV = tmem + 256, tDK = tmem + 384;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -208,7 +211,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       constexpr uint32_t id_dq = idesc_bf16(D, BM, true, true);      // dQ^T: D x 64, K = 128
       // base descriptors, built once; per-instruction offsets are compile-time constants
       const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);        // K as K-major A (S^T)
-      const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);        // V as K-major A (dP^T)
       const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);    // K^T as MN-major A (dQ^T)
       const uint64_t dPt = sdesc_sw128(smem_u32(sPt), 16, 1024);        // P^T, K-major A (dV)
       const uint64_t dDSt = sdesc_sw128(smem_u32(sDSt), 16, 1024);      // dS^T, K-major A (dK)
@@ -219,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 8192, 1024);    // q as MN-major B (dK)
       const uint64_t dO_mn = sdesc_sw128(smem_u32(sDO), 8192, 1024);   // dO as MN-major B (dV)
       bool ok = mbar_wait(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
+      ok = ok && mbar_wait(&bar[bVTmem], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_sdp = [&](int j) -> bool {
         const int st = j % NS;
@@ -231,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t bb = (kk >> 2) * 8192 + (kk & 3) * 32;
           umma_bf16_ss(tS, sdesc_add(dK_k, ao), sdesc_add(bq, bb), id_st, kk > 0);
-          umma_bf16_ss(tDP, sdesc_add(dV_k, ao), sdesc_add(bo, bb), id_st, kk > 0);
+          umma_bf16_ts(tDP, tV + kk * 8, sdesc_add(bo, bb), id_st, kk > 0);
         }
         umma_commit(&bar[bSFull]);
         return true;
@@ -247,7 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       if (ok && n > 0) ok = issue_sdp(0);
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % NS;
-        const int db = j & 1;  // dQ^T TMEM buffer
         if (j + 1 < n && !(ok = issue_sdp(j + 1))) break;
         if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
@@ -258,15 +260,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           umma_bf16_ss(tDV, sdesc_add(dPt, kk * 32), sdesc_add(omn, kk * 2048), id_kv, acc);
           umma_bf16_ss(tDK, sdesc_add(dDSt, kk * 32), sdesc_add(qmn, kk * 2048), id_kv, acc);
         }
-        if (!mbar_wait(&bar[bDQFree + db], ((j >> 1) & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait(&bar[bDQFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tdq = tDQ0 + db * 64;
+        const uint32_t tdq = tDQ;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           umma_bf16_ss(tdq, sdesc_add(dK_mn, kk * 2048), sdesc_add(dDSt_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
         umma_commit(&bar[bQEmpty + st]);
         umma_commit(&bar[bPtFree]);
-        umma_commit(&bar[bDQFull + db]);
+        umma_commit(&bar[bDQFull]);
       }
       (void)it;
       (void)r;
@@ -286,11 +288,29 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const int32_t W = p.window;
     const float sl2 = p.scale_log2;
     const uint32_t pt_row = smem_u32(sPt), ds_row = smem_u32(sDSt);
+    bool ok = true;
+    if (wg == 0) {
+      // V rows (this thread's key) from the swizzled tile into TMEM, as the A operand of dP^T
+      ok = mbar_wait_warp(&bar[bKVFull], 0, p.status, kDevTimeoutSoftmax);
+      if (ok) {
+        const uint32_t vrow = smem_u32(sV);
+#pragma unroll
+        for (int h = 0; h < KH; ++h) {
+          uint32_t vals[32];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) ld_shared_v4(vrow + h * 16384 + sw128_offset(krow, ch), vals + ch * 4);
+          tmem_st32(tV + lane_base + h * 32, vals);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[bVTmem]);
+    }
     QIter it;
     QTile r;
     int j = 0;
-    bool ok = true;
-    while (next_qtile(p, t, kvh, it, r)) {
+    while (ok && next_qtile(p, t, kvh, it, r)) {
       const int st = j % NS;
       if (!mbar_wait_warp(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
       if (!mbar_wait_warp(&bar[bSFull], j & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
@@ -408,16 +428,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     QTile r;
     int j = 0;
     while (next_qtile(p, t, kvh, it, r)) {
-      const int st = j & 1;
-      if (!mbar_wait_warp(&bar[bDQFull + st], (j >> 1) & 1, p.status, kDevTimeoutEpilogue)) break;
+      if (!mbar_wait_warp(&bar[bDQFull], j & 1, p.status, kDevTimeoutEpilogue)) break;
       tc_fence_after();
       uint32_t v[BM];
-      tmem_ld32(tDQ0 + st * 64 + lane_base, v);
-      tmem_ld32(tDQ0 + st * 64 + lane_base + 32, v + 32);
+      tmem_ld32(tDQ + lane_base, v);
+      tmem_ld32(tDQ + lane_base + 32, v + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[bDQFree + st]);
+      if (lane == 0) mbar_arrive(&bar[bDQFree]);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         if (lane == 0) bulk_wait_group_read<0>();  // this warp's previous reduce has read its region

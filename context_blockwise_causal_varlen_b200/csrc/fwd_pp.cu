@@ -89,17 +89,6 @@ enum PBar {
   pNum = 16
 };
 
-// tcgen05.mma with the A operand (P) in tensor memory
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_constant__ FwdParams p) {
   using L = PPSmem<D>;
