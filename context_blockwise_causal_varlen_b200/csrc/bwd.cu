@@ -14,7 +14,7 @@
 // reduce-add.
 //
 // Warps: 0 TMA producer (q, dO, lse*log2e and Delta rows of a 3-stage ring),
-// 1 UMMA issuer (+ TMEM owner), 2-9 P / dS in two warpgroups that split the 64
+// 1 UMMA issuer (+ TMEM owner; the whole warp runs the loop, one elected lane issues), 2-9 P / dS in two warpgroups that split the 64
 // q columns (one key row per thread) and then the dV / dK epilogue, 10-13 dQ readout.
 // TMEM columns: S^T [0,64), dP^T [64,128), dQ^T [128,192), V [192, 192+D/2), dV [256,256+D),
 // dK [384,384+D).  V sits in TMEM (copied once from shared memory) as the A operand of
@@ -33,6 +33,7 @@ constexpr int kThreads = 448;
 constexpr int NS = 3;     // q / dO / row stages
 constexpr int kRowBox = BM + 4;  // lse/Delta box: 68 floats from a 16-byte aligned start
 constexpr int kRowSlot = 96;     // floats per row buffer: 384 bytes keeps every TMA destination 128-byte aligned
+constexpr int kDQRows = 16;      // q rows per dQ bulk reduce (four per q tile)
 
 struct QTile {
   int32_t q_row;   // first q row
@@ -101,10 +102,17 @@ struct BwdSmem {
   static constexpr uint32_t kDO = kQ + NS * kQT;      // NS stages
   static constexpr uint32_t kPt = kDO + NS * kQT;
   static constexpr uint32_t kDSt = kPt + kPT;
-  static constexpr uint32_t kDQ = kDSt + kPT;             // fp32 staging: 4 warps x [32][D/4]
-  static constexpr uint32_t kRow = kDQ + (BM / 2) * D * 4;  // per stage: lse*log2e and Delta slots
+  static constexpr uint32_t kDQBuf = kDQRows * D * 4;     // fp32 staging buffer: 4 warps x [16][D/4]
+  static constexpr uint32_t kDQ = kDSt + kPT;              // two staging buffers
+  // P^T / dS^T are double-buffered.  The second pair lives in the V tile when it fits
+  // there (V is read from shared memory only once, to copy it into TMEM).
+  static constexpr bool kPdsInV = kKV >= 2 * kPT;
+  static constexpr uint32_t kX = kDQ + 2 * kDQBuf;         // second P^T / dS^T pair when not in V
+  static constexpr uint32_t kPt1 = kPdsInV ? kV : kX;
+  static constexpr uint32_t kDSt1 = kPt1 + kPT;
+  static constexpr uint32_t kRow = kX + (kPdsInV ? 0 : 2 * kPT);  // per stage: lse*log2e and Delta slots
   static constexpr uint32_t kBars = kRow + NS * 2 * kRowSlot * 4;
-  static constexpr uint32_t kEnd = kBars + 128;
+  static constexpr uint32_t kEnd = kBars + 256;
   static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
   static_assert(kDynamic <= 232448, "shared memory budget");
 };
@@ -116,12 +124,12 @@ enum BBar {
   bSFull = 7,
   bSFree = 8,
   bPFull = 9,
-  bPtFree = 10,
-  bDQFull = 11,
-  bDQFree = 12,
-  bVTmem = 13,
-  bAccDone = 14,
-  bBNum = 15
+  bPtFree = 10,  // +P^T / dS^T buffer (2)
+  bDQFull = 12,
+  bDQFree = 13,
+  bVTmem = 14,
+  bAccDone = 15,
+  bBNum = 16
 };
 
 
@@ -160,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     mbar_init(&bar[bSFree], 8);
     mbar_init(&bar[bPFull], 8);
     mbar_init(&bar[bPtFree], 1);
+    mbar_init(&bar[bPtFree + 1], 1);
     mbar_init(&bar[bAccDone], 1);
     fence_mbar_init();
   }
@@ -204,29 +213,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ UMMA issuer (whole warp, one lane issues)
+    {
       constexpr uint32_t id_st = idesc_bf16(BN, BM, false, false);   // S^T, dP^T: 128 x 64, K = D
       constexpr uint32_t id_kv = idesc_bf16(BN, D, false, true);     // dV, dK: 128 x D, K = 64
       constexpr uint32_t id_dq = idesc_bf16(D, BM, true, true);      // dQ^T: D x 64, K = 128
       // base descriptors, built once; per-instruction offsets are compile-time constants
       const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);        // K as K-major A (S^T)
       const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);    // K^T as MN-major A (dQ^T)
-      const uint64_t dPt = sdesc_sw128(smem_u32(sPt), 16, 1024);        // P^T, K-major A (dV)
-      const uint64_t dDSt = sdesc_sw128(smem_u32(sDSt), 16, 1024);      // dS^T, K-major A (dK)
-      const uint64_t dDSt_mn = sdesc_sw128(smem_u32(sDSt), 16384, 1024);  // dS^T, MN-major B (dQ^T)
+      // P^T / dS^T buffer b of 2 (q tile j uses buffer j & 1)
+      const uint64_t dPt[2] = {sdesc_sw128(smem_u32(sPt), 16, 1024),       // P^T, K-major A (dV)
+                               sdesc_sw128(smem_u32(sm + L::kPt1), 16, 1024)};
+      const uint64_t dDSt[2] = {sdesc_sw128(smem_u32(sDSt), 16, 1024),     // dS^T, K-major A (dK)
+                                sdesc_sw128(smem_u32(sm + L::kDSt1), 16, 1024)};
+      const uint64_t dDSt_mn[2] = {sdesc_sw128(smem_u32(sDSt), 16384, 1024),  // dS^T, MN-major B (dQ^T)
+                                   sdesc_sw128(smem_u32(sm + L::kDSt1), 16384, 1024)};
       // stage s of q / dO sits s * kQT bytes after stage 0
       const uint64_t dQ_k = sdesc_sw128(smem_u32(sQ), 16, 1024);       // q as K-major B (S^T)
       const uint64_t dO_k = sdesc_sw128(smem_u32(sDO), 16, 1024);      // dO as K-major B (dP^T)
       const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 8192, 1024);    // q as MN-major B (dK)
       const uint64_t dO_mn = sdesc_sw128(smem_u32(sDO), 8192, 1024);   // dO as MN-major B (dV)
-      bool ok = mbar_wait(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
-      ok = ok && mbar_wait(&bar[bVTmem], 0, p.status, kDevTimeoutMma);
+      bool ok = mbar_wait_warp(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
+      ok = ok && mbar_wait_warp(&bar[bVTmem], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_sdp = [&](int j) -> bool {
         const int st = j % NS;
-        if (!mbar_wait(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutMma)) return false;
-        if (!mbar_wait(&bar[bSFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait_warp(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait_warp(&bar[bSFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) return false;
         tc_fence_after();
         const uint64_t bq = sdesc_add(dQ_k, st * L::kQT), bo = sdesc_add(dO_k, st * L::kQT);
 #pragma unroll
@@ -251,29 +264,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % NS;
         if (j + 1 < n && !(ok = issue_sdp(j + 1))) break;
-        if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const uint64_t omn = sdesc_add(dO_mn, st * L::kQT), qmn = sdesc_add(dQ_mn, st * L::kQT);
+        const int pb = j & 1;
+        const uint64_t apt = pb ? dPt[1] : dPt[0], ads = pb ? dDSt[1] : dDSt[0];
+        const uint64_t bds = pb ? dDSt_mn[1] : dDSt_mn[0];
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16_ss(tDV, sdesc_add(dPt, kk * 32), sdesc_add(omn, kk * 2048), id_kv, acc);
-          umma_bf16_ss(tDK, sdesc_add(dDSt, kk * 32), sdesc_add(qmn, kk * 2048), id_kv, acc);
+          umma_bf16_ss(tDV, sdesc_add(apt, kk * 32), sdesc_add(omn, kk * 2048), id_kv, acc);
+          umma_bf16_ss(tDK, sdesc_add(ads, kk * 32), sdesc_add(qmn, kk * 2048), id_kv, acc);
         }
-        if (!mbar_wait(&bar[bDQFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[bDQFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tdq = tDQ;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ss(tdq, sdesc_add(dK_mn, kk * 2048), sdesc_add(dDSt_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tdq, sdesc_add(dK_mn, kk * 2048), sdesc_add(bds, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
         umma_commit(&bar[bQEmpty + st]);
-        umma_commit(&bar[bPtFree]);
+        umma_commit(&bar[bPtFree + pb]);
         umma_commit(&bar[bDQFull]);
       }
       (void)it;
       (void)r;
       if (n > 0) umma_commit(&bar[bAccDone]);
-      else mbar_arrive(&bar[bAccDone]);
+      else if (lane == 0) mbar_arrive(&bar[bAccDone]);
     }
   } else if (warp < 10) {
     // ------------------------------------------------------------------ P / dS (thread = key row)
@@ -287,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const bool kvalid = krow < t.rows;
     const int32_t W = p.window;
     const float sl2 = p.scale_log2;
-    const uint32_t pt_row = smem_u32(sPt), ds_row = smem_u32(sDSt);
+    const uint32_t pt_buf[2] = {smem_u32(sPt), smem_u32(sm + L::kPt1)};
+    const uint32_t ds_buf[2] = {smem_u32(sDSt), smem_u32(sm + L::kDSt1)};
     bool ok = true;
     if (wg == 0) {
       // V rows (this thread's key) from the swizzled tile into TMEM, as the A operand of dP^T
@@ -359,7 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           }
         }
       }
-      if (j > 0 && !mbar_wait_warp(&bar[bPtFree], (j - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+      // buffer j & 1 was last read by the UMMAs of q tile j - 2
+      const int pb = j & 1;
+      if (j >= 2 && !mbar_wait_warp(&bar[bPtFree + pb], ((j >> 1) - 1) & 1, p.status, kDevTimeoutSoftmax)) {
+        ok = false;
+        break;
+      }
+      const uint32_t pt_row = pb ? pt_buf[1] : pt_buf[0], ds_row = pb ? ds_buf[1] : ds_buf[0];
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         const int chunk = (c0 >> 3) + ch;
@@ -416,14 +439,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------------ dQ readout (thread = head-dim row)
-    // Each warp owns D/4 head-dim rows and adds its [32 x D/4] slices (two per q tile)
+    // Each warp owns D/4 head-dim rows and adds its [16 x D/4] slices (four per q tile)
     // with its own bulk reduces, so the four warps never wait on one another.
     const int quarter = warp & 3;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     constexpr int DW = D / 4;  // head-dim rows per warp
     // M = 128: lane l of quarter q holds d = 32q + l; M = 64: lanes 0-15 of quarter q hold d = 16q + l
     const bool dvalid = lane < DW;
-    float* region = sDQ + quarter * ((BM / 2) * DW);
+    // two staging buffers per warp, used in turn, so the reduce in flight never blocks the next slice
+    float* region0 = sDQ + quarter * (kDQRows * DW);
     QIter it;
     QTile r;
     int j = 0;
@@ -438,17 +462,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[bDQFree]);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        if (lane == 0) bulk_wait_group_read<0>();  // this warp's previous reduce has read its region
+      for (int pc = 0; pc < BM / kDQRows; ++pc) {
+        float* region = region0 + (pc & 1) * (L::kDQBuf / 4);
+        if (lane == 0) bulk_wait_group_read<1>();  // the reduce that last used this buffer has read it
         __syncwarp();
         if (dvalid) {
 #pragma unroll
-          for (int c = 0; c < BM / 2; ++c) region[c * DW + lane] = __uint_as_float(v[hf * 32 + c]) * p.scale;
+          for (int c = 0; c < kDQRows; ++c) region[c * DW + lane] = __uint_as_float(v[pc * kDQRows + c]) * p.scale;
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row + hf * 32);
+          tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row + pc * kDQRows);
           bulk_commit_group();
         }
       }

@@ -213,8 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     producer_done:;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ UMMA issuer (whole warp, one lane issues)
+    {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
       // base descriptors, built once; per-instruction offsets are compile-time constants
@@ -222,12 +222,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);      // stage s at + s * kTileBytes
       const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
-      bool ok = mbar_wait(&bar[bQFull], 0, p.status, kDevTimeoutMma);
+      bool ok = mbar_wait_warp(&bar[bQFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_pv = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) return false;
-        if (!mbar_wait(&bar[bVFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait_warp(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait_warp(&bar[bVFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
         tc_fence_after();
         const uint64_t dv = sdesc_add(dV0, st * L::kTileBytes);
 #pragma unroll
@@ -244,8 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       while (ok && next_tile<PAGED>(p, t, it, r)) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait(&bar[bKFull + st], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
-        if (!mbar_wait(&bar[bSFree + st], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[bKFull + st], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[bSFree + st], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const uint64_t dk = sdesc_add(dK0, st * L::kTileBytes);
         const uint32_t ts = tS0 + st * 128;
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       }
       if (ok && i > 0) ok = issue_pv(i - 1);
       if (i > 0) umma_commit(&bar[bODone]);
-      else mbar_arrive(&bar[bODone]);
+      else if (lane == 0) mbar_arrive(&bar[bODone]);
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue (warps 2..5)

@@ -159,8 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ UMMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------------ UMMA issuer (whole warp, one lane issues)
+    {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
       const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);      // tile x at + x * kTile
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         while (next_ktile(p, t, qp0, qp1, c, r)) ++n;
       }
       const int ntile = has_b ? 2 : 1;
-      bool ok = mbar_wait(&bar[pQFull], 0, p.status, kDevTimeoutMma);
+      bool ok = mbar_wait_warp(&bar[pQFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_s = [&](int x, int i) {
         const uint64_t dq = sdesc_add(dQ0, x * L::kTile), dk = sdesc_add(dK0, (i & 1) * L::kTile);
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         umma_commit(&bar[pPVDone + x]);
       };
       if (ok && n > 0) {
-        ok = mbar_wait(&bar[pKFull], 0, p.status, kDevTimeoutMma);
+        ok = mbar_wait_warp(&bar[pKFull], 0, p.status, kDevTimeoutMma);
         tc_fence_after();
         if (ok) {
           for (int x = 0; x < ntile; ++x) issue_s(x, 0);
@@ -203,16 +203,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       }
       for (int i = 0; ok && i < n; ++i) {
         const int st = i & 1;
-        if (!mbar_wait(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         for (int x = 0; x < ntile && ok; ++x) {
-          if (!mbar_wait(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait_warp(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
           tc_fence_after();
           issue_pv(x, i);
           if (i + 1 < n) {
             const int st1 = (i + 1) & 1;
-            if (!mbar_wait(&bar[pKFull + st1], ((i + 1) >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait_warp(&bar[pKFull + st1], ((i + 1) >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
             // P_x(i) lives in the columns S_x(i+1) will overwrite: let PV_x(i) finish reading it first
-            if (!mbar_wait(&bar[pPVDone + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait_warp(&bar[pPVDone + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
             tc_fence_after();
             issue_s(x, i + 1);
             if (x == ntile - 1) umma_commit(&bar[pKEmpty + st1]);
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         if (ok) umma_commit(&bar[pVEmpty + st]);
       }
       if (n > 0) umma_commit(&bar[pODone]);
-      else mbar_arrive(&bar[pODone]);
+      else if (lane == 0) mbar_arrive(&bar[pODone]);
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue (warps 2..9)
