@@ -253,25 +253,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         const bool cz = r.causal || W > 0;
         const int32_t kmin = r.kpos0, kmax = r.kpos0 + r.nvalid - 1;
         const bool need_mask = !((r.nvalid == BN) && (!cz || kmax <= xq0) && (W <= 0 || xq1 - kmin < W));
-        float mx = -INFINITY;
         if (need_mask) {
           int32_t hi = r.nvalid - 1, lo = 0;
           if (cz) hi = min(hi, qpos - r.kpos0);
           if (W > 0) lo = max(lo, qpos - W + 1 - r.kpos0);
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const float v = (c >= lo && c <= hi) ? __uint_as_float(s[c]) * sl2 : -INFINITY;
-            s[c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const float v = __uint_as_float(s[c]) * sl2;
-            s[c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
-          }
+          for (int c = 0; c < BN; ++c)
+            if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
         }
+        // row maximum of the raw scores (the scale is positive, so it commutes)
+        float mraw = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) mraw = max3f(mraw, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        const float mx = mraw * sl2;  // log2 units
         float m_use = m, alpha = 1.f;
         bool rescale_o = false;
         if (mx > m + kRescaleThreshold) {
@@ -284,11 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         uint32_t pk[BN / 2];
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2_approx(__uint_as_float(s[c]) - msub);
-          const float p1 = ex2_approx(__uint_as_float(s[c + 1]) - msub);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -msub));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -msub));
           const uint32_t pb = pack_bf16x2(p0, p1);
           rowsum += p0 + p1;
-          rowsum_r += __uint_as_float(pb << 16) + __uint_as_float(pb & 0xffff0000u);
+          rowsum_r = add_bf16x2_f32(rowsum_r, pb);
           pk[c / 2] = pb;
         }
         l = l * alpha + rowsum;
