@@ -650,11 +650,11 @@ int make_bwd_maps(BwdParams* p, const void* q, const void* dout, const void* k, 
 
 int64_t pad4(int64_t t) { return (t + 3) / 4 * 4; }
 
-// [H, t_pad] fp32 rows (lse * log2e or Delta) as a 2-D map, box of 68 rows
+// [H, t_pad] pairs {lse * log2e, Delta} as a 2-D fp32 map, box of 66 pairs
 int make_row_map(CUtensorMap* m, const float* rows, int64_t t_pad, int H) {
-  uint64_t dims[2] = {(uint64_t)std::max<int64_t>(t_pad, 4), (uint64_t)H};
-  uint64_t st[1] = {(uint64_t)t_pad};
-  uint32_t box[2] = {68, 1};
+  uint64_t dims[2] = {(uint64_t)std::max<int64_t>(2 * t_pad, 8), (uint64_t)H};
+  uint64_t st[1] = {(uint64_t)(2 * t_pad)};  // in elements
+  uint32_t box[2] = {132, 1};
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 2, rows, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
@@ -693,8 +693,7 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, plan);
   const int64_t tp = pad4(a->total);
-  float* delta = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
-  float* lse2 = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
+  float* rows = static_cast<float*>(c.take((size_t)H * tp * 2 * sizeof(float)));
   float* dq_acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   BwdParams p{};
@@ -708,8 +707,7 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   p.scale = resolve_scale(a->scale, D);
   p.scale_log2 = p.scale * kLog2e;
   p.window = a->window > 0 ? a->window : 0;
-  if ((rc = make_row_map(&p.tm_lse, lse2, tp, H))) return rc;
-  if ((rc = make_row_map(&p.tm_delta, delta, tp, H))) return rc;
+  if ((rc = make_row_map(&p.tm_rows, rows, tp, H))) return rc;
   p.dk = a->dk;
   p.dv = a->dv;
   p.dkv_stride_t = (int64_t)Hkv * D;
@@ -718,7 +716,7 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, delta, lse2, dq_acc, s),
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows, dq_acc, s),
                       "backward preprocess")))
     return rc;
   const int grid = grid_of(plan.tasks.size(), 1);
@@ -764,8 +762,7 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, plan);
   const int64_t tp = pad4(a->total_q);
-  float* delta = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
-  float* lse2 = static_cast<float*>(c.take((size_t)H * tp * sizeof(float)));
+  float* rows = static_cast<float*>(c.take((size_t)H * tp * 2 * sizeof(float)));
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   BwdParams p{};
   if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, a->dq_acc, a->total_q, a->total_k, H, Hkv, D))) return rc;
@@ -778,8 +775,7 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.scale = resolve_scale(a->scale, D);
   p.scale_log2 = p.scale * kLog2e;
   p.window = a->window > 0 ? a->window : 0;
-  if ((rc = make_row_map(&p.tm_lse, lse2, tp, H))) return rc;
-  if ((rc = make_row_map(&p.tm_delta, delta, tp, H))) return rc;
+  if ((rc = make_row_map(&p.tm_rows, rows, tp, H))) return rc;
   p.dk = a->dk_acc;
   p.dv = a->dv_acc;
   p.dkv_stride_t = (int64_t)Hkv * D;
@@ -788,7 +784,7 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, delta, lse2, nullptr, s),
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, rows, nullptr, s),
                       "backward preprocess")))
     return rc;
   return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch");

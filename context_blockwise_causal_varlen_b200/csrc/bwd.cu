@@ -31,8 +31,8 @@ constexpr int BN = 128;  // keys per CTA
 constexpr int BM = 64;   // q rows per streamed tile
 constexpr int kThreads = 448;
 constexpr int NS = 3;     // q / dO / row stages
-constexpr int kRowBox = BM + 4;  // lse/Delta box: 68 floats from a 16-byte aligned start
-constexpr int kRowSlot = 96;     // floats per row buffer: 384 bytes keeps every TMA destination 128-byte aligned
+constexpr int kRowPairs = BM + 2;  // {lse, Delta} box: 66 pairs from a 16-byte aligned start
+constexpr int kRowSlot = 160;      // floats per stage: 640 bytes keeps every TMA destination 128-byte aligned
 constexpr int kDQRows = 16;      // q rows per dQ bulk reduce (four per q tile)
 
 struct QTile {
@@ -95,7 +95,7 @@ struct BwdSmem {
   static constexpr uint32_t kKV = BN * D * 2;   // K or V tile (128 x D)
   static constexpr uint32_t kQT = BM * D * 2;   // a q / dO tile (64 x D)
   static constexpr uint32_t kPT = BN * BM * 2;  // P^T or dS^T (128 x 64)
-  static constexpr uint32_t kRowBytes = kRowBox * 4;  // bytes one row box delivers
+  static constexpr uint32_t kRowBytes = kRowPairs * 8;  // bytes one row box delivers
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kKV;
   static constexpr uint32_t kQ = kV + kKV;            // NS stages
@@ -111,7 +111,7 @@ struct BwdSmem {
   static constexpr uint32_t kPt1 = kPdsInV ? kV : kX;
   static constexpr uint32_t kDSt1 = kPt1 + kPT;
   static constexpr uint32_t kRow = kX + (kPdsInV ? 0 : 2 * kPT);  // per stage: lse*log2e and Delta slots
-  static constexpr uint32_t kBars = kRow + NS * 2 * kRowSlot * 4;
+  static constexpr uint32_t kBars = kRow + NS * kRowSlot * 4;
   static constexpr uint32_t kEnd = kBars + 256;
   static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
   static_assert(kDynamic <= 232448, "shared memory budget");
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* sPt = sm + L::kPt;
   uint8_t* sDSt = sm + L::kDSt;
   float* sDQ = reinterpret_cast<float*>(sm + L::kDQ);
-  float* sRow = reinterpret_cast<float*>(sm + L::kRow);  // [stage][lse*log2e 68 | Delta 68]
+  float* sRow = reinterpret_cast<float*>(sm + L::kRow);  // [stage][66 pairs {lse*log2e, Delta}]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + bBNum);
 
@@ -200,15 +200,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         const int st = j % NS;
         if (!mbar_wait(&bar[bQEmpty + st], ((j / NS) & 1) ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
         uint64_t* full = &bar[bQFull + st];
-        mbar_arrive_expect_tx(full, 2 * L::kQT + 2 * L::kRowBytes);
+        mbar_arrive_expect_tx(full, 2 * L::kQT + L::kRowBytes);
         for (int h = 0; h < KH; ++h) {
           tma_load_3d(sQ + st * L::kQT + h * 8192, &p.tm_q, full, h * 64, r.head, r.q_row);
           tma_load_3d(sDO + st * L::kQT + h * 8192, &p.tm_do, full, h * 64, r.head, r.q_row);
         }
-        float* row = sRow + st * 2 * kRowSlot;
-        const int x = r.q_row & ~3;  // 16-byte aligned start; the softmax indexes from q_row & 3
-        tma_load_2d(row, &p.tm_lse, full, x, r.head);
-        tma_load_2d(row + kRowSlot, &p.tm_delta, full, x, r.head);
+        // pairs from an even q row (a 16-byte aligned start); the softmax indexes from q_row & 1
+        tma_load_2d(sRow + st * kRowSlot, &p.tm_rows, full, 2 * (r.q_row & ~1), r.head);
         ++j;
       }
     }
@@ -332,8 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       if (!mbar_wait_warp(&bar[bQFull + st], (j / NS) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
       if (!mbar_wait_warp(&bar[bSFull], j & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
       tc_fence_after();
-      const float* lrow = sRow + st * 2 * kRowSlot + (r.q_row & 3) + c0;
-      const float* drow = lrow + kRowSlot;
+      const float2* lrow = reinterpret_cast<const float2*>(sRow + st * kRowSlot) + (r.q_row & 1) + c0;
       uint32_t pp[16], pd[16];
       {
         uint32_t s[32], dp[32];
@@ -348,11 +345,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!r.need_mask) {
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -lrow[c]));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -lrow[c + 1]));
+            const float2 r0 = lrow[c], r1 = lrow[c + 1];
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -r0.x));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -r1.x));
             pp[c / 2] = pack_bf16x2(p0, p1);
-            pd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - drow[c]),
-                                    p1 * (__uint_as_float(dp[c + 1]) - drow[c + 1]));
+            pd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - r0.y), p1 * (__uint_as_float(dp[c + 1]) - r1.y));
           }
         } else {
           // this key row sees the q columns [lo, hi] (positions are linear in the column)
@@ -366,10 +363,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
             for (int e = 0; e < 2; ++e) {
               const int col = c0 + c + e;
               const bool vis = col >= lo && col <= hi;
-              const float pe = vis ? ex2_approx(fmaf(__uint_as_float(s[c + e]), sl2, -lrow[c + e])) : 0.f;
+              const float2 re = lrow[c + e];
+              const float pe = vis ? ex2_approx(fmaf(__uint_as_float(s[c + e]), sl2, -re.x)) : 0.f;
               pv[e] = pe;
               // rows past the segment hold whatever the row buffer holds: keep them out of dS
-              dv[e] = vis ? pe * (__uint_as_float(dp[c + e]) - drow[c + e]) : 0.f;
+              dv[e] = vis ? pe * (__uint_as_float(dp[c + e]) - re.y) : 0.f;
             }
             pp[c / 2] = pack_bf16x2(pv[0], pv[1]);
             pd[c / 2] = pack_bf16x2(dv[0], dv[1]);

@@ -51,8 +51,7 @@ struct BwdParams {
   int32_t num_heads, heads_per_kv, num_kv_heads;
   float scale, scale_log2;
   int32_t window;
-  CUtensorMap tm_lse;   // (Tpad, H) fp32: merged lse * log2(e), box (68, 1)
-  CUtensorMap tm_delta; // (Tpad, H) fp32: rowsum(dO * O), box (68, 1)
+  CUtensorMap tm_rows;  // (2 Tpad, H) fp32: {merged lse * log2(e), rowsum(dO * O)} per q row, box (132, 1)
   // dk/dv outputs: bf16 (write) or fp32 (accumulate)
   void* dk;
   void* dv;
@@ -69,7 +68,7 @@ int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream);
 // Per (token, head): Delta = rowsum(dout * out) and lse * log2(e), written [H, t_pad]
 // (t_pad = total rounded up to a multiple of 4); optionally zero dq_acc.
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
-                          int32_t heads, int32_t head_dim, float* delta, float* lse2, float* dq_acc,
+                          int32_t heads, int32_t head_dim, float* rows, float* dq_acc,
                           cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);

@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ out, flo
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ dout,
                                                     const __nv_bfloat16* __restrict__ out,
-                                                    const float* __restrict__ lse, float* __restrict__ delta,
-                                                    float* __restrict__ lse2, int64_t total, int64_t t_pad, int heads) {
+                                                    const float* __restrict__ lse, float2* __restrict__ rows,
+                                                    int64_t total, int64_t t_pad, int heads) {
   constexpr int E = D / 32;
   const int64_t rowid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -95,8 +95,7 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
   if (lane == 0) {
     const int64_t tok = rowid / heads;
     const int h = (int)(rowid % heads);
-    delta[(int64_t)h * t_pad + tok] = s;
-    lse2[(int64_t)h * t_pad + tok] = lse[(int64_t)h * total + tok] * 1.4426950408889634f;
+    rows[(int64_t)h * t_pad + tok] = make_float2(lse[(int64_t)h * total + tok] * 1.4426950408889634f, s);
   }
 }
 
@@ -132,19 +131,20 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
 }
 
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
-                          int32_t heads, int32_t head_dim, float* delta, float* lse2, float* dq_acc,
+                          int32_t heads, int32_t head_dim, float* rows, float* dq_acc,
                           cudaStream_t stream) {
-  const int64_t rows = total * heads;
-  if (rows == 0) return 0;
+  const int64_t n = total * heads;
+  if (n == 0) return 0;
   if (dq_acc) {
-    cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)rows * head_dim * sizeof(float), stream);
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)n * head_dim * sizeof(float), stream);
     if (e != cudaSuccess) return (int)e;
   }
-  const int64_t blocks = (rows + 7) / 8;
+  const int64_t blocks = (n + 7) / 8;
   auto d = reinterpret_cast<const __nv_bfloat16*>(dout);
   auto o = reinterpret_cast<const __nv_bfloat16*>(out);
-  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, delta, lse2, total, t_pad, heads);
-  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, delta, lse2, total, t_pad, heads);
+  float2* r2 = reinterpret_cast<float2*>(rows);
+  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, r2, total, t_pad, heads);
+  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, r2, total, t_pad, heads);
   else return (int)cudaErrorInvalidValue;
   return (int)cudaGetLastError();
 }
