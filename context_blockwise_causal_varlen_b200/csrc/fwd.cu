@@ -213,8 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     producer_done:;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ UMMA issuer (whole warp, one lane issues)
-    {
+    // ------------------------------------------------------------------ UMMA issuer
+    // One lane runs the loop: here that measured about 6% faster than the warp-uniform
+    // loop with an elected issuing lane that the ping-pong forward and the backward use.
+    if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
       // base descriptors, built once; per-instruction offsets are compile-time constants
@@ -222,20 +224,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
       const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);      // stage s at + s * kTileBytes
       const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
-      bool ok = mbar_wait_warp(&bar[bQFull], 0, p.status, kDevTimeoutMma);
+      bool ok = mbar_wait(&bar[bQFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_pv = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait_warp(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) return false;
-        if (!mbar_wait_warp(&bar[bVFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) return false;
+        if (!mbar_wait(&bar[bVFull + st], (j >> 1) & 1, p.status, kDevTimeoutMma)) return false;
         tc_fence_after();
         const uint64_t dv = sdesc_add(dV0, st * L::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ss(tO, sdesc_add(dP, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(dv, kk * 2048), idesc_o,
+          umma_bf16_ss_1t(tO, sdesc_add(dP, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_add(dv, kk * 2048), idesc_o,
                        (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&bar[bVEmpty + st]);
-        umma_commit(&bar[bPVDone]);
+        umma_commit_1t(&bar[bVEmpty + st]);
+        umma_commit_1t(&bar[bPVDone]);
         return true;
       };
       TileIter it;
@@ -244,24 +246,24 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       while (ok && next_tile<PAGED>(p, t, it, r)) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait_warp(&bar[bKFull + st], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
-        if (!mbar_wait_warp(&bar[bSFree + st], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait(&bar[bKFull + st], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait(&bar[bSFree + st], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const uint64_t dk = sdesc_add(dK0, st * L::kTileBytes);
         const uint32_t ts = tS0 + st * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16_ss(ts, sdesc_add(dQ, off), sdesc_add(dk, off), idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss_1t(ts, sdesc_add(dQ, off), sdesc_add(dk, off), idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bar[bKEmpty + st]);
-        umma_commit(&bar[bSFull + st]);
+        umma_commit_1t(&bar[bKEmpty + st]);
+        umma_commit_1t(&bar[bSFull + st]);
         if (i > 0 && !issue_pv(i - 1)) { ok = false; break; }
         ++i;
       }
       if (ok && i > 0) ok = issue_pv(i - 1);
-      if (i > 0) umma_commit(&bar[bODone]);
-      else if (lane == 0) mbar_arrive(&bar[bODone]);
+      if (i > 0) umma_commit_1t(&bar[bODone]);
+      else mbar_arrive(&bar[bODone]);
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue (warps 2..5)
@@ -291,18 +293,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[bSFree + sb]);
 
-      float mx = -INFINITY;
       if (r.need_mask && (!PAGED || p.kv_mode == kKvContiguous)) {
         // positions are linear in the column: the visible columns of this row are [lo, hi]
         int32_t hi = r.nvalid - 1, lo = 0;
         if (r.causal || W > 0) hi = min(hi, qpos - r.kpos0);
         if (W > 0) lo = max(lo, qpos - W + 1 - r.kpos0);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const float v = (c >= lo && c <= hi) ? __uint_as_float(s[c]) * sl2 : -INFINITY;
-          s[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
+        for (int c = 0; c < BN; ++c)
+          if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
       } else if (r.need_mask) {
         // round-robin pages: position = page base + offset inside the page
 #pragma unroll
@@ -311,18 +309,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           bool vis = c < r.nvalid;
           if (r.causal || W > 0) vis = vis && (kpos <= qpos);
           if (W > 0) vis = vis && (qpos - kpos < W);
-          const float v = vis ? __uint_as_float(s[c]) * sl2 : -INFINITY;
-          s[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const float v = __uint_as_float(s[c]) * sl2;
-          s[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          if (!vis) s[c] = __float_as_uint(-INFINITY);
         }
       }
+      // row maximum of the raw scores (the scale is positive, so it commutes)
+      float mraw = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) mraw = max3f(mraw, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+      const float mx = mraw * sl2;  // log2 units
       // running max: keep a stale max while the new one is within 2^8 (values stay bounded)
       float m_use = m, alpha = 1.f;
       bool rescale_o = false;
@@ -336,11 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2_approx(__uint_as_float(s[c]) - msub);
-        const float p1 = ex2_approx(__uint_as_float(s[c + 1]) - msub);
+        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -msub));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -msub));
         const uint32_t pb = pack_bf16x2(p0, p1);
         rowsum += p0 + p1;
-        rowsum_r += __uint_as_float(pb << 16) + __uint_as_float(pb & 0xffff0000u);
+        rowsum_r = add_bf16x2_f32(rowsum_r, pb);
         pk[c / 2] = pb;
       }
       l = l * alpha + rowsum;
