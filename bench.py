@@ -402,7 +402,7 @@ def main():
     value = total_flops / (ms * 1e-3) / 1e12
     if rank == 0:
         # the dominant kernel: the block backward (10 of the 14 flops per pair)
-        dom_ms, dom_flops, dom_name = (bwd_ms, f_bwd, "bwd_kernel") if bwd_ms >= fwd_ms else (fwd_ms, f_fwd, "fwd_kernel")
+        dom_ms, dom_flops, dom_name = (bwd_ms, f_bwd, "bwd_kernel") if bwd_ms >= fwd_ms else (fwd_ms, f_fwd, "fwd_pp_kernel")
         achieved = dom_flops / (dom_ms * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

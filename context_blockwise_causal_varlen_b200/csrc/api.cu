@@ -387,7 +387,7 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   if ((rc = upload_plan(pd, plan, s))) return rc;
   const int grid = grid_of(plan.tasks.size(), 1);
   if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
-  return launch_rc(launch_fwd_pingpong(p, D, grid, s), "block forward launch");
+  return launch_rc(launch_fwd_pingpong(p, D, false, grid, s), "block forward launch");
 }
 
 // ------------------------------------------------------------------------ merge
@@ -433,7 +433,7 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
     p.num_tasks = (int)L.fused.tasks.size();
     p.out = a->out;
     p.out_mode = kOutBf16;
-    return launch_rc(launch_fwd_pingpong(p, D, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch");
+    return launch_rc(launch_fwd_pingpong(p, D, false, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch");
   }
   std::vector<PlanDev> pds;
   for (auto& pl : L.steps) {
@@ -447,7 +447,7 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
     p.num_tasks = (int)L.steps[st].tasks.size();
     p.out = acc;
     p.out_mode = st == 0 ? kOutF32 : kOutMerge;
-    if ((rc = launch_rc(launch_fwd_pingpong(p, D, grid_of(L.steps[st].tasks.size(), 1), s), "ring step launch")))
+    if ((rc = launch_rc(launch_fwd_pingpong(p, D, false, grid_of(L.steps[st].tasks.size(), 1), s), "ring step launch")))
       return rc;
   }
   return launch_rc(launch_convert_bf16(acc, a->out, a->total * H * D, 1.f, s), "output conversion");
@@ -476,7 +476,7 @@ static int kvp_checks(const cbv_kvp_args* a) {
 static size_t kvp_layout(const cbv_kvp_args* a, Plan* plan_out) {
   const int n_local = a->blocks_per_shard * a->block_size;
   Plan plan = plan_kvp(a->q_len, a->num_heads, a->shards, n_local, a->seg_size, (KvMode)a->kv_mode, a->block_size,
-                       a->global_q_offset, a->sliding_window, a->shard_out != nullptr, 128);
+                       a->global_q_offset, a->sliding_window, a->shard_out != nullptr, kPairRows);
   Carve c(nullptr);
   c.take(kStatusBytes);
   carve_plan(c, plan);
@@ -542,7 +542,7 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
     p.lse = a->lse ? a->lse : lse_scratch;
     p.lse_stride_h = a->q_len;
     p.lse_stride_t = 1;
-    return launch_rc(launch_fwd(p, D, true, grid, s), "prefill launch");
+    return launch_rc(launch_fwd_pingpong(p, D, true, grid, s), "prefill launch");
   }
   // per-shard partials, then an explicit online-softmax merge of the shards
   p.out = a->shard_out;
@@ -554,7 +554,7 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   p.lse_stride_h = a->q_len;
   p.lse_stride_t = 1;
   p.lse_shard_stride = (int64_t)H * a->q_len;
-  if ((rc = launch_rc(launch_fwd(p, D, true, grid, s), "prefill launch"))) return rc;
+  if ((rc = launch_rc(launch_fwd_pingpong(p, D, true, grid, s), "prefill launch"))) return rc;
   cudaError_t e = cudaMemcpyAsync(acc, a->shard_out, rows * D * sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(lse_scratch, a->shard_lse, rows * sizeof(float), cudaMemcpyDeviceToDevice, s);
   if (e != cudaSuccess) return cuda_fail(e, "copying shard 0");

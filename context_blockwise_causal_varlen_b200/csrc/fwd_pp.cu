@@ -1,12 +1,19 @@
-// Block forward on tcgen05, two q tiles per CTA ("ping-pong").
+// Block forward on tcgen05: flash-style attention of up to 256 q rows (two 128-row
+// tiles, "ping-pong") against a list of k/v segments, returning (out, lse) or merging
+// into a running pair.
 //
-// Same operation as fwd.cu (the per-block flash forward of the NeMo AutoModel
-// zig-zag ring page, _block_forward, with the blocks of a tile merged by the
-// online-softmax identity, update_out_and_lse, on chip), organised so that the
-// tensor core never waits for one softmax: a CTA owns two 128-row q tiles A and B
-// of the same head that stream the same k/v tiles.  While warpgroup A turns S_A
-// into P_A, the tensor core computes S_B or PV_B, and the other way round.
+// This is the per-block kernel of the NeMo AutoModel zig-zag ring page
+// (_block_forward: one flash varlen forward block) and, in its paged instantiation,
+// of the KV-parallel segmented prefill (NKI attention_kv_parallel_segmented_cte:
+// per-shard segment loop over a paged cache with online softmax).  Consecutive
+// segments belonging to different ring blocks (or shards) are combined by the
+// online-softmax log-sum-exp identity (update_out_and_lse) applied in place to the
+// TMEM accumulator; with out_mode = kOutMerge the epilogue applies the same identity
+// to a running (out, lse) pair in HBM, so no separate merge pass is needed.
 //
+// The two q tiles A and B of a CTA belong to the same head and stream the same k/v
+// tiles, so the tensor core never waits for one softmax: while warpgroup A turns
+// S_A into P_A, the tensor core computes S_B or PV_B, and the other way round.
 // P never leaves TMEM: the softmax writes P (bf16, two per 32-bit column) over the
 // S columns it has just read, and PV takes its A operand from TMEM.
 //
@@ -27,7 +34,12 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: keep a stale max while it is within 2^8
 
 struct KTile {
-  int32_t k_row, kpos0, nvalid, causal;
+  int32_t k_row;   // first row (non-paged: tensor row; paged: shard-local token)
+  int32_t kpos0;   // position of column 0 (paged: position of the tile's first token)
+  int32_t kmax;    // largest position in the tile
+  int32_t nvalid;  // valid columns
+  int32_t causal;
+  int32_t shard;
 };
 
 struct KIter {
@@ -35,7 +47,16 @@ struct KIter {
   Seg seg;
 };
 
-// k tiles that at least one row of q positions [qp0, qp1] can see (non-paged).
+// global position of shard-local token t of a paged KV cache
+__device__ __forceinline__ int32_t kvp_position(const FwdParams& p, int32_t shard, int32_t t) {
+  if (p.kv_mode == kKvRoundRobin)
+    return ((t / p.block_size) * p.shards + shard) * p.block_size + t % p.block_size;
+  return shard * p.n_local + t;
+}
+
+// k tiles that at least one row of q positions [qp0, qp1] can see.  Every role runs
+// its own copy and sees the same sequence.
+template <bool PAGED>
 __device__ __forceinline__ bool next_ktile(const FwdParams& p, const TileTask& t, int32_t qp0, int32_t qp1,
                                            KIter& it, KTile& r) {
   const int32_t W = p.window;
@@ -44,22 +65,37 @@ __device__ __forceinline__ bool next_ktile(const FwdParams& p, const TileTask& t
       if (it.si >= t.nseg) return false;
       it.seg = p.segs[t.seg0 + it.si];
       it.si++;
-      const bool cz = (it.seg.flags & kSegCausal) || W > 0;
-      int32_t cmax = it.seg.rows - 1, cmin = 0;
-      if (cz) cmax = min(cmax, qp1 - it.seg.pos0);
-      if (W > 0) cmin = max(0, qp0 - W + 1 - it.seg.pos0);
-      if (cmax < cmin) {
-        it.j = it.jn = 0;
-        continue;
+      if (!PAGED) {
+        const bool cz = (it.seg.flags & kSegCausal) || W > 0;
+        int32_t cmax = it.seg.rows - 1, cmin = 0;
+        if (cz) cmax = min(cmax, qp1 - it.seg.pos0);
+        if (W > 0) cmin = max(0, qp0 - W + 1 - it.seg.pos0);
+        if (cmax < cmin) {
+          it.j = it.jn = 0;
+          continue;
+        }
+        it.j = cmin / BN;
+        it.jn = cmax / BN + 1;
+      } else {
+        it.j = 0;
+        it.jn = (it.seg.rows + BN - 1) / BN;
       }
-      it.j = cmin / BN;
-      it.jn = cmax / BN + 1;
     }
     const int32_t c0 = it.j++ * BN;
     r.nvalid = min(BN, it.seg.rows - c0);
     r.k_row = it.seg.row0 + c0;
-    r.kpos0 = it.seg.pos0 + c0;
     r.causal = it.seg.flags & kSegCausal;
+    if (!PAGED) {
+      r.shard = 0;
+      r.kpos0 = it.seg.pos0 + c0;
+      r.kmax = r.kpos0 + r.nvalid - 1;
+    } else {
+      r.shard = it.seg.flags >> kSegShardShift;
+      r.kpos0 = kvp_position(p, r.shard, r.k_row);
+      r.kmax = kvp_position(p, r.shard, r.k_row + r.nvalid - 1);
+      if (r.kpos0 > qp1) continue;
+      if (W > 0 && r.kmax < qp0 - W + 1) continue;
+    }
     return true;
   }
 }
@@ -89,7 +125,7 @@ enum PBar {
   pNum = 16
 };
 
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_constant__ FwdParams p) {
   using L = PPSmem<D>;
   constexpr int QH = D / 64;
@@ -144,17 +180,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       KIter it;
       KTile r;
       int i = 0;
-      while (next_ktile(p, t, qp0, qp1, it, r)) {
+      while (next_ktile<PAGED>(p, t, qp0, qp1, it, r)) {
         const int st = i & 1;
         const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait(&bar[pKEmpty + st], ph ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
-        mbar_arrive_expect_tx(&bar[pKFull + st], L::kTile);
-        for (int h = 0; h < QH; ++h)
-          tma_load_3d(sK + st * L::kTile + h * 16384, &p.tm_k, &bar[pKFull + st], h * 64, kvh, r.k_row);
-        if (!mbar_wait(&bar[pVEmpty + st], ph ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
-        mbar_arrive_expect_tx(&bar[pVFull + st], L::kTile);
-        for (int h = 0; h < QH; ++h)
-          tma_load_3d(sV + st * L::kTile + h * 16384, &p.tm_v, &bar[pVFull + st], h * 64, kvh, r.k_row);
+        bool ok = true;
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          uint64_t* empty = &bar[(kv == 0 ? pKEmpty : pVEmpty) + st];
+          uint64_t* full = &bar[(kv == 0 ? pKFull : pVFull) + st];
+          const CUtensorMap* map = kv == 0 ? &p.tm_k : &p.tm_v;
+          uint8_t* dst = (kv == 0 ? sK : sV) + st * L::kTile;
+          if (!mbar_wait(empty, ph ^ 1, p.status, kDevTimeoutTmaEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full, L::kTile);
+          if (!PAGED) {
+            for (int h = 0; h < QH; ++h) tma_load_3d(dst + h * 16384, map, full, h * 64, kvh, r.k_row);
+          } else {
+            // one box per page of block_size tokens, found through the shard's block table
+            const int bs = p.block_size;
+            for (int pg = 0; pg < BN / bs; ++pg) {
+              const int blk = min((r.k_row + pg * bs) / bs, p.blocks_per_shard - 1);
+              const int page = __ldg(&p.block_tables[(int64_t)r.shard * p.blocks_per_shard + blk]);
+              for (int h = 0; h < QH; ++h) tma_load_4d(dst + h * 16384 + pg * bs * 128, map, full, h * 64, 0, kvh, page);
+            }
+          }
+        }
+        if (!ok) break;
         ++i;
       }
     }
@@ -170,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       {
         KIter c;
         KTile r;
-        while (next_ktile(p, t, qp0, qp1, c, r)) ++n;
+        while (next_ktile<PAGED>(p, t, qp0, qp1, c, r)) ++n;
       }
       const int ntile = has_b ? 2 : 1;
       bool ok = mbar_wait_warp(&bar[pQFull], 0, p.status, kDevTimeoutMma);
@@ -242,24 +294,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
     if (x == 0 || has_b) {
       KIter it;
       KTile r;
-      while (next_ktile(p, t, qp0, qp1, it, r)) {
+      while (next_ktile<PAGED>(p, t, qp0, qp1, it, r)) {
         if (!mbar_wait_warp(&bar[pSFull + x], i & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
         tc_fence_after();
         uint32_t s[BN];
 #pragma unroll
         for (int c = 0; c < BN; c += 32) tmem_ld32(tS + c, s + c);
         tmem_ld_wait();
-        // this tile's rows see the columns [lo, hi] of this k tile
         const bool cz = r.causal || W > 0;
-        const int32_t kmin = r.kpos0, kmax = r.kpos0 + r.nvalid - 1;
-        const bool need_mask = !((r.nvalid == BN) && (!cz || kmax <= xq0) && (W <= 0 || xq1 - kmin < W));
-        if (need_mask) {
+        const bool need_mask = !((r.nvalid == BN) && (!cz || r.kmax <= xq0) && (W <= 0 || xq1 - r.kpos0 < W));
+        if (need_mask && (!PAGED || p.kv_mode == kKvContiguous)) {
+          // positions are linear in the column: this row sees the columns [lo, hi]
           int32_t hi = r.nvalid - 1, lo = 0;
           if (cz) hi = min(hi, qpos - r.kpos0);
           if (W > 0) lo = max(lo, qpos - W + 1 - r.kpos0);
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
+        } else if (need_mask) {
+          // round-robin pages: position = page base + offset inside the page
+#pragma unroll
+          for (int c = 0; c < BN; ++c) {
+            const int32_t kpos = r.kpos0 + (c / p.block_size) * p.shards * p.block_size + (c % p.block_size);
+            bool vis = c < r.nvalid;
+            if (cz) vis = vis && (kpos <= qpos);
+            if (W > 0) vis = vis && (qpos - kpos < W);
+            if (!vis) s[c] = __float_as_uint(-INFINITY);
+          }
         }
         // row maximum of the raw scores (the scale is positive, so it commutes)
         float mraw = -INFINITY;
@@ -319,7 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       const float lse_b = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
       const bool valid = trow < t.rows;
       const int64_t orow = (int64_t)(t.row0 + trow);
-      float* lse_ptr = p.lse + (int64_t)head * p.lse_stride_h + orow * p.lse_stride_t;
+      const int64_t shard_off = t.aux >= 0 ? (int64_t)t.aux : 0;  // per-shard outputs
+      float* lse_ptr = p.lse + shard_off * p.lse_shard_stride + (int64_t)head * p.lse_stride_h + orow * p.lse_stride_t;
       float wa = 0.f, wb = 1.f, lse_new = lse_b;
       if (p.out_mode == kOutMerge && valid) {
         const float lse_a = *lse_ptr;
@@ -345,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
         if (p.out_mode == kOutBf16) {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.out_stride_t +
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + shard_off * p.out_shard_stride + orow * p.out_stride_t +
                                (int64_t)head * p.out_stride_h + c;
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
@@ -357,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
             *reinterpret_cast<uint4*>(dst + e) = v;
           }
         } else {
-          float* dst = reinterpret_cast<float*>(p.out) + orow * p.out_stride_t + (int64_t)head * p.out_stride_h + c;
+          float* dst = reinterpret_cast<float*>(p.out) + shard_off * p.out_shard_stride + orow * p.out_stride_t +
+                     (int64_t)head * p.out_stride_h + c;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             float4 v;
@@ -385,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int D>
+template <int D, bool PAGED>
 int launch_pp_t(const FwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = fwd_pp_kernel<D>;
+  auto kern = fwd_pp_kernel<D, PAGED>;
   const uint32_t smem = PPSmem<D>::kDynamic;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
@@ -397,10 +460,10 @@ int launch_pp_t(const FwdParams& p, int grid, cudaStream_t stream) {
 
 }  // namespace
 
-int launch_fwd_pingpong(const FwdParams& p, int head_dim, int grid, cudaStream_t stream) {
+int launch_fwd_pingpong(const FwdParams& p, int head_dim, bool paged, int grid, cudaStream_t stream) {
   if (grid <= 0) return 0;
-  if (head_dim == 128) return launch_pp_t<128>(p, grid, stream);
-  if (head_dim == 64) return launch_pp_t<64>(p, grid, stream);
+  if (head_dim == 128) return paged ? launch_pp_t<128, true>(p, grid, stream) : launch_pp_t<128, false>(p, grid, stream);
+  if (head_dim == 64) return paged ? launch_pp_t<64, true>(p, grid, stream) : launch_pp_t<64, false>(p, grid, stream);
   return (int)cudaErrorInvalidValue;
 }
 

@@ -60,9 +60,8 @@ struct BwdParams {
   int* status;
 };
 
-int launch_fwd(const FwdParams& p, int head_dim, bool paged, int grid, cudaStream_t stream);
-// Non-paged forward with two 128-row q tiles per task (task.rows <= 256).
-int launch_fwd_pingpong(const FwdParams& p, int head_dim, int grid, cudaStream_t stream);
+// Forward with two 128-row q tiles per task (task.rows <= 256); paged selects the page-table K/V loads.
+int launch_fwd_pingpong(const FwdParams& p, int head_dim, bool paged, int grid, cudaStream_t stream);
 int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream);
 
 // Per (token, head): Delta = rowsum(dout * out) and lse * log2(e), written [H, t_pad]
