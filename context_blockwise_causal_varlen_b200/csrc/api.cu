@@ -352,10 +352,15 @@ size_t cbv_block_fwd_workspace_size(const cbv_block_fwd_args* a) {
 int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   int rc = block_fwd_checks(a);
   if (rc) return rc;
+  if (a->total_q == 0) return CBV_OK;  // no query rows: nothing to write
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
     return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  // without key rows no k tile is ever loaded; the maps then describe one q row instead
+  const void* kp = a->total_k > 0 ? a->k : a->q;
+  const void* vp = a->total_k > 0 ? a->v : a->q;
+  const int64_t kst = a->total_k > 0 ? (int64_t)Hkv * D : (int64_t)H * D;
   Plan plan = plan_block_fwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs,
                              a->causal != 0, a->window, H, kPairRows);
   Carve c(a->workspace);
@@ -365,8 +370,8 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
     return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   FwdParams p{};
   if ((rc = map_thd(&p.tm_q, a->q, a->total_q, H, D, (int64_t)H * D, D, 128))) return rc;
-  if ((rc = map_thd(&p.tm_k, a->k, a->total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
-  if ((rc = map_thd(&p.tm_v, a->v, a->total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  if ((rc = map_thd(&p.tm_k, kp, a->total_k, Hkv, D, kst, D, 128))) return rc;
+  if ((rc = map_thd(&p.tm_v, vp, a->total_k, Hkv, D, kst, D, 128))) return rc;
   p.tasks = pd.tasks;
   p.segs = pd.segs;
   p.num_tasks = (int)plan.tasks.size();
@@ -393,9 +398,10 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
 // ------------------------------------------------------------------------ merge
 int cbv_attn_merge(float* out, float* lse, const void* block_out, int32_t block_out_dtype, const float* block_lse,
                    float* weight_out, int64_t seqlen, int32_t num_heads, int32_t head_dim, void* stream) {
-  if (!out || !lse || !block_out || !block_lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (head_dim != 64 && head_dim != 128) return fail(CBV_ERR_UNSUPPORTED_HEAD_DIM, "head_dim %d", head_dim);
   if (seqlen < 0 || num_heads <= 0) return fail(CBV_ERR_BAD_SHAPE, "bad shape");
+  if (seqlen == 0) return CBV_OK;
+  if (!out || !lse || !block_out || !block_lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (block_out_dtype != CBV_DTYPE_BF16 && block_out_dtype != CBV_DTYPE_F32) return fail(CBV_ERR_BAD_DTYPE, "bad dtype");
   if (!aligned16(out) || !aligned16(block_out)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   return launch_rc(launch_merge(out, lse, block_out, block_out_dtype == CBV_DTYPE_F32, block_lse, weight_out, seqlen,
@@ -412,6 +418,7 @@ size_t cbv_zigzag_ring_fwd_workspace_size(const cbv_ring_args* a) {
 int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
   int rc = ring_common_checks(a);
   if (rc) return rc;
+  if (a->total == 0) return CBV_OK;  // no rows: nothing to write
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
     return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -495,6 +502,7 @@ size_t cbv_kvp_workspace_size(const cbv_kvp_args* a) {
 int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   int rc = kvp_checks(a);
   if (rc) return rc;
+  if (a->q_len == 0) return CBV_OK;  // no query rows: nothing to write
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Plan plan;
   const size_t need = kvp_layout(a, &plan);
@@ -584,6 +592,7 @@ int cbv_varlen_decode(const cbv_decode_args* a, void* stream) {
   if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
   if (a->num_heads / a->num_kv_heads > 16) return fail(CBV_ERR_GQA_MISMATCH, "at most 16 q heads per kv head");
   if (a->num_seqs < 0 || a->total_q < a->num_seqs || a->total_k < 0) return fail(CBV_ERR_BAD_SHAPE, "bad sizes");
+  if (a->num_seqs == 0) return CBV_OK;  // no sequences: nothing to write
   if (!a->cu_seqlens_q || !a->cu_seqlens_k) return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens is NULL");
   if (!a->workspace || a->workspace_bytes < kStatusBytes) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", kStatusBytes);
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
@@ -682,6 +691,7 @@ size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a) {
 int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   int rc = ring_common_checks(a);
   if (rc) return rc;
+  if (a->total == 0) return CBV_OK;  // no rows: nothing to write
   if (!a->dout || !a->out || !a->lse || !a->dq || !a->dk || !a->dv) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) || !aligned16(a->dout) ||
       !aligned16(a->dq) || !aligned16(a->dk) || !aligned16(a->dv))
@@ -754,6 +764,7 @@ size_t cbv_block_bwd_workspace_size(const cbv_block_bwd_args* a) {
 int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   int rc = block_bwd_checks(a);
   if (rc) return rc;
+  if (a->total_q == 0 || a->total_k == 0) return CBV_OK;  // no (q, k) pair: the accumulators are unchanged
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
   Plan plan = plan_block_bwd(a->cu_seqlens_q, a->cu_seqlens_k, a->q_pos_base, a->k_pos_base, a->num_docs,

@@ -168,3 +168,18 @@ def test_kvp_rejects_bad_block_and_segment_sizes():
     assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"
     a.block_size, a.seg_size = 32, 100
     assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"
+
+
+def test_empty_problems_return_ok_without_touching_the_device():
+    # no rows: every entry point validates its arguments and returns before any CUDA call
+    for cu in (np.array([0], np.int32), np.array([0, 0, 0], np.int32)):
+        a, _ = _ring_args(cu=cu)
+        assert cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None) == 0, cbv.lib().cbv_last_error_message()
+        assert cbv.lib().cbv_zigzag_ring_bwd(ctypes.byref(a), None) == 0, cbv.lib().cbv_last_error_message()
+    assert cbv.lib().cbv_attn_merge(None, None, None, cbv.DTYPE_F32, None, None, 0, 2, 128, None) == 0
+    d = cbv.DecodeArgs(struct_size=ctypes.sizeof(cbv.DecodeArgs), abi_version=cbv.ABI_VERSION, num_seqs=0, total_q=0,
+                       total_k=0, num_heads=8, num_kv_heads=2, head_dim=128)
+    assert cbv.lib().cbv_varlen_decode(ctypes.byref(d), None) == 0
+    # but a malformed empty call is still an error
+    a, _ = _ring_args(cu=np.array([0], np.int32), head_dim=80)
+    assert cbv.STATUS[cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None)] == "UNSUPPORTED_HEAD_DIM"

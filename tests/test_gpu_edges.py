@@ -1,0 +1,133 @@
+"""Edge cases on the GPU against the fp64 oracle: empty documents and inputs, the smallest
+window, wide GQA groups, keyless rows, every paged block size, and the merge's identities."""
+import numpy as np
+import pytest
+import torch
+
+import context_blockwise_causal_varlen_b200 as cbv
+from oracle import attention as A
+from oracle import paged as PG
+from synth import block_permutation, cu_from_lengths, streams
+from tests.gpu_util import check_lse, check_out, check_rel, dev, f64, gen, host, sync
+
+pytestmark = pytest.mark.gpu
+
+
+def _ring_case(seed, lengths, H, HKV, D):
+    cu = cu_from_lengths(lengths)
+    S = int(cu[-1])
+    q, k, v, do = gen(seed, (S, H, D), (S, HKV, D), (S, HKV, D), (S, H, D))
+    return cu, q, k, v, do
+
+
+@pytest.mark.parametrize("layout", ["zigzag", "contiguous"])
+@pytest.mark.parametrize("schedule", [cbv.SCHEDULE_FUSED, cbv.SCHEDULE_STEPWISE])
+def test_empty_and_tiny_documents_in_the_batch(layout, schedule):
+    # documents of length 0 and of one token per chunk sit between ordinary ones
+    lengths, cp = [0, 264, 0, 4, 520, 0], 2
+    cu, q, k, v, do = _ring_case(40, lengths, 2, 2, 128)
+    scale = 0.1
+    out, lse = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, cp, scale=scale, layout=layout, schedule=schedule)
+    dq, dk, dv = cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out, lse, cu, cp, scale=scale, layout=layout)
+    sync()
+    ro, rl = A.attention_fwd(f64(q), f64(k), f64(v), cu, cu, scale)
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+    rq, rk, rv = A.attention_bwd(f64(do), f64(q), f64(k), f64(v), host(out), rl, cu, cu, scale)
+    check_rel(host(dq), rq, what="dq")
+    check_rel(host(dk), rk, what="dk")
+    check_rel(host(dv), rv, what="dv")
+
+
+def test_empty_input_and_all_empty_documents():
+    for lengths in ([], [0], [0, 0, 0]):
+        cu = cu_from_lengths(lengths)
+        e = torch.empty((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+        out, lse = cbv.zigzag_ring_fwd(e, e, e, cu, 2)
+        dq, dk, dv = cbv.zigzag_ring_bwd(e, e, e, e, out, lse, cu, 2)
+        sync()
+        assert out.shape == (0, 2, 128) and lse.shape == (2, 0) and dq.shape == (0, 2, 128)
+
+
+def test_window_of_one_sees_only_the_query_itself():
+    cu, q, k, v, do = _ring_case(41, [256, 512], 2, 2, 64)
+    out, lse = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, 2, scale=0.125, window=1)
+    dq, dk, dv = cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out, lse, cu, 2, scale=0.125, window=1)
+    sync()
+    # one visible key: out = v_i, lse = s_ii, dv = dO, and dq = dk = 0 (dP - Delta vanishes up to
+    # the rounding of two fp32 dot products)
+    np.testing.assert_array_equal(host(out), f64(v))
+    check_lse(host(lse), (0.125 * (f64(q) * f64(k)).sum(-1)).T)
+    assert np.abs(host(dq)).max() <= 1e-3 and np.abs(host(dk)).max() <= 1e-3
+    np.testing.assert_array_equal(host(dv), f64(do))
+
+
+def test_wide_gqa_group_with_head_dim_64():
+    cu, q, k, v, do = _ring_case(42, [512, 128, 264], 8, 1, 64)
+    scale = 0.125
+    out, lse = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, 2, scale=scale)
+    dq, dk, dv = cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out, lse, cu, 2, scale=scale)
+    sync()
+    ro, rl = A.attention_fwd(f64(q), f64(k), f64(v), cu, cu, scale)
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+    rq, rk, rv = A.attention_bwd(f64(do), f64(q), f64(k), f64(v), host(out), rl, cu, cu, scale)
+    check_rel(host(dq), rq, what="dq")
+    check_rel(host(dk), rk, what="dk")
+    check_rel(host(dv), rv, what="dv")
+
+
+def test_block_forward_rows_without_keys():
+    # document 0 has queries but no keys; document 1 has keys but no queries; document 2 is ordinary
+    cu_q, cu_k = np.array([0, 70, 70, 200], np.int32), np.array([0, 0, 90, 330], np.int32)
+    q, k, v = gen(43, (200, 2, 128), (330, 2, 128), (330, 2, 128))
+    out, lse = cbv.attn_block_fwd(dev(q), dev(k), dev(v), cu_q, cu_k, scale=0.1, causal=True)
+    sync()
+    ro, rl = A.attention_fwd(f64(q), f64(k), f64(v), cu_q, cu_k, 0.1, causal=True)
+    assert np.all(host(out)[:70] == 0) and np.all(np.isneginf(host(lse)[:, :70]))
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+
+
+@pytest.mark.parametrize("bs,D,mode", [(8, 128, PG.ROUND_ROBIN), (16, 64, PG.CONTIGUOUS), (64, 128, PG.ROUND_ROBIN),
+                                       (128, 64, PG.ROUND_ROBIN), (128, 128, PG.CONTIGUOUS)])
+def test_kvp_prefill_every_block_size(bs, D, mode):
+    R, n_local, hq, hkv, S = 2, 256, 4, 2, 200
+    bps = n_local // bs
+    nb = R * bps
+    q, kc, vc = gen(44, (hq, S, D), (nb, hkv, bs, D), (nb, hkv, bs, D))
+    perm = block_permutation(streams(144, 1)[0], nb)
+    bt = PG.shard_block_tables(perm, R, mode)
+    gqo = R * n_local - S - 5
+    K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, mode)
+    for window in (0, 77):
+        ro, rl = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=window)
+        kv_mode = cbv.KV_ROUND_ROBIN if mode == PG.ROUND_ROBIN else cbv.KV_CONTIGUOUS
+        out, lse = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), kv_mode=kv_mode,
+                                             seg_size=128, scale=0.1, global_q_offset=gqo, sliding_window=window)
+        sync()
+        check_out(host(out), ro, what=f"out bs={bs} W={window}")
+        check_lse(host(lse), rl, what=f"lse bs={bs} W={window}")
+
+
+def test_merge_identities_of_minus_infinity():
+    S, H, D = 64, 2, 128
+    (a,) = gen(45, (S, H, D))
+    (b,) = gen(46, (S, H, D))
+    out = torch.from_numpy(a).cuda()
+    lse = torch.full((H, S), 0.5, device="cuda")
+    # a block with lse = -inf leaves the running pair unchanged
+    o2, l2 = cbv.attn_merge(out.clone(), lse.clone(), dev(b), torch.full((H, S), -float("inf"), device="cuda"))
+    sync()
+    assert torch.equal(o2, out) and torch.equal(l2, lse)
+    # a running pair with lse = -inf takes the block
+    blk = dev(b)
+    o3, l3 = cbv.attn_merge(torch.zeros_like(out), torch.full((H, S), -float("inf"), device="cuda"), blk,
+                            torch.full((H, S), 0.25, device="cuda"))
+    sync()
+    assert torch.equal(o3, blk.float()) and torch.all(l3 == 0.25)
+    # both -inf: stays -inf, out unchanged
+    o4, l4 = cbv.attn_merge(out.clone(), torch.full((H, S), -float("inf"), device="cuda"), blk,
+                            torch.full((H, S), -float("inf"), device="cuda"))
+    sync()
+    assert torch.equal(o4, out) and torch.all(torch.isneginf(l4))
