@@ -55,6 +55,7 @@ __device__ __forceinline__ bool next_qtile(const BwdParams& p, const TileTask& t
   const int32_t kp0 = t.pos0, kp1 = t.pos0 + t.rows - 1;
   const int32_t W = p.window;
   while (true) {
+    if (it.hs >= p.heads_per_kv) return false;  // exhausted (and stays so when called again)
     if (it.j >= it.jn) {
       if (it.si >= t.nseg) {
         it.hs++;
@@ -123,13 +124,13 @@ enum BBar {
   bQEmpty = 4,   // +stage (NS)
   bSFull = 7,
   bSFree = 8,
-  bPFull = 9,
-  bPtFree = 10,  // +P^T / dS^T buffer (2)
-  bDQFull = 12,
-  bDQFree = 13,
-  bVTmem = 14,
-  bAccDone = 15,
-  bBNum = 16
+  bPFull = 9,    // +P^T / dS^T buffer (2)
+  bPtFree = 11,  // +P^T / dS^T buffer (2)
+  bDQFull = 13,
+  bDQFree = 14,
+  bVTmem = 15,
+  bAccDone = 16,
+  bBNum = 17
 };
 
 
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     mbar_init(&bar[bSFull], 1);
     mbar_init(&bar[bSFree], 8);
     mbar_init(&bar[bPFull], 8);
+    mbar_init(&bar[bPFull + 1], 8);
     mbar_init(&bar[bPtFree], 1);
     mbar_init(&bar[bPtFree + 1], 1);
     mbar_init(&bar[bAccDone], 1);
@@ -262,10 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % NS;
         if (j + 1 < n && !(ok = issue_sdp(j + 1))) break;
-        if (!mbar_wait_warp(&bar[bPFull], j & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        // one PFull per P^T / dS^T buffer: a fast softmax warp may finish tile j + 1 before a slow
+        // one has finished tile j, and their arrivals must not complete the same phase
+        const int pb = j & 1;
+        if (!mbar_wait_warp(&bar[bPFull + pb], (j >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const uint64_t omn = sdesc_add(dO_mn, st * L::kQT), qmn = sdesc_add(dQ_mn, st * L::kQT);
-        const int pb = j & 1;
         const uint64_t apt = pb ? dPt[1] : dPt[0], ads = pb ? dDSt[1] : dDSt[0];
         const uint64_t bds = pb ? dDSt_mn[1] : dDSt_mn[0];
 #pragma unroll
@@ -389,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[bPFull]);
+      if (lane == 0) mbar_arrive(&bar[bPFull + pb]);
       ++j;
     }
     // ---------------------------------------------------------------- dK / dV epilogue
