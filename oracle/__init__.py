@@ -17,7 +17,9 @@ method (cited per function by page title and section):
   block by block, merged with the log-sum-exp identity, and their backward
   fed the merged out/lse;
 * ``paged``      - KV-parallel segmented prefill over a paged KV cache;
-* ``decode``     - one-query-per-sequence GQA varlen decode.
+* ``decode``     - one-query-per-sequence GQA varlen decode;
+* ``cached``     - EAGLE-3 cached attention: the causal sequence block plus the
+  per-position cache diagonals in one softmax, and its analytic gradients.
 
 Pins (tests marked ``not gpu``): brute force on tiny inputs, closed forms
 (q = 0 gives lse = log|visible| and out = mean of visible values), finite
