@@ -68,18 +68,59 @@ def profile_traffic(name: str):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and clock-event reasons sampled every 5 ms while the timed region runs.
+
+    Reads NVML (the library nvidia-smi reports from; read-only queries) in a thread, so that
+    a timed region of a few tens of milliseconds still holds several samples; falls back to
+    ``nvidia-smi -lms 100`` when NVML cannot be loaded."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
 
     def __init__(self, index: int):
         self.index = index
+        self.rows: list[tuple[float, float, list[str]]] = []
         self.lines: list[str] = []
         self.proc = None
+        self.nvml = None
+        self.stop_flag = threading.Event()
+        self.first = threading.Event()
+
+    def _handle(self, nv):
+        try:
+            import torch
+
+            pr = torch.cuda.get_device_properties(self.index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll(self, nv, h):
+        max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop_flag.is_set():
+            mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+            bits = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+            self.rows.append((mhz, max_mhz, [n for b, n in self.REASONS.items() if bits & b], time.monotonic()))
+            self.first.set()
+            time.sleep(0.005)
 
     def start(self):
+        try:
+            import pynvml as nv
+
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.nvml = nv
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            self.first.wait(timeout=5)
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE,
@@ -91,31 +132,47 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
+            parts = [x.strip() for x in line.strip().split(",")]
             if len(parts) != 8:
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+                names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+                self.rows.append((float(parts[0]), float(parts[1]),
+                                  [names[i] for i, v in enumerate(parts[4:8]) if v.lower() == "active"],
+                                  time.monotonic()))
             except ValueError:
                 continue
+
+    def begin(self):
+        """Marks the start of the timed region: earlier samples are dropped."""
+        self.t_begin = time.monotonic()
+
+    def stop(self):
+        t_end = time.monotonic()
+        if self.nvml is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            source = "nvml 5 ms"
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            source = "nvidia-smi 100 ms"
+        else:
+            return None
+        t0 = getattr(self, "t_begin", 0.0)
+        rows = [r for r in self.rows if t0 <= r[3] <= t_end]
         if not rows:
             return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        reasons = sorted({n for _, _, r, _ in rows for n in r})
         return {"sm_mhz": float(np.median([r[0] for r in rows])), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "source": source}
 
 
 # ----------------------------------------------------------------------------- workload
@@ -219,7 +276,7 @@ def extra_benchmarks(device, pk, pk_kind):
 
     import context_blockwise_causal_varlen_b200 as cbv
     from synth import torch_normal_bf16
-    from synth.workloads import long_doc, paged_prefill, varlen_decode
+    from synth.workloads import long_doc, packed_zigzag, paged_prefill, varlen_decode
 
     res = {}
     tf_peak = pk["bf16_tflops"]
@@ -247,6 +304,45 @@ def extra_benchmarks(device, pk, pk_kind):
                     "fwd_bwd_frac": (f_fwd + f_bwd) / (t_f + t_b) / 1e9 / tf_peak, "ms": t_f + t_b}
         del q, k, v, do, st
         torch.cuda.empty_cache()
+    # EAGLE-3 cached ring on the packed workload: the sequence block plus 3 cache diagonals.  The
+    # diagonals' cost is the time above the plain ring on the same sequence block, set against the
+    # bytes that the two diagonal kernels must move (and the fp32 block output they add).
+    w = packed_zigzag()
+    nb, S, H, D = 4, w.total, w.heads, w.head_dim
+    q = torch_normal_bf16((S, H, D), 31, device)
+    ck = torch_normal_bf16((nb, S, H, D), 32, device)
+    cv = torch_normal_bf16((nb, S, H, D), 33, device)
+    do = torch_normal_bf16((S, H, D), 34, device)
+    st = {}
+
+    def cfwd():
+        st["o"], st["l"] = cbv.cached_ring_fwd(q, ck, cv, w.cu_seqlens, w.cp)
+
+    def cbwd():
+        cbv.cached_ring_bwd(do, q, ck, cv, st["o"], st["l"], w.cu_seqlens, w.cp)
+
+    def pfwd():
+        st["po"], st["pl"] = cbv.zigzag_ring_fwd(q, ck[0], cv[0], w.cu_seqlens, w.cp)
+
+    def pbwd():
+        cbv.zigzag_ring_bwd(do, q, ck[0], cv[0], st["po"], st["pl"], w.cu_seqlens, w.cp)
+
+    cfwd()
+    pfwd()
+    t_cf, t_cb = timed(cfwd, 8, 3), timed(cbwd, 8, 3)
+    t_pf, t_pb = timed(pfwd, 8, 3), timed(pbwd, 8, 3)
+    e = S * H * D
+    diag_kv = 2 * (nb - 1) * S * H * D * 2
+    b_fwd = e * 2 + e * 4 + diag_kv + S * H * 8 + e * 2 + e * 2  # q, o32, k/v diagonals, lse r/w, out, o32's extra write
+    b_bwd = 3 * e * 2 + 2 * diag_kv + S * H * 4  # q, dO, out; k/v diagonals read, their gradients written; lse
+    pairs = visible_pairs(w.cu_seqlens)
+    f_all = 14 * D * H * pairs
+    res[f"cached_ring_{w.name}_NB{nb}"] = {
+        "fwd_bwd_tflops": f_all / (t_cf + t_cb) / 1e9, "ms": t_cf + t_cb, "plain_ms": t_pf + t_pb,
+        "diag_fwd_ms": t_cf - t_pf, "diag_bwd_ms": t_cb - t_pb,
+        "diag_fwd_gbs": b_fwd / max(t_cf - t_pf, 1e-6) / 1e6, "diag_bwd_gbs": b_bwd / max(t_cb - t_pb, 1e-6) / 1e6}
+    del q, ck, cv, do, st
+    torch.cuda.empty_cache()
     # paged KV-parallel prefill, round-robin shards
     for window in (0, 8192):
         w = paged_prefill(window=window)
@@ -427,6 +523,7 @@ def main():
     clocks = ClockSampler(local)
     clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.begin()
     t0.record()
     for _ in range(args.steps):
         step(record=True)

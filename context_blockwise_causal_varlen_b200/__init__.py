@@ -132,6 +132,20 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
+class CachedRingArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("cache_k", ctypes.c_void_p), ("cache_v", ctypes.c_void_p),
+        ("num_blocks", ctypes.c_int32), ("total", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("num_docs", ctypes.c_int32), ("cu_seqlens", c_i32p), ("max_seqlen", ctypes.c_int32),
+        ("cp", ctypes.c_int32), ("layout", ctypes.c_int32), ("scale", ctypes.c_float), ("window", ctypes.c_int32),
+        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
+        ("dq", ctypes.c_void_p), ("dcache_k", ctypes.c_void_p), ("dcache_v", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 EXPORTS = [
     "cbv_last_error_message", "cbv_abi_version", "cbv_read_status",
     "cbv_local_cu_seqlens", "cbv_half_cu_seqlens", "cbv_get_half_index", "cbv_get_half_lse", "cbv_rank_tokens",
@@ -141,6 +155,8 @@ EXPORTS = [
     "cbv_zigzag_ring_bwd", "cbv_block_bwd_workspace_size", "cbv_attn_block_bwd",
     "cbv_kvp_workspace_size", "cbv_kvp_segmented_prefill", "cbv_decode_workspace_size", "cbv_varlen_decode",
     "cbv_noalloc_scratch_bytes", "cbv_zigzag_ring_fwd_noalloc",
+    "cbv_cached_ring_fwd_workspace_size", "cbv_cached_ring_fwd", "cbv_cached_ring_bwd_workspace_size",
+    "cbv_cached_ring_bwd",
 ]
 
 
@@ -156,13 +172,15 @@ def _declare(L):
     L.cbv_rank_pair_counts.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i64p]
     L.cbv_ring_step.argtypes = [ctypes.c_int32] * 4 + [c_i32p, c_i32p]
     for name, st in (("block_fwd", BlockFwdArgs), ("zigzag_ring_fwd", RingArgs), ("zigzag_ring_bwd", RingArgs),
-                     ("block_bwd", BlockBwdArgs), ("kvp", KvpArgs), ("decode", DecodeArgs)):
+                     ("block_bwd", BlockBwdArgs), ("kvp", KvpArgs), ("decode", DecodeArgs),
+                     ("cached_ring_fwd", CachedRingArgs), ("cached_ring_bwd", CachedRingArgs)):
         f = getattr(L, f"cbv_{name}_workspace_size")
         f.argtypes = [ctypes.POINTER(st)]
         f.restype = ctypes.c_size_t
     for name, st in (("cbv_attn_block_fwd", BlockFwdArgs), ("cbv_zigzag_ring_fwd", RingArgs),
                      ("cbv_zigzag_ring_bwd", RingArgs), ("cbv_attn_block_bwd", BlockBwdArgs),
-                     ("cbv_kvp_segmented_prefill", KvpArgs), ("cbv_varlen_decode", DecodeArgs)):
+                     ("cbv_kvp_segmented_prefill", KvpArgs), ("cbv_varlen_decode", DecodeArgs),
+                     ("cbv_cached_ring_fwd", CachedRingArgs), ("cbv_cached_ring_bwd", CachedRingArgs)):
         getattr(L, name).argtypes = [ctypes.POINTER(st), ctypes.c_void_p]
     L.cbv_noalloc_scratch_bytes.restype = ctypes.c_size_t
     L.cbv_zigzag_ring_fwd_noalloc.argtypes = [ctypes.POINTER(RingArgs), ctypes.c_void_p]
@@ -316,6 +334,51 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_zigzag_ring_bwd(ctypes.byref(a), _stream(q.device)))
     return (dq, dk, dv, ws) if return_workspace else (dq, dk, dv)
+
+
+def _cached_args(q, cache_k, cache_v, cu, cp, scale, window, layout, max_seqlen, **tensors):
+    S, H, D = q.shape
+    return CachedRingArgs(**_header(CachedRingArgs), q=_ptr(q), cache_k=_ptr(cache_k), cache_v=_ptr(cache_v),
+                          num_blocks=cache_k.shape[0], total=S, num_heads=H, num_kv_heads=cache_k.shape[2],
+                          head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu), max_seqlen=max_seqlen, cp=cp,
+                          layout=_layout(layout), scale=_scale(scale), window=int(window),
+                          **{k: _ptr(t) for k, t in tensors.items()})
+
+
+def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
+                    max_seqlen: int = 0, out=None, lse=None, return_workspace=False):
+    """EAGLE-3 cached ring forward: block 0 of ``cache_k/cache_v [NB,S,Hkv,D]`` is the sequence
+    (ring over ``cp`` virtual ranks), blocks 1.. are per-position diagonals; one softmax.
+    Returns ``(out [S,H,D] bf16, lse [H,S] f32)``."""
+    q, cache_k, cache_v = _bf16(q, "q"), _bf16(cache_k, "cache_k"), _bf16(cache_v, "cache_v")
+    S, H, _ = q.shape
+    cu = _host_i32(cu_seqlens)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    a = _cached_args(q, cache_k, cache_v, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse)
+    ws = _workspace(lib().cbv_cached_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_cached_ring_fwd(ctypes.byref(a), _stream(q.device)))
+    return (out, lse, ws) if return_workspace else (out, lse)
+
+
+def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, scale=None, window: int = 0,
+                    layout="zigzag", max_seqlen: int = 0, dq=None, dcache_k=None, dcache_v=None,
+                    return_workspace=False):
+    """EAGLE-3 cached ring backward fed the merged out/lse: ``(dq, dcache_k, dcache_v)`` bf16."""
+    dout, q, cache_k, cache_v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (cache_k, "cache_k"),
+                                                               (cache_v, "cache_v"), (out, "out")))
+    cu = _host_i32(cu_seqlens)
+    dq = torch.empty_like(q) if dq is None else dq
+    dcache_k = torch.empty_like(cache_k) if dcache_k is None else dcache_k
+    dcache_v = torch.empty_like(cache_v) if dcache_v is None else dcache_v
+    lse = lse.contiguous()
+    a = _cached_args(q, cache_k, cache_v, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse, dout=dout,
+                     dq=dq, dcache_k=dcache_k, dcache_v=dcache_v)
+    ws = _workspace(lib().cbv_cached_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_cached_ring_bwd(ctypes.byref(a), _stream(q.device)))
+    return (dq, dcache_k, dcache_v, ws) if return_workspace else (dq, dcache_k, dcache_v)
 
 
 def attn_block_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int = 0, scale=None, causal: bool = True,

@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 OUT_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libcbv.so")
 
-SOURCES = ["api.cu", "fwd_pp.cu", "bwd.cu", "decode.cu", "misc.cu", "noalloc.cu", "plan.cpp"]
+SOURCES = ["api.cu", "fwd_pp.cu", "bwd.cu", "cached.cu", "decode.cu", "misc.cu", "noalloc.cu", "plan.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-lineinfo", f"-I{os.path.join(ROOT, 'include')}"]
 

@@ -688,15 +688,13 @@ size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a) {
   return c.off;
 }
 
-int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
-  int rc = ring_common_checks(a);
-  if (rc) return rc;
-  if (a->total == 0) return CBV_OK;  // no rows: nothing to write
-  if (!a->dout || !a->out || !a->lse || !a->dq || !a->dk || !a->dv) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+// Everything of the ring backward but the final dq conversion: dq stays in the fp32
+// accumulator carved from the workspace, returned through *dq_acc_out.
+static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_out) {
+  if (!a->dout || !a->out || !a->lse || !a->dk || !a->dv) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) || !aligned16(a->dout) ||
-      !aligned16(a->dq) || !aligned16(a->dk) || !aligned16(a->dv))
+      !aligned16(a->dk) || !aligned16(a->dv))
     return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
   Plan plan = plan_ring_bwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, Hkv, 128);
   Carve c(a->workspace);
@@ -706,6 +704,7 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   float* rows = static_cast<float*>(c.take((size_t)H * tp * 2 * sizeof(float)));
   float* dq_acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
+  int rc;
   BwdParams p{};
   if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, dq_acc, a->total, a->total, H, Hkv, D))) return rc;
   p.tasks = pd.tasks;
@@ -729,9 +728,21 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows, dq_acc, s),
                       "backward preprocess")))
     return rc;
-  const int grid = grid_of(plan.tasks.size(), 1);
-  if ((rc = launch_rc(launch_bwd(p, D, grid, s), "backward launch"))) return rc;
-  return launch_rc(launch_convert_bf16(dq_acc, a->dq, a->total * H * D, 1.f, s), "dq conversion");
+  *dq_acc_out = dq_acc;
+  return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch");
+}
+
+int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
+  int rc = ring_common_checks(a);
+  if (rc) return rc;
+  if (a->total == 0) return CBV_OK;  // no rows: nothing to write
+  if (!a->dq) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->dq)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* dq_acc = nullptr;
+  if ((rc = ring_bwd_core(a, s, &dq_acc))) return rc;
+  return launch_rc(launch_convert_bf16(dq_acc, a->dq, a->total * a->num_heads * a->head_dim, 1.f, s),
+                   "dq conversion");
 }
 
 static int block_bwd_checks(const cbv_block_bwd_args* a) {
@@ -799,6 +810,128 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
                       "backward preprocess")))
     return rc;
   return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch");
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------ EAGLE-3 cached ring
+namespace {
+
+// The ring arguments of block 0: the sequence keys and values are the first cache block.
+cbv_ring_args cached_block0(const cbv_cached_ring_args* a) {
+  cbv_ring_args r{};
+  r.struct_size = sizeof(cbv_ring_args);
+  r.abi_version = CBV_ABI_VERSION;
+  r.q = a->q;
+  r.k = a->cache_k;
+  r.v = a->cache_v;
+  r.total = a->total;
+  r.num_heads = a->num_heads;
+  r.num_kv_heads = a->num_kv_heads;
+  r.head_dim = a->head_dim;
+  r.num_docs = a->num_docs;
+  r.cu_seqlens = a->cu_seqlens;
+  r.max_seqlen = a->max_seqlen;
+  r.cp = a->cp;
+  r.layout = a->layout;
+  r.scale = a->scale;
+  r.causal = 1;
+  r.window = a->window;
+  r.schedule = CBV_SCHEDULE_FUSED;
+  r.out = a->out;
+  r.lse = a->lse;
+  r.dout = a->dout;
+  r.dq = a->dq;
+  r.dk = a->dcache_k;
+  r.dv = a->dcache_v;
+  r.workspace = a->workspace;
+  r.workspace_bytes = a->workspace_bytes;
+  return r;
+}
+
+int cached_checks(const cbv_cached_ring_args* a) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_cached_ring_args), a->abi_version);
+  if (rc) return rc;
+  if (a->num_blocks < 1 || a->num_blocks > cbv::cached_max_blocks())
+    return fail(CBV_ERR_BAD_ARG, "num_blocks must be in [1, %d]", cbv::cached_max_blocks());
+  cbv_ring_args r = cached_block0(a);
+  return ring_common_checks(&r);
+}
+
+size_t cached_fwd_bytes(const cbv_cached_ring_args* a, const cbv_ring_args& r) {
+  size_t b = ring_fwd_layout(&r).bytes;
+  if (a->num_blocks > 1) b = (b + 255) / 256 * 256 + (size_t)a->total * a->num_heads * a->head_dim * sizeof(float);
+  return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t cbv_cached_ring_fwd_workspace_size(const cbv_cached_ring_args* a) {
+  if (cached_checks(a)) return 0;
+  cbv_ring_args r = cached_block0(a);
+  return cached_fwd_bytes(a, r);
+}
+
+int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream) {
+  int rc = cached_checks(a);
+  if (rc) return rc;
+  if (a->total == 0) return CBV_OK;
+  cbv_ring_args r = cached_block0(a);
+  if (a->num_blocks == 1) return cbv_zigzag_ring_fwd(&r, stream);  // the sequence alone
+  if (!a->q || !a->cache_k || !a->cache_v || !a->out || !a->lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->q) || !aligned16(a->cache_k) || !aligned16(a->cache_v) || !aligned16(a->out))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  const size_t need = cached_fwd_bytes(a, r);
+  if (!a->workspace || a->workspace_bytes < need) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", need);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads;
+  RingFwdLayout L = ring_fwd_layout(&r);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, L.fused);
+  float* o32 = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
+  FwdParams p = ring_fwd_params(&r, &rc);
+  if (rc) return rc;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, L.fused, s))) return rc;
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)L.fused.tasks.size();
+  p.out = o32;  // block 0, normalised, fp32: the diagonals merge into it before rounding
+  p.out_mode = kOutF32;
+  if ((rc = launch_rc(launch_fwd_pingpong(p, D, false, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch")))
+    return rc;
+  return launch_rc(cbv::launch_diag_merge(a->q, a->cache_k, a->cache_v, a->num_blocks, a->total, H, a->num_kv_heads,
+                                          D, resolve_scale(a->scale, D), o32, a->lse, a->out, s),
+                   "diagonal merge");
+}
+
+size_t cbv_cached_ring_bwd_workspace_size(const cbv_cached_ring_args* a) {
+  if (cached_checks(a)) return 0;
+  cbv_ring_args r = cached_block0(a);
+  return cbv_zigzag_ring_bwd_workspace_size(&r);
+}
+
+int cbv_cached_ring_bwd(const cbv_cached_ring_args* a, void* stream) {
+  int rc = cached_checks(a);
+  if (rc) return rc;
+  if (a->total == 0) return CBV_OK;
+  cbv_ring_args r = cached_block0(a);
+  if (a->num_blocks == 1) return cbv_zigzag_ring_bwd(&r, stream);
+  if (!a->dq || !a->dcache_k || !a->dcache_v) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->dq)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* dq_acc = nullptr;
+  if ((rc = ring_bwd_core(&r, s, &dq_acc))) return rc;  // block 0 into dcache[0], dq in fp32
+  const int D = a->head_dim;
+  return launch_rc(cbv::launch_diag_grad(a->q, a->cache_k, a->cache_v, a->num_blocks, a->total, a->num_heads,
+                                         a->num_kv_heads, D, resolve_scale(a->scale, D), a->dout, a->out, a->lse,
+                                         dq_acc, a->dq, a->dcache_k, a->dcache_v, s),
+                   "diagonal gradients");
 }
 
 }  // extern "C"

@@ -31,7 +31,8 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_layouts_match_the_c_compiler():
     structs = {"cbv_block_fwd_args": cbv.BlockFwdArgs, "cbv_ring_args": cbv.RingArgs,
-               "cbv_block_bwd_args": cbv.BlockBwdArgs, "cbv_kvp_args": cbv.KvpArgs, "cbv_decode_args": cbv.DecodeArgs}
+               "cbv_block_bwd_args": cbv.BlockBwdArgs, "cbv_kvp_args": cbv.KvpArgs, "cbv_decode_args": cbv.DecodeArgs,
+               "cbv_cached_ring_args": cbv.CachedRingArgs}
     src = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
     for cname, st in structs.items():
         src.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
@@ -183,3 +184,45 @@ def test_empty_problems_return_ok_without_touching_the_device():
     # but a malformed empty call is still an error
     a, _ = _ring_args(cu=np.array([0], np.int32), head_dim=80)
     assert cbv.STATUS[cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None)] == "UNSUPPORTED_HEAD_DIM"
+
+
+def _cached_args(**kw):
+    cu = kw.pop("cu", np.array([0, 96, 256], np.int32))
+    a = cbv.CachedRingArgs(struct_size=ctypes.sizeof(cbv.CachedRingArgs), abi_version=cbv.ABI_VERSION, num_blocks=3,
+                           total=int(cu[-1]), num_heads=4, num_kv_heads=2, head_dim=128, num_docs=len(cu) - 1,
+                           cu_seqlens=cu.ctypes.data_as(cbv.c_i32p), cp=2)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, cu
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("num_blocks", 0, "BAD_ARG"),
+    ("num_blocks", 9, "BAD_ARG"),
+    ("head_dim", 96, "UNSUPPORTED_HEAD_DIM"),
+    ("num_kv_heads", 3, "GQA_MISMATCH"),
+    ("cp", 5, "NOT_DIVISIBLE_2CP"),
+    ("struct_size", 8, "VERSION"),
+    ("layout", 4, "BAD_ARG"),
+])
+def test_cached_ring_argument_errors_are_reported_before_any_launch(field, value, status):
+    a, cu = _cached_args(**{field: value})
+    for f in (cbv.lib().cbv_cached_ring_fwd, cbv.lib().cbv_cached_ring_bwd):
+        assert cbv.STATUS[f(ctypes.byref(a), None)] == status, cbv.lib().cbv_last_error_message()
+    assert cbv.lib().cbv_cached_ring_fwd_workspace_size(ctypes.byref(a)) == 0
+    assert cbv.lib().cbv_cached_ring_bwd_workspace_size(ctypes.byref(a)) == 0
+
+
+def test_cached_ring_workspace_holds_the_fp32_block_output():
+    a, cu = _cached_args()
+    n = cbv.lib().cbv_cached_ring_fwd_workspace_size(ctypes.byref(a))
+    assert n >= 256 * 4 * 128 * 4  # block 0's normalised output in fp32
+    a.num_blocks = 1  # the sequence alone: the plain ring forward's scratch
+    r, _ = _ring_args(num_heads=4, head_dim=128)
+    assert cbv.lib().cbv_cached_ring_fwd_workspace_size(ctypes.byref(a)) == \
+        cbv.lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(r))
+    assert cbv.lib().cbv_cached_ring_bwd_workspace_size(ctypes.byref(a)) == \
+        cbv.lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(r))
+    a, _ = _cached_args(cu=np.array([0, 0], np.int32))
+    assert cbv.lib().cbv_cached_ring_fwd(ctypes.byref(a), None) == 0
+    assert cbv.lib().cbv_cached_ring_bwd(ctypes.byref(a), None) == 0
