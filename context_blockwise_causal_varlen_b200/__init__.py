@@ -135,13 +135,14 @@ class DecodeArgs(ctypes.Structure):
 class CachedRingArgs(ctypes.Structure):
     _fields_ = [
         ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
-        ("q", ctypes.c_void_p), ("cache_k", ctypes.c_void_p), ("cache_v", ctypes.c_void_p),
-        ("num_blocks", ctypes.c_int32), ("total", ctypes.c_int64),
+        ("q", ctypes.c_void_p), ("cache_k", ctypes.POINTER(ctypes.c_void_p)),
+        ("cache_v", ctypes.POINTER(ctypes.c_void_p)), ("num_blocks", ctypes.c_int32), ("total", ctypes.c_int64),
         ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("num_docs", ctypes.c_int32), ("cu_seqlens", c_i32p), ("max_seqlen", ctypes.c_int32),
         ("cp", ctypes.c_int32), ("layout", ctypes.c_int32), ("scale", ctypes.c_float), ("window", ctypes.c_int32),
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
-        ("dq", ctypes.c_void_p), ("dcache_k", ctypes.c_void_p), ("dcache_v", ctypes.c_void_p),
+        ("dq", ctypes.c_void_p), ("dcache_k", ctypes.POINTER(ctypes.c_void_p)),
+        ("dcache_v", ctypes.POINTER(ctypes.c_void_p)),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
     ]
 
@@ -336,26 +337,43 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
     return (dq, dk, dv, ws) if return_workspace else (dq, dk, dv)
 
 
-def _cached_args(q, cache_k, cache_v, cu, cp, scale, window, layout, max_seqlen, **tensors):
+def _blocks(cache, name: str) -> list[torch.Tensor]:
+    """A stacked ``[NB, T, Hkv, D]`` tensor or a list of ``[T, Hkv, D]`` tensors, as bf16 blocks."""
+    blocks = list(cache.unbind(0)) if isinstance(cache, torch.Tensor) else list(cache)
+    return [_bf16(b, f"{name}[{i}]") for i, b in enumerate(blocks)]
+
+
+def _ptr_array(blocks):
+    return (ctypes.c_void_p * len(blocks))(*[b.data_ptr() for b in blocks])
+
+
+def _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, dck=None, dcv=None, **tensors):
     S, H, D = q.shape
-    return CachedRingArgs(**_header(CachedRingArgs), q=_ptr(q), cache_k=_ptr(cache_k), cache_v=_ptr(cache_v),
-                          num_blocks=cache_k.shape[0], total=S, num_heads=H, num_kv_heads=cache_k.shape[2],
-                          head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu), max_seqlen=max_seqlen, cp=cp,
-                          layout=_layout(layout), scale=_scale(scale), window=int(window),
-                          **{k: _ptr(t) for k, t in tensors.items()})
+    keep = [_ptr_array(ck), _ptr_array(cv)] + ([_ptr_array(dck), _ptr_array(dcv)] if dck is not None else [])
+    a = CachedRingArgs(**_header(CachedRingArgs), q=_ptr(q), num_blocks=len(ck), total=S, num_heads=H,
+                       num_kv_heads=ck[0].shape[1], head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu),
+                       max_seqlen=max_seqlen, cp=cp, layout=_layout(layout), scale=_scale(scale),
+                       window=int(window), **{k: _ptr(t) for k, t in tensors.items()})
+    a.cache_k = ctypes.cast(keep[0], ctypes.POINTER(ctypes.c_void_p))
+    a.cache_v = ctypes.cast(keep[1], ctypes.POINTER(ctypes.c_void_p))
+    if dck is not None:
+        a.dcache_k = ctypes.cast(keep[2], ctypes.POINTER(ctypes.c_void_p))
+        a.dcache_v = ctypes.cast(keep[3], ctypes.POINTER(ctypes.c_void_p))
+    return a, keep
 
 
 def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
                     max_seqlen: int = 0, out=None, lse=None, return_workspace=False):
-    """EAGLE-3 cached ring forward: block 0 of ``cache_k/cache_v [NB,S,Hkv,D]`` is the sequence
-    (ring over ``cp`` virtual ranks), blocks 1.. are per-position diagonals; one softmax.
-    Returns ``(out [S,H,D] bf16, lse [H,S] f32)``."""
-    q, cache_k, cache_v = _bf16(q, "q"), _bf16(cache_k, "cache_k"), _bf16(cache_v, "cache_v")
+    """EAGLE-3 cached ring forward.  ``cache_k`` / ``cache_v``: a stacked ``[NB,S,Hkv,D]`` tensor or a
+    list of ``[S,Hkv,D]`` tensors; block 0 is the sequence (ring over ``cp`` virtual ranks), blocks
+    1.. are per-position diagonals; one softmax.  Returns ``(out [S,H,D] bf16, lse [H,S] f32)``."""
+    q = _bf16(q, "q")
+    ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
     S, H, _ = q.shape
     cu = _host_i32(cu_seqlens)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
-    a = _cached_args(q, cache_k, cache_v, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse)
+    a, keep = _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse)
     ws = _workspace(lib().cbv_cached_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_cached_ring_fwd(ctypes.byref(a), _stream(q.device)))
@@ -365,16 +383,27 @@ def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window
 def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, scale=None, window: int = 0,
                     layout="zigzag", max_seqlen: int = 0, dq=None, dcache_k=None, dcache_v=None,
                     return_workspace=False):
-    """EAGLE-3 cached ring backward fed the merged out/lse: ``(dq, dcache_k, dcache_v)`` bf16."""
-    dout, q, cache_k, cache_v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (cache_k, "cache_k"),
-                                                               (cache_v, "cache_v"), (out, "out")))
+    """EAGLE-3 cached ring backward fed the merged out/lse: ``(dq, dcache_k, dcache_v)`` bf16.  The cache
+    gradients come back in the form of the cache (stacked tensor or list) unless given."""
+    dout, q, out = _bf16(dout, "dout"), _bf16(q, "q"), _bf16(out, "out")
+    ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
     cu = _host_i32(cu_seqlens)
     dq = torch.empty_like(q) if dq is None else dq
-    dcache_k = torch.empty_like(cache_k) if dcache_k is None else dcache_k
-    dcache_v = torch.empty_like(cache_v) if dcache_v is None else dcache_v
+    stacked = isinstance(cache_k, torch.Tensor)
+    if dcache_k is None:
+        dcache_k = torch.empty((len(ck),) + tuple(ck[0].shape), dtype=q.dtype, device=q.device) if stacked \
+            else [torch.empty_like(b) for b in ck]
+    if dcache_v is None:
+        dcache_v = torch.empty((len(cv),) + tuple(cv[0].shape), dtype=q.dtype, device=q.device) if stacked \
+            else [torch.empty_like(b) for b in cv]
+    dck, dcv = _blocks(dcache_k, "dcache_k"), _blocks(dcache_v, "dcache_v")
+    for b, given in zip(dck + dcv, list(dcache_k.unbind(0) if isinstance(dcache_k, torch.Tensor) else dcache_k)
+                        + list(dcache_v.unbind(0) if isinstance(dcache_v, torch.Tensor) else dcache_v)):
+        if b.data_ptr() != given.data_ptr():
+            raise CbvError(-2, "dcache blocks must be contiguous bf16 CUDA tensors")
     lse = lse.contiguous()
-    a = _cached_args(q, cache_k, cache_v, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse, dout=dout,
-                     dq=dq, dcache_k=dcache_k, dcache_v=dcache_v)
+    a, keep = _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, dck=dck, dcv=dcv, out=out, lse=lse,
+                           dout=dout, dq=dq)
     ws = _workspace(lib().cbv_cached_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_cached_ring_bwd(ctypes.byref(a), _stream(q.device)))

@@ -823,8 +823,8 @@ cbv_ring_args cached_block0(const cbv_cached_ring_args* a) {
   r.struct_size = sizeof(cbv_ring_args);
   r.abi_version = CBV_ABI_VERSION;
   r.q = a->q;
-  r.k = a->cache_k;
-  r.v = a->cache_v;
+  r.k = a->cache_k ? a->cache_k[0] : nullptr;
+  r.v = a->cache_v ? a->cache_v[0] : nullptr;
   r.total = a->total;
   r.num_heads = a->num_heads;
   r.num_kv_heads = a->num_kv_heads;
@@ -842,8 +842,8 @@ cbv_ring_args cached_block0(const cbv_cached_ring_args* a) {
   r.lse = a->lse;
   r.dout = a->dout;
   r.dq = a->dq;
-  r.dk = a->dcache_k;
-  r.dv = a->dcache_v;
+  r.dk = a->dcache_k ? a->dcache_k[0] : nullptr;
+  r.dv = a->dcache_v ? a->dcache_v[0] : nullptr;
   r.workspace = a->workspace;
   r.workspace_bytes = a->workspace_bytes;
   return r;
@@ -853,10 +853,31 @@ int cached_checks(const cbv_cached_ring_args* a) {
   if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
   int rc = check_header(a->struct_size, sizeof(cbv_cached_ring_args), a->abi_version);
   if (rc) return rc;
-  if (a->num_blocks < 1 || a->num_blocks > cbv::cached_max_blocks())
-    return fail(CBV_ERR_BAD_ARG, "num_blocks must be in [1, %d]", cbv::cached_max_blocks());
+  if (a->num_blocks < 1 || a->num_blocks > cbv::kCacheMaxBlocks)
+    return fail(CBV_ERR_BAD_ARG, "num_blocks must be in [1, %d]", cbv::kCacheMaxBlocks);
   cbv_ring_args r = cached_block0(a);
   return ring_common_checks(&r);
+}
+
+// The block addresses, checked: every block present and 16-byte aligned (gradients too when
+// `grads`).
+int cached_blocks(const cbv_cached_ring_args* a, bool grads, cbv::CacheBlocks* cb) {
+  *cb = cbv::CacheBlocks{};
+  if (!a->cache_k || !a->cache_v || (grads && (!a->dcache_k || !a->dcache_v)))
+    return fail(CBV_ERR_BAD_ARG, "NULL cache block array");
+  for (int i = 0; i < a->num_blocks; ++i) {
+    cb->k[i] = a->cache_k[i];
+    cb->v[i] = a->cache_v[i];
+    if (grads) {
+      cb->dk[i] = a->dcache_k[i];
+      cb->dv[i] = a->dcache_v[i];
+    }
+    if (!cb->k[i] || !cb->v[i] || (grads && (!cb->dk[i] || !cb->dv[i])))
+      return fail(CBV_ERR_BAD_ARG, "NULL cache block %d", i);
+    if (!aligned16(cb->k[i]) || !aligned16(cb->v[i]) || (grads && (!aligned16(cb->dk[i]) || !aligned16(cb->dv[i]))))
+      return fail(CBV_ERR_MISALIGNED, "cache block %d must be 16-byte aligned", i);
+  }
+  return CBV_OK;
 }
 
 size_t cached_fwd_bytes(const cbv_cached_ring_args* a, const cbv_ring_args& r) {
@@ -879,11 +900,12 @@ int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream) {
   int rc = cached_checks(a);
   if (rc) return rc;
   if (a->total == 0) return CBV_OK;
+  cbv::CacheBlocks cb;
+  if ((rc = cached_blocks(a, false, &cb))) return rc;
   cbv_ring_args r = cached_block0(a);
   if (a->num_blocks == 1) return cbv_zigzag_ring_fwd(&r, stream);  // the sequence alone
-  if (!a->q || !a->cache_k || !a->cache_v || !a->out || !a->lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
-  if (!aligned16(a->q) || !aligned16(a->cache_k) || !aligned16(a->cache_v) || !aligned16(a->out))
-    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  if (!a->q || !a->out || !a->lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->q) || !aligned16(a->out)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   const size_t need = cached_fwd_bytes(a, r);
   if (!a->workspace || a->workspace_bytes < need) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", need);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -905,8 +927,8 @@ int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream) {
   p.out_mode = kOutF32;
   if ((rc = launch_rc(launch_fwd_pingpong(p, D, false, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch")))
     return rc;
-  return launch_rc(cbv::launch_diag_merge(a->q, a->cache_k, a->cache_v, a->num_blocks, a->total, H, a->num_kv_heads,
-                                          D, resolve_scale(a->scale, D), o32, a->lse, a->out, s),
+  return launch_rc(cbv::launch_diag_merge(a->q, cb, a->num_blocks, a->total, H, a->num_kv_heads, D,
+                                          resolve_scale(a->scale, D), o32, a->lse, a->out, s),
                    "diagonal merge");
 }
 
@@ -920,17 +942,18 @@ int cbv_cached_ring_bwd(const cbv_cached_ring_args* a, void* stream) {
   int rc = cached_checks(a);
   if (rc) return rc;
   if (a->total == 0) return CBV_OK;
+  cbv::CacheBlocks cb;
+  if ((rc = cached_blocks(a, true, &cb))) return rc;
   cbv_ring_args r = cached_block0(a);
   if (a->num_blocks == 1) return cbv_zigzag_ring_bwd(&r, stream);
-  if (!a->dq || !a->dcache_k || !a->dcache_v) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!a->dq) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (!aligned16(a->dq)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* dq_acc = nullptr;
   if ((rc = ring_bwd_core(&r, s, &dq_acc))) return rc;  // block 0 into dcache[0], dq in fp32
   const int D = a->head_dim;
-  return launch_rc(cbv::launch_diag_grad(a->q, a->cache_k, a->cache_v, a->num_blocks, a->total, a->num_heads,
-                                         a->num_kv_heads, D, resolve_scale(a->scale, D), a->dout, a->out, a->lse,
-                                         dq_acc, a->dq, a->dcache_k, a->dcache_v, s),
+  return launch_rc(cbv::launch_diag_grad(a->q, cb, a->num_blocks, a->total, a->num_heads, a->num_kv_heads, D,
+                                         resolve_scale(a->scale, D), a->dout, a->out, a->lse, dq_acc, a->dq, s),
                    "diagonal gradients");
 }
 

@@ -2,7 +2,8 @@
 // page (_CachedRingAttention / _CachedZigZagRingAttention), merged into or differentiated
 // against the sequence block that the ring kernels handle.
 //
-// The cache holds num_blocks blocks [T, Hkv, D]; block 0 is the sequence (the ring's k/v),
+// The cache holds num_blocks blocks [T, Hkv, D], each at its own address; block 0 is the
+// sequence (the ring's k/v),
 // and every block i >= 1 contributes one key per query position t: score
 // s_i = scale <q_t, k_i[t]>, value v_i[t].  All blocks form one softmax per (t, head).
 //
@@ -25,7 +26,6 @@ namespace cbv {
 
 namespace {
 
-constexpr int kMaxBlocks = 8;  // cache blocks (the sequence and up to 7 diagonals)
 constexpr int kThreads = 256;
 
 // sum over the L lanes of this lane's row (L a power of two, rows aligned to L lanes)
@@ -64,12 +64,13 @@ __device__ __forceinline__ void load8f(const float* p, float* x) {
 }
 
 // One row per (t, q head h).  o32 holds block 0's normalised output; out and lse get the merge.
+__device__ __forceinline__ const __nv_bfloat16* blk(const void* p) { return static_cast<const __nv_bfloat16*>(p); }
+__device__ __forceinline__ __nv_bfloat16* blk_w(void* p) { return static_cast<__nv_bfloat16*>(p); }
+
 template <int D, int NB>
-__global__ void __launch_bounds__(kThreads) diag_merge_kernel(const __nv_bfloat16* __restrict__ q,
-                                                              const __nv_bfloat16* __restrict__ ck,
-                                                              const __nv_bfloat16* __restrict__ cv, int64_t T, int H,
-                                                              int Hkv, float scale, const float* __restrict__ o32,
-                                                              float* __restrict__ lse,
+__global__ void __launch_bounds__(kThreads) diag_merge_kernel(const __nv_bfloat16* __restrict__ q, const CacheBlocks cb,
+                                                              int64_t T, int H, int Hkv, float scale,
+                                                              const float* __restrict__ o32, float* __restrict__ lse,
                                                               __nv_bfloat16* __restrict__ out) {
   constexpr int L = D / 8;  // lanes per row
   const int64_t row = ((int64_t)blockIdx.x * kThreads + threadIdx.x) / L;
@@ -78,8 +79,7 @@ __global__ void __launch_bounds__(kThreads) diag_merge_kernel(const __nv_bfloat1
   const int64_t r = valid ? row : 0;  // out-of-range lanes compute on row 0 (for the shuffles) and store nothing
   const int64_t t = r / H;
   const int h = (int)(r % H);
-  const int64_t blk = T * Hkv * D;  // elements per cache block
-  const int64_t kvoff = (t * Hkv + h / (H / Hkv)) * D + c;
+  const int64_t kvoff = (t * Hkv + h / (H / Hkv)) * D + c;  // this row's k / v within a block
   float qv[8];
   load8(q + r * D + c, qv);
   const float l0 = lse[(int64_t)h * T + t];
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kThreads) diag_merge_kernel(const __nv_bfloat1
 #pragma unroll
   for (int i = 1; i < NB; ++i) {
     float k[8];
-    load8(ck + i * blk + kvoff, k);
+    load8(blk(cb.k[i]) + kvoff, k);
     float d = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) d = fmaf(qv[e], k[e], d);
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) diag_merge_kernel(const __nv_bfloat1
 #pragma unroll
   for (int i = 1; i < NB; ++i) {
     float v[8];
-    load8(cv + i * blk + kvoff, v);
+    load8(blk(cb.v[i]) + kvoff, v);
     const float w = __expf(s[i] - ln);
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, v[e], acc[e]);
@@ -122,10 +122,9 @@ __global__ void __launch_bounds__(kThreads) diag_merge_kernel(const __nv_bfloat1
 // Pass 2 forms each block's dk / dv from them, re-reading q and dO (now in L1).
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads) diag_grad_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ ck, const __nv_bfloat16* __restrict__ cv,
-    int64_t T, int H, int Hkv, float scale, const __nv_bfloat16* __restrict__ dout,
-    const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse, const float* __restrict__ dq_acc,
-    __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dck, __nv_bfloat16* __restrict__ dcv) {
+    const __nv_bfloat16* __restrict__ q, const CacheBlocks cb, int64_t T, int H, int Hkv, float scale,
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse,
+    const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq) {
   constexpr int L = D / 8;
   constexpr int kRows = kThreads / L;  // rows per CTA
   extern __shared__ float2 pds[];      // [kRows][G][NB - 1] of {p, dS}
@@ -137,7 +136,6 @@ __global__ void __launch_bounds__(kThreads) diag_grad_kernel(
   const int64_t r = valid ? row : 0;
   const int64_t t = r / Hkv;
   const int kh = (int)(r % Hkv);
-  const int64_t blk = T * Hkv * D;
   const int64_t kvoff = r * D + c;
   float2* my = pds + (size_t)lr * G * (NB - 1);
   for (int g = 0; g < G; ++g) {
@@ -156,8 +154,8 @@ __global__ void __launch_bounds__(kThreads) diag_grad_kernel(
 #pragma unroll
     for (int i = 1; i < NB; ++i) {
       float k[8], v[8];
-      load8(ck + i * blk + kvoff, k);
-      load8(cv + i * blk + kvoff, v);
+      load8(blk(cb.k[i]) + kvoff, k);
+      load8(blk(cb.v[i]) + kvoff, v);
       float sd = 0.f, pd = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -191,26 +189,24 @@ __global__ void __launch_bounds__(kThreads) diag_grad_kernel(
         dv[e] = fmaf(pd.x, dov[e], dv[e]);
       }
     }
-    store8(dck + i * blk + kvoff, dk);
-    store8(dcv + i * blk + kvoff, dv);
+    store8(blk_w(cb.dk[i]) + kvoff, dk);
+    store8(blk_w(cb.dv[i]) + kvoff, dv);
   }
 }
 
 template <int D, int NB>
-int merge_nb(const void* q, const void* ck, const void* cv, int64_t T, int H, int Hkv, float scale, const float* o32,
+int merge_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, float scale, const float* o32,
              float* lse, void* out, cudaStream_t stream) {
   const int64_t lanes = T * H * (D / 8);
   const int64_t blocks = (lanes + kThreads - 1) / kThreads;
-  diag_merge_kernel<D, NB><<<blocks, kThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(ck),
-      static_cast<const __nv_bfloat16*>(cv), T, H, Hkv, scale, o32, lse, static_cast<__nv_bfloat16*>(out));
+  diag_merge_kernel<D, NB><<<blocks, kThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), cb, T, H, Hkv,
+                                                             scale, o32, lse, static_cast<__nv_bfloat16*>(out));
   return (int)cudaGetLastError();
 }
 
 template <int D, int NB>
-int grad_nb(const void* q, const void* ck, const void* cv, int64_t T, int H, int Hkv, float scale, const void* dout,
-            const void* out, const float* lse, const float* dq_acc, void* dq, void* dck, void* dcv,
-            cudaStream_t stream) {
+int grad_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, float scale, const void* dout,
+            const void* out, const float* lse, const float* dq_acc, void* dq, cudaStream_t stream) {
   constexpr int kRows = kThreads / (D / 8);
   const size_t smem = (size_t)kRows * (H / Hkv) * (NB - 1) * sizeof(float2);
   auto kern = diag_grad_kernel<D, NB>;
@@ -221,62 +217,58 @@ int grad_nb(const void* q, const void* ck, const void* cv, int64_t T, int H, int
   }
   const int64_t blocks = (T * Hkv + kRows - 1) / kRows;
   auto c = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
-  auto w = [](void* p) { return static_cast<__nv_bfloat16*>(p); };
-  kern<<<blocks, kThreads, smem, stream>>>(c(q), c(ck), c(cv), T, H, Hkv, scale, c(dout), c(out), lse, dq_acc, w(dq),
-                                           w(dck), w(dcv));
+  kern<<<blocks, kThreads, smem, stream>>>(c(q), cb, T, H, Hkv, scale, c(dout), c(out), lse, dq_acc,
+                                           static_cast<__nv_bfloat16*>(dq));
   return (int)cudaGetLastError();
 }
 
 template <int D>
-int merge_d(int nb, const void* q, const void* ck, const void* cv, int64_t T, int H, int Hkv, float scale,
-            const float* o32, float* lse, void* out, cudaStream_t s) {
+int merge_d(int nb, const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, float scale, const float* o32,
+            float* lse, void* out, cudaStream_t s) {
   switch (nb) {
-    case 2: return merge_nb<D, 2>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
-    case 3: return merge_nb<D, 3>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
-    case 4: return merge_nb<D, 4>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
-    case 5: return merge_nb<D, 5>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
-    case 6: return merge_nb<D, 6>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
-    case 7: return merge_nb<D, 7>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
-    case 8: return merge_nb<D, 8>(q, ck, cv, T, H, Hkv, scale, o32, lse, out, s);
+    case 2: return merge_nb<D, 2>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
+    case 3: return merge_nb<D, 3>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
+    case 4: return merge_nb<D, 4>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
+    case 5: return merge_nb<D, 5>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
+    case 6: return merge_nb<D, 6>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
+    case 7: return merge_nb<D, 7>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
+    case 8: return merge_nb<D, 8>(q, cb, T, H, Hkv, scale, o32, lse, out, s);
     default: return (int)cudaErrorInvalidValue;
   }
 }
 
 template <int D>
-int grad_d(int nb, const void* q, const void* ck, const void* cv, int64_t T, int H, int Hkv, float scale,
-           const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq, void* dck, void* dcv,
-           cudaStream_t s) {
+int grad_d(int nb, const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, float scale, const void* dout,
+           const void* out, const float* lse, const float* dq_acc, void* dq, cudaStream_t s) {
   switch (nb) {
-    case 2: return grad_nb<D, 2>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
-    case 3: return grad_nb<D, 3>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
-    case 4: return grad_nb<D, 4>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
-    case 5: return grad_nb<D, 5>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
-    case 6: return grad_nb<D, 6>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
-    case 7: return grad_nb<D, 7>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
-    case 8: return grad_nb<D, 8>(q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, s);
+    case 2: return grad_nb<D, 2>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 3: return grad_nb<D, 3>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 4: return grad_nb<D, 4>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 5: return grad_nb<D, 5>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 6: return grad_nb<D, 6>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 7: return grad_nb<D, 7>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 8: return grad_nb<D, 8>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
     default: return (int)cudaErrorInvalidValue;
   }
 }
 
 }  // namespace
 
-int launch_diag_merge(const void* q, const void* ck, const void* cv, int nb, int64_t T, int H, int Hkv, int D,
-                      float scale, const float* o32, float* lse, void* out, cudaStream_t stream) {
+int launch_diag_merge(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
+                      const float* o32, float* lse, void* out, cudaStream_t stream) {
   if (T * H == 0) return 0;
-  if (D == 128) return merge_d<128>(nb, q, ck, cv, T, H, Hkv, scale, o32, lse, out, stream);
-  if (D == 64) return merge_d<64>(nb, q, ck, cv, T, H, Hkv, scale, o32, lse, out, stream);
+  if (D == 128) return merge_d<128>(nb, q, cb, T, H, Hkv, scale, o32, lse, out, stream);
+  if (D == 64) return merge_d<64>(nb, q, cb, T, H, Hkv, scale, o32, lse, out, stream);
   return (int)cudaErrorInvalidValue;
 }
 
-int launch_diag_grad(const void* q, const void* ck, const void* cv, int nb, int64_t T, int H, int Hkv, int D,
-                     float scale, const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq,
-                     void* dck, void* dcv, cudaStream_t stream) {
+int launch_diag_grad(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
+                     const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq,
+                     cudaStream_t stream) {
   if (T * Hkv == 0) return 0;
-  if (D == 128) return grad_d<128>(nb, q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, stream);
-  if (D == 64) return grad_d<64>(nb, q, ck, cv, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, dck, dcv, stream);
+  if (D == 128) return grad_d<128>(nb, q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, stream);
+  if (D == 64) return grad_d<64>(nb, q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, stream);
   return (int)cudaErrorInvalidValue;
 }
-
-int cached_max_blocks() { return kMaxBlocks; }
 
 }  // namespace cbv

@@ -72,16 +72,22 @@ int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, i
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
 
-// EAGLE-3 cached attention diagonals (cached.cu).  Cache blocks are [nb, T, Hkv, D] bf16,
-// lse is [H, T] fp32.  diag_merge: o32 holds block 0's normalised fp32 output; writes out
-// (bf16) and the merged lse in place.  diag_grad: with the merged out / lse, writes
-// dq = dq_acc + diagonal terms (bf16) and dcache_k / dcache_v blocks 1..nb-1.
-int launch_diag_merge(const void* q, const void* ck, const void* cv, int nb, int64_t T, int H, int Hkv, int D,
-                      float scale, const float* o32, float* lse, void* out, cudaStream_t stream);
-int launch_diag_grad(const void* q, const void* ck, const void* cv, int nb, int64_t T, int H, int Hkv, int D,
-                     float scale, const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq,
-                     void* dck, void* dcv, cudaStream_t stream);
-int cached_max_blocks();
+// EAGLE-3 cached attention diagonals (cached.cu).  Each cache block is [T, Hkv, D] bf16 at its
+// own address; lse is [H, T] fp32.  diag_merge: o32 holds block 0's normalised fp32 output;
+// writes out (bf16) and the merged lse in place.  diag_grad: with the merged out / lse, writes
+// dq = dq_acc + diagonal terms (bf16) and the gradients of blocks 1..nb-1.
+constexpr int kCacheMaxBlocks = 8;
+struct CacheBlocks {
+  const void* k[kCacheMaxBlocks];
+  const void* v[kCacheMaxBlocks];
+  void* dk[kCacheMaxBlocks];
+  void* dv[kCacheMaxBlocks];
+};
+int launch_diag_merge(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
+                      const float* o32, float* lse, void* out, cudaStream_t stream);
+int launch_diag_grad(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
+                     const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq,
+                     cudaStream_t stream);
 // Standalone merge of (block_out, block_lse) into a running fp32 (out, lse).
 int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
                  float* weight_out, int64_t seqlen, int32_t heads, int32_t head_dim, cudaStream_t stream);

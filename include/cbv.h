@@ -215,42 +215,45 @@ size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a);
 int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream);
 
 /* ========================================================================= EAGLE-3 cached ring
- * NeMo AutoModel ring_attention, _CachedZigZagRingAttention (layout = CBV_LAYOUT_ZIGZAG) and
- * _CachedRingAttention (CBV_LAYOUT_CONTIGUOUS): attention of the packed batch over a KV cache
- * of num_blocks blocks, cache_k[i] / cache_v[i] of shape [total, num_kv_heads, head_dim]
- * (the pages' [B, num_blocks, T, H, D] with B = 1, block axis first).  Block 0 is the sequence
- * itself and is attended causally (sliding window optional) the ring way, exactly as
- * cbv_zigzag_ring_fwd; every block i >= 1 adds one key per query token t, the cache entry at
- * the same position (the per-position diagonal): score scale <q_t, cache_k[i][t]>, value
- * cache_v[i][t].  All keys of a row form ONE softmax: the diagonals are merged into block 0's
- * result with the log-sum-exp identity of update_out_and_lse.  The backward is fed the merged
- * out and lse: block 0 by the ring backward, the diagonals in closed form (p_i = exp(s_i - lse),
- * dS_i = p_i (<dO_t, v_i[t]> - <dO_t, out_t>), dv_i[t] = sum over the kv head's q heads of
- * p_i dO_t, dk_i[t] = scale sum dS_i q_t, dq_t += scale dS_i k_i[t]).
+ * NeMo AutoModel ring_attention, _CachedZigZagRingAttention / cached_zigzag_ring_attention
+ * (layout = CBV_LAYOUT_ZIGZAG) and _CachedRingAttention / cached_ring_attention
+ * (CBV_LAYOUT_CONTIGUOUS): attention of the packed batch over a KV cache of num_blocks
+ * blocks, each [total, num_kv_heads, head_dim] (the pages' list of [B, T, H, D] tensors, or the
+ * block axis of [B, num_blocks, T, H, D], with B = 1).  Block 0 is the sequence itself and is
+ * attended causally (sliding window optional) the ring way, exactly as cbv_zigzag_ring_fwd;
+ * every block i >= 1 adds one key per query token t, the cache entry at the same position
+ * (the per-position diagonal): score scale <q_t, cache_k[i][t]>, value cache_v[i][t].  All keys
+ * of a row form ONE softmax: the diagonals are merged into block 0's result with the
+ * log-sum-exp identity of update_out_and_lse (ring_attention._merge_diag).  The backward is fed
+ * the merged out and lse: block 0 by the ring backward, the diagonals in closed form
+ * (p_i = exp(s_i - lse), dS_i = p_i (<dO_t, v_i[t]> - <dO_t, out_t>); dv_i[t] and dk_i[t] sum
+ * p_i dO_t and scale dS_i q_t over the kv head's q heads; dq_t += scale dS_i k_i[t]).
+ * The blocks are passed as host arrays of num_blocks device pointers, so separate tensors and
+ * slices of one stacked tensor serve alike; every pointer must be 16-byte aligned.
  * 1 <= num_blocks <= 8 (else CBV_ERR_BAD_ARG); causal only, fused schedule; the other rules,
  * errors and layouts are those of cbv_ring_args.  Every dcache block is written (not added). */
 typedef struct cbv_cached_ring_args {
-  uint32_t struct_size; /* sizeof(cbv_cached_ring_args) */
-  uint32_t abi_version; /* CBV_ABI_VERSION */
-  const void* q;        /* device bf16 [total, num_heads, head_dim] */
-  const void* cache_k;  /* device bf16 [num_blocks, total, num_kv_heads, head_dim] */
-  const void* cache_v;
+  uint32_t struct_size;        /* sizeof(cbv_cached_ring_args) */
+  uint32_t abi_version;        /* CBV_ABI_VERSION */
+  const void* q;               /* device bf16 [total, num_heads, head_dim] */
+  const void* const* cache_k;  /* host array [num_blocks] of device bf16 [total, num_kv_heads, head_dim] */
+  const void* const* cache_v;
   int32_t num_blocks;
   int64_t total;
   int32_t num_heads, num_kv_heads, head_dim;
   int32_t num_docs;
-  const int32_t* cu_seqlens; /* host int32 [num_docs+1], GLOBAL */
-  int32_t max_seqlen;        /* 0 or >= every document length */
-  int32_t cp;                /* virtual ranks, >= 1 */
-  int32_t layout;            /* cbv_layout */
+  const int32_t* cu_seqlens;   /* host int32 [num_docs+1], GLOBAL */
+  int32_t max_seqlen;          /* 0 or >= every document length */
+  int32_t cp;                  /* virtual ranks, >= 1 */
+  int32_t layout;              /* cbv_layout */
   float scale;
   int32_t window;
-  void* out;                 /* device bf16 [total, num_heads, head_dim]: forward output, backward input */
-  float* lse;                /* device f32 [num_heads, total]: forward output, backward input (merged) */
-  const void* dout;          /* backward: device bf16 [total, num_heads, head_dim] */
-  void* dq;                  /* backward: device bf16 [total, num_heads, head_dim] */
-  void* dcache_k;            /* backward: device bf16 [num_blocks, total, num_kv_heads, head_dim] */
-  void* dcache_v;
+  void* out;                   /* device bf16 [total, num_heads, head_dim]: forward output, backward input */
+  float* lse;                  /* device f32 [num_heads, total]: forward output, backward input (merged) */
+  const void* dout;            /* backward: device bf16 [total, num_heads, head_dim] */
+  void* dq;                    /* backward: device bf16 [total, num_heads, head_dim] */
+  void* const* dcache_k;       /* backward: host array [num_blocks] of device bf16 outputs, shaped as cache_k */
+  void* const* dcache_v;
   void* workspace;
   size_t workspace_bytes;
 } cbv_cached_ring_args;

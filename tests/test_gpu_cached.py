@@ -100,3 +100,22 @@ def test_window_of_one_sees_only_the_diagonals_and_itself():
     ro, rl = C.cached_fwd(f64(q), f64(ck), f64(cv), cu, 0.2, window=1)
     check_out(host(out), ro)
     check_lse(host(lse), rl)
+
+
+def test_separate_block_tensors_equal_the_stacked_cache():
+    # the public form: the cache as a list of [S, Hkv, D] tensors at unrelated addresses
+    cu, q, ck, cv, do = _case(16, [256, 128], 4, 2, 128, 3)
+    tq, tdo = dev(q), dev(do)
+    sk, sv = dev(ck), dev(cv)
+    lk = [dev(ck[i]) for i in range(3)]
+    lv = [dev(cv[i]) for i in range(3)]
+    out_s, lse_s = cbv.cached_ring_fwd(tq, sk, sv, cu, 2)
+    out_l, lse_l = cbv.cached_ring_fwd(tq, lk, lv, cu, 2)
+    dq_s, dk_s, dv_s = cbv.cached_ring_bwd(tdo, tq, sk, sv, out_s, lse_s, cu, 2)
+    dq_l, dk_l, dv_l = cbv.cached_ring_bwd(tdo, tq, lk, lv, out_l, lse_l, cu, 2)
+    sync()
+    assert torch.equal(out_s, out_l) and torch.equal(lse_s, lse_l)
+    assert isinstance(dk_l, list) and len(dk_l) == 3 and dk_s.shape == (3, 384, 2, 128)
+    for i in range(3):  # key-stationary block 0 and the closed-form diagonals are deterministic
+        assert torch.equal(dk_s[i], dk_l[i]) and torch.equal(dv_s[i], dv_l[i])
+    check_rel(host(dq_l), host(dq_s), rel=8e-3, what="dq")
