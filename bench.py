@@ -304,6 +304,16 @@ def extra_benchmarks(device, pk, pk_kind):
                     "fwd_bwd_frac": (f_fwd + f_bwd) / (t_f + t_b) / 1e9 / tf_peak, "ms": t_f + t_b}
         del q, k, v, do, st
         torch.cuda.empty_cache()
+    # deterministic backward (dq summed in 64-bit fixed point) against the default, packed workload
+    w = packed_zigzag()
+    q, k, v, do = make_ring_inputs(w.cu_seqlens, w.heads, w.head_dim, 41, device)
+    o, l = cbv.zigzag_ring_fwd(q, k, v, w.cu_seqlens, w.cp)
+    t_fast = timed(lambda: cbv.zigzag_ring_bwd(do, q, k, v, o, l, w.cu_seqlens, w.cp), 8, 3)
+    t_det = timed(lambda: cbv.zigzag_ring_bwd(do, q, k, v, o, l, w.cu_seqlens, w.cp, deterministic=True), 8, 3)
+    f_bwd = 10 * w.head_dim * w.heads * visible_pairs(w.cu_seqlens)
+    res[f"deterministic_bwd_{w.name}"] = {"bwd_tflops": f_bwd / t_det / 1e9, "ms": t_det, "default_ms": t_fast}
+    del q, k, v, do, o, l
+    torch.cuda.empty_cache()
     # EAGLE-3 cached ring on the packed workload: the sequence block plus 3 cache diagonals.  The
     # diagonals' cost is the time above the plain ring on the same sequence block, set against the
     # bytes that the two diagonal kernels must move (and the fp32 block output they add).

@@ -81,7 +81,7 @@ class RingArgs(ctypes.Structure):
         ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("num_docs", ctypes.c_int32), ("cu_seqlens", c_i32p), ("max_seqlen", ctypes.c_int32),
         ("cp", ctypes.c_int32), ("layout", ctypes.c_int32), ("scale", ctypes.c_float), ("causal", ctypes.c_int32),
-        ("window", ctypes.c_int32), ("schedule", ctypes.c_int32),
+        ("window", ctypes.c_int32), ("schedule", ctypes.c_int32), ("deterministic", ctypes.c_int32),
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
         ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
@@ -98,7 +98,7 @@ class BlockBwdArgs(ctypes.Structure):
         ("num_docs", ctypes.c_int32),
         ("cu_seqlens_q", c_i32p), ("cu_seqlens_k", c_i32p), ("q_pos_base", c_i32p), ("k_pos_base", c_i32p),
         ("scale", ctypes.c_float), ("causal", ctypes.c_int32), ("window", ctypes.c_int32),
-        ("dq_acc", ctypes.c_void_p), ("dk_acc", ctypes.c_void_p), ("dv_acc", ctypes.c_void_p),
+        ("deterministic", ctypes.c_int32), ("dq_acc", ctypes.c_void_p), ("dk_acc", ctypes.c_void_p), ("dv_acc", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
     ]
 
@@ -140,7 +140,7 @@ class CachedRingArgs(ctypes.Structure):
         ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("num_docs", ctypes.c_int32), ("cu_seqlens", c_i32p), ("max_seqlen", ctypes.c_int32),
         ("cp", ctypes.c_int32), ("layout", ctypes.c_int32), ("scale", ctypes.c_float), ("window", ctypes.c_int32),
-        ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
+        ("deterministic", ctypes.c_int32), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dout", ctypes.c_void_p),
         ("dq", ctypes.c_void_p), ("dcache_k", ctypes.POINTER(ctypes.c_void_p)),
         ("dcache_v", ctypes.POINTER(ctypes.c_void_p)),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
@@ -319,8 +319,9 @@ def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, l
 
 
 def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
-                    max_seqlen: int = 0, dq=None, dk=None, dv=None, return_workspace=False):
-    """Ring backward fed the merged out/lse: ``(dq, dk, dv)`` bf16."""
+                    max_seqlen: int = 0, dq=None, dk=None, dv=None, return_workspace=False, deterministic=False):
+    """Ring backward fed the merged out/lse: ``(dq, dk, dv)`` bf16.  ``deterministic``: dq summed in
+    64-bit fixed point, bit-identical from run to run."""
     dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
     S, H, D = q.shape
     cu = _host_i32(cu_seqlens)
@@ -330,7 +331,8 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
     a = RingArgs(**_header(RingArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), total=S, num_heads=H, num_kv_heads=k.shape[1],
                  head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu), max_seqlen=max_seqlen, cp=cp,
                  layout=_layout(layout), scale=_scale(scale), causal=1, window=int(window), schedule=0,
-                 out=_ptr(out), lse=_ptr(lse.contiguous()), dout=_ptr(dout), dq=_ptr(dq), dk=_ptr(dk), dv=_ptr(dv))
+                 deterministic=int(bool(deterministic)), out=_ptr(out), lse=_ptr(lse.contiguous()), dout=_ptr(dout),
+                 dq=_ptr(dq), dk=_ptr(dk), dv=_ptr(dv))
     ws = _workspace(lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_zigzag_ring_bwd(ctypes.byref(a), _stream(q.device)))
@@ -347,13 +349,15 @@ def _ptr_array(blocks):
     return (ctypes.c_void_p * len(blocks))(*[b.data_ptr() for b in blocks])
 
 
-def _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, dck=None, dcv=None, **tensors):
+def _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, dck=None, dcv=None, deterministic=False,
+                 **tensors):
     S, H, D = q.shape
     keep = [_ptr_array(ck), _ptr_array(cv)] + ([_ptr_array(dck), _ptr_array(dcv)] if dck is not None else [])
     a = CachedRingArgs(**_header(CachedRingArgs), q=_ptr(q), num_blocks=len(ck), total=S, num_heads=H,
                        num_kv_heads=ck[0].shape[1], head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu),
                        max_seqlen=max_seqlen, cp=cp, layout=_layout(layout), scale=_scale(scale),
-                       window=int(window), **{k: _ptr(t) for k, t in tensors.items()})
+                       window=int(window), deterministic=int(bool(deterministic)),
+                       **{k: _ptr(t) for k, t in tensors.items()})
     a.cache_k = ctypes.cast(keep[0], ctypes.POINTER(ctypes.c_void_p))
     a.cache_v = ctypes.cast(keep[1], ctypes.POINTER(ctypes.c_void_p))
     if dck is not None:
@@ -382,7 +386,7 @@ def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window
 
 def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, scale=None, window: int = 0,
                     layout="zigzag", max_seqlen: int = 0, dq=None, dcache_k=None, dcache_v=None,
-                    return_workspace=False):
+                    return_workspace=False, deterministic=False):
     """EAGLE-3 cached ring backward fed the merged out/lse: ``(dq, dcache_k, dcache_v)`` bf16.  The cache
     gradients come back in the form of the cache (stacked tensor or list) unless given."""
     dout, q, out = _bf16(dout, "dout"), _bf16(q, "q"), _bf16(out, "out")
@@ -402,8 +406,8 @@ def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, sc
         if b.data_ptr() != given.data_ptr():
             raise CbvError(-2, "dcache blocks must be contiguous bf16 CUDA tensors")
     lse = lse.contiguous()
-    a, keep = _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, dck=dck, dcv=dcv, out=out, lse=lse,
-                           dout=dout, dq=dq)
+    a, keep = _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, dck=dck, dcv=dcv,
+                           deterministic=deterministic, out=out, lse=lse, dout=dout, dq=dq)
     ws = _workspace(lib().cbv_cached_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_cached_ring_bwd(ctypes.byref(a), _stream(q.device)))
@@ -449,7 +453,8 @@ def attn_merge(out, lse, block_out, block_lse, return_weight: bool = False):
 
 
 def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=None, causal: bool = True,
-                   window: int = 0, q_pos_base=None, k_pos_base=None, dq_acc=None, dk_acc=None, dv_acc=None):
+                   window: int = 0, q_pos_base=None, k_pos_base=None, dq_acc=None, dk_acc=None, dv_acc=None,
+                   deterministic=False):
     """One block's backward fed the merged ``(out, lse)``; adds into f32 ``(dq_acc, dk_acc, dv_acc)``."""
     dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
     Sq, H, D = q.shape
@@ -465,7 +470,8 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
                      lse=_ptr(lse.contiguous()), total_q=Sq, total_k=Sk, num_heads=H, num_kv_heads=Hkv, head_dim=D,
                      num_docs=len(cq) - 1, cu_seqlens_q=_p32(cq), cu_seqlens_k=_p32(ck), q_pos_base=_p32(qb),
                      k_pos_base=_p32(kb), scale=_scale(scale), causal=int(bool(causal)), window=int(window),
-                     dq_acc=_ptr(dq_acc), dk_acc=_ptr(dk_acc), dv_acc=_ptr(dv_acc))
+                     deterministic=int(bool(deterministic)), dq_acc=_ptr(dq_acc), dk_acc=_ptr(dk_acc),
+                     dv_acc=_ptr(dv_acc))
     ws = _workspace(lib().cbv_block_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_attn_block_bwd(ctypes.byref(a), _stream(q.device)))

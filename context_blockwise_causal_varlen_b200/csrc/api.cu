@@ -684,29 +684,35 @@ size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a) {
   carve_plan(c, plan);
   c.take((size_t)a->num_heads * pad4(a->total) * sizeof(float));           // Delta
   c.take((size_t)a->num_heads * pad4(a->total) * sizeof(float));           // lse * log2e
-  c.take((size_t)a->total * a->num_heads * a->head_dim * sizeof(float));   // dq accumulator
+  c.take(a->deterministic ? (size_t)fixed_tpad(a->total) * a->num_heads * a->head_dim * 8  // dq accumulator
+                          : (size_t)a->total * a->num_heads * a->head_dim * 4);
   return c.off;
 }
 
-// Everything of the ring backward but the final dq conversion: dq stays in the fp32
-// accumulator carved from the workspace, returned through *dq_acc_out.
-static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_out) {
+// Everything of the ring backward but the final dq conversion: dq stays in the accumulator
+// carved from the workspace (fp32, or 64-bit fixed point when a->deterministic), returned
+// through *dq_acc_out / *dq_fixed_out (the other one is set to null).
+static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_out,
+                         unsigned long long** dq_fixed_out) {
   if (!a->dout || !a->out || !a->lse || !a->dk || !a->dv) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out) || !aligned16(a->dout) ||
       !aligned16(a->dk) || !aligned16(a->dv))
     return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  const bool det = a->deterministic != 0;
   Plan plan = plan_ring_bwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, Hkv, 128);
   Carve c(a->workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, plan);
   const int64_t tp = pad4(a->total);
   float* rows = static_cast<float*>(c.take((size_t)H * tp * 2 * sizeof(float)));
-  float* dq_acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
+  const size_t dq_bytes = det ? (size_t)fixed_tpad(a->total) * H * D * 8 : (size_t)a->total * H * D * 4;
+  void* dq_buf = c.take(dq_bytes);
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   int rc;
   BwdParams p{};
-  if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, dq_acc, a->total, a->total, H, Hkv, D))) return rc;
+  if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, static_cast<float*>(dq_buf), a->total, a->total, H, Hkv, D)))
+    return rc;
   p.tasks = pd.tasks;
   p.segs = pd.segs;
   p.num_tasks = (int)plan.tasks.size();
@@ -722,13 +728,16 @@ static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_
   p.dkv_stride_t = (int64_t)Hkv * D;
   p.dkv_stride_h = D;
   p.dkv_accumulate = 0;
+  p.dq_fixed = det ? static_cast<unsigned long long*>(dq_buf) : nullptr;
+  p.dq_fixed_tpad = fixed_tpad(a->total);
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows, dq_acc, s),
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows, dq_buf, dq_bytes, s),
                       "backward preprocess")))
     return rc;
-  *dq_acc_out = dq_acc;
+  *dq_acc_out = det ? nullptr : static_cast<float*>(dq_buf);
+  *dq_fixed_out = p.dq_fixed;
   return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch");
 }
 
@@ -740,9 +749,12 @@ int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
   if (!aligned16(a->dq)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* dq_acc = nullptr;
-  if ((rc = ring_bwd_core(a, s, &dq_acc))) return rc;
-  return launch_rc(launch_convert_bf16(dq_acc, a->dq, a->total * a->num_heads * a->head_dim, 1.f, s),
-                   "dq conversion");
+  unsigned long long* dq_fixed = nullptr;
+  if ((rc = ring_bwd_core(a, s, &dq_acc, &dq_fixed))) return rc;
+  const int64_t n = a->total * a->num_heads * a->head_dim;
+  if (dq_fixed)
+    return launch_rc(launch_fixed_to_bf16(dq_fixed, a->dq, a->total, a->num_heads, a->head_dim, s), "dq conversion");
+  return launch_rc(launch_convert_bf16(dq_acc, a->dq, n, 1.f, s), "dq conversion");
 }
 
 static int block_bwd_checks(const cbv_block_bwd_args* a) {
@@ -769,6 +781,7 @@ size_t cbv_block_bwd_workspace_size(const cbv_block_bwd_args* a) {
   carve_plan(c, plan);
   c.take((size_t)a->num_heads * pad4(a->total_q) * sizeof(float));
   c.take((size_t)a->num_heads * pad4(a->total_q) * sizeof(float));
+  if (a->deterministic) c.take((size_t)fixed_tpad(a->total_q) * a->num_heads * a->head_dim * 8);  // fixed-point dq
   return c.off;
 }
 
@@ -785,9 +798,13 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   PlanDev pd = carve_plan(c, plan);
   const int64_t tp = pad4(a->total_q);
   float* rows = static_cast<float*>(c.take((size_t)H * tp * 2 * sizeof(float)));
+  const size_t fix_bytes = a->deterministic ? (size_t)fixed_tpad(a->total_q) * H * D * 8 : 0;
+  auto* dq_fixed = a->deterministic ? static_cast<unsigned long long*>(c.take(fix_bytes)) : nullptr;
   if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
   BwdParams p{};
   if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, a->dq_acc, a->total_q, a->total_k, H, Hkv, D))) return rc;
+  p.dq_fixed = dq_fixed;
+  p.dq_fixed_tpad = fixed_tpad(a->total_q);
   p.tasks = pd.tasks;
   p.segs = pd.segs;
   p.num_tasks = (int)plan.tasks.size();
@@ -806,10 +823,12 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, rows, nullptr, s),
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, rows, dq_fixed, fix_bytes, s),
                       "backward preprocess")))
     return rc;
-  return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch");
+  if ((rc = launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch"))) return rc;
+  if (!dq_fixed) return CBV_OK;
+  return launch_rc(launch_fixed_add_f32(dq_fixed, a->dq_acc, a->total_q, H, D, s), "dq accumulation");
 }
 
 }  // extern "C"
@@ -838,6 +857,7 @@ cbv_ring_args cached_block0(const cbv_cached_ring_args* a) {
   r.causal = 1;
   r.window = a->window;
   r.schedule = CBV_SCHEDULE_FUSED;
+  r.deterministic = a->deterministic;
   r.out = a->out;
   r.lse = a->lse;
   r.dout = a->dout;
@@ -950,10 +970,12 @@ int cbv_cached_ring_bwd(const cbv_cached_ring_args* a, void* stream) {
   if (!aligned16(a->dq)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* dq_acc = nullptr;
-  if ((rc = ring_bwd_core(&r, s, &dq_acc))) return rc;  // block 0 into dcache[0], dq in fp32
+  unsigned long long* dq_fixed = nullptr;
+  if ((rc = ring_bwd_core(&r, s, &dq_acc, &dq_fixed))) return rc;  // block 0 into dcache[0], dq kept unrounded
   const int D = a->head_dim;
   return launch_rc(cbv::launch_diag_grad(a->q, cb, a->num_blocks, a->total, a->num_heads, a->num_kv_heads, D,
-                                         resolve_scale(a->scale, D), a->dout, a->out, a->lse, dq_acc, a->dq, s),
+                                         resolve_scale(a->scale, D), a->dout, a->out, a->lse, dq_acc, dq_fixed,
+                                         a->dq, s),
                    "diagonal gradients");
 }
 

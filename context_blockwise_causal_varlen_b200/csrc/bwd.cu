@@ -463,20 +463,50 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[bDQFree]);
+      if (p.dq_fixed == nullptr) {
 #pragma unroll
-      for (int pc = 0; pc < BM / kDQRows; ++pc) {
-        float* region = region0 + (pc & 1) * (L::kDQBuf / 4);
-        if (lane == 0) bulk_wait_group_read<1>();  // the reduce that last used this buffer has read it
-        __syncwarp();
-        if (dvalid) {
+        for (int pc = 0; pc < BM / kDQRows; ++pc) {
+          float* region = region0 + (pc & 1) * (L::kDQBuf / 4);
+          if (lane == 0) bulk_wait_group_read<1>();  // the reduce that last used this buffer has read it
+          __syncwarp();
+          if (dvalid) {
 #pragma unroll
-          for (int c = 0; c < kDQRows; ++c) region[c * DW + lane] = __uint_as_float(v[pc * kDQRows + c]) * p.scale;
+            for (int c = 0; c < kDQRows; ++c) region[c * DW + lane] = __uint_as_float(v[pc * kDQRows + c]) * p.scale;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row + pc * kDQRows);
+            bulk_commit_group();
+          }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_3d(&p.tm_dq, region, quarter * DW, r.head, r.q_row + pc * kDQRows);
-          bulk_commit_group();
+      } else {
+        // Deterministic: 8-row slices of 64-bit fixed point (units of 2^-32) in the same buffers,
+        // each added by one integer bulk reduce (the accumulator keeps a warp's rows contiguous).
+        // Rows past the tile's valid rows hold exact zeros, as in the fp32 path.
+        constexpr int kFixRows = kDQRows / 2;
+        unsigned long long* fregion0 = reinterpret_cast<unsigned long long*>(region0);
+        const float fscale = p.scale * 4294967296.f;
+#pragma unroll
+        for (int pc = 0; pc < BM / kFixRows; ++pc) {
+          unsigned long long* region = fregion0 + (pc & 1) * (L::kDQBuf / 8);
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          if (dvalid) {
+#pragma unroll
+            for (int c = 0; c < kFixRows; ++c)
+              region[c * DW + lane] =
+                  (unsigned long long)__float2ll_rn(__uint_as_float(v[pc * kFixRows + c]) * fscale);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (pc * kFixRows < r.nvalid)
+              bulk_reduce_add_u64(p.dq_fixed + fixed_index(r.q_row + pc * kFixRows, r.head, quarter * DW,
+                                                           p.dq_fixed_tpad, D),
+                                  region, kFixRows * DW * 8);
+            bulk_commit_group();
+          }
         }
       }
       ++j;

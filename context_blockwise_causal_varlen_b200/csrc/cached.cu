@@ -124,7 +124,7 @@ template <int D, int NB>
 __global__ void __launch_bounds__(kThreads) diag_grad_kernel(
     const __nv_bfloat16* __restrict__ q, const CacheBlocks cb, int64_t T, int H, int Hkv, float scale,
     const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse,
-    const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq) {
+    const float* __restrict__ dq_acc, const unsigned long long* __restrict__ dq_fixed, __nv_bfloat16* __restrict__ dq) {
   constexpr int L = D / 8;
   constexpr int kRows = kThreads / L;  // rows per CTA
   extern __shared__ float2 pds[];      // [kRows][G][NB - 1] of {p, dS}
@@ -145,7 +145,17 @@ __global__ void __launch_bounds__(kThreads) diag_grad_kernel(
     load8(q + qoff, qv);
     load8(dout + qoff, dov);
     load8(out + qoff, ov);
-    load8f(dq_acc + qoff, acc);
+    if (dq_fixed) {  // deterministic mode: 64-bit fixed point in units of 2^-32, quarter-major layout
+      const unsigned long long* f = dq_fixed + fixed_index(t, h, c, fixed_tpad(T), D);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const ulonglong2 u = __ldg(reinterpret_cast<const ulonglong2*>(f + e));
+        acc[e] = __ll2float_rn((long long)u.x) * 2.3283064365386963e-10f;
+        acc[e + 1] = __ll2float_rn((long long)u.y) * 2.3283064365386963e-10f;
+      }
+    } else {
+      load8f(dq_acc + qoff, acc);
+    }
     float delta = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) delta = fmaf(dov[e], ov[e], delta);
@@ -206,7 +216,8 @@ int merge_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, fl
 
 template <int D, int NB>
 int grad_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, float scale, const void* dout,
-            const void* out, const float* lse, const float* dq_acc, void* dq, cudaStream_t stream) {
+            const void* out, const float* lse, const float* dq_acc, const unsigned long long* dq_fixed, void* dq,
+            cudaStream_t stream) {
   constexpr int kRows = kThreads / (D / 8);
   const size_t smem = (size_t)kRows * (H / Hkv) * (NB - 1) * sizeof(float2);
   auto kern = diag_grad_kernel<D, NB>;
@@ -217,7 +228,7 @@ int grad_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, flo
   }
   const int64_t blocks = (T * Hkv + kRows - 1) / kRows;
   auto c = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
-  kern<<<blocks, kThreads, smem, stream>>>(c(q), cb, T, H, Hkv, scale, c(dout), c(out), lse, dq_acc,
+  kern<<<blocks, kThreads, smem, stream>>>(c(q), cb, T, H, Hkv, scale, c(dout), c(out), lse, dq_acc, dq_fixed,
                                            static_cast<__nv_bfloat16*>(dq));
   return (int)cudaGetLastError();
 }
@@ -239,15 +250,16 @@ int merge_d(int nb, const void* q, const CacheBlocks& cb, int64_t T, int H, int 
 
 template <int D>
 int grad_d(int nb, const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, float scale, const void* dout,
-           const void* out, const float* lse, const float* dq_acc, void* dq, cudaStream_t s) {
+           const void* out, const float* lse, const float* dq_acc, const unsigned long long* dq_fixed, void* dq,
+           cudaStream_t s) {
   switch (nb) {
-    case 2: return grad_nb<D, 2>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
-    case 3: return grad_nb<D, 3>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
-    case 4: return grad_nb<D, 4>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
-    case 5: return grad_nb<D, 5>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
-    case 6: return grad_nb<D, 6>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
-    case 7: return grad_nb<D, 7>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
-    case 8: return grad_nb<D, 8>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, s);
+    case 2: return grad_nb<D, 2>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
+    case 3: return grad_nb<D, 3>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
+    case 4: return grad_nb<D, 4>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
+    case 5: return grad_nb<D, 5>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
+    case 6: return grad_nb<D, 6>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
+    case 7: return grad_nb<D, 7>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
+    case 8: return grad_nb<D, 8>(q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, s);
     default: return (int)cudaErrorInvalidValue;
   }
 }
@@ -263,11 +275,11 @@ int launch_diag_merge(const void* q, const CacheBlocks& cb, int nb, int64_t T, i
 }
 
 int launch_diag_grad(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
-                     const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq,
-                     cudaStream_t stream) {
+                     const void* dout, const void* out, const float* lse, const float* dq_acc,
+                     const unsigned long long* dq_fixed, void* dq, cudaStream_t stream) {
   if (T * Hkv == 0) return 0;
-  if (D == 128) return grad_d<128>(nb, q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, stream);
-  if (D == 64) return grad_d<64>(nb, q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq, stream);
+  if (D == 128) return grad_d<128>(nb, q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, stream);
+  if (D == 64) return grad_d<64>(nb, q, cb, T, H, Hkv, scale, dout, out, lse, dq_acc, dq_fixed, dq, stream);
   return (int)cudaErrorInvalidValue;
 }
 

@@ -57,6 +57,11 @@ struct BwdParams {
   void* dv;
   int64_t dkv_stride_t, dkv_stride_h;
   int32_t dkv_accumulate;  // 0: write bf16; 1: add into fp32
+  // non-null: dq accumulates here as 64-bit fixed point in units of 2^-32, added by integer
+  // reduces, so the sum does not depend on the order the key tiles' partials arrive in
+  // (deterministic mode); null: fp32 reduce-adds through tm_dq.  Layout: see fixed_index().
+  unsigned long long* dq_fixed;
+  int64_t dq_fixed_tpad;
   int* status;
 };
 
@@ -65,12 +70,25 @@ int launch_fwd_pingpong(const FwdParams& p, int head_dim, bool paged, int grid, 
 int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream);
 
 // Per (token, head): Delta = rowsum(dout * out) and lse * log2(e), written [H, t_pad]
-// (t_pad = total rounded up to a multiple of 4); optionally zero dq_acc.
+// (t_pad = total rounded up to a multiple of 4); optionally zero the dq accumulator
+// (dq_zero, zero_bytes).
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
-                          int32_t heads, int32_t head_dim, float* rows, float* dq_acc,
+                          int32_t heads, int32_t head_dim, float* rows, void* dq_zero, size_t zero_bytes,
                           cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
+// The fixed-point dq accumulator of the deterministic backward is [H][4][t_pad][D/4]: each of the
+// four dQ readout warps owns a quarter of the head dims, and its slice of consecutive q rows is
+// contiguous, so one bulk reduce adds it.  t_pad = fixed_tpad(T) leaves room for a full 64-row
+// q tile starting at any row < T.
+__host__ __device__ inline int64_t fixed_tpad(int64_t T) { return (T + 64 + 7) / 8 * 8; }
+__host__ __device__ inline int64_t fixed_index(int64_t t, int h, int d, int64_t tpad, int D) {
+  const int dw = D / 4;
+  return ((int64_t)(h * 4 + d / dw) * tpad + t) * dw + d % dw;
+}
+// Fixed-point dq (units of 2^-32, the layout above) -> bf16 [T, H, D], or added into fp32 [T, H, D].
+int launch_fixed_to_bf16(const unsigned long long* src, void* dst, int64_t T, int H, int D, cudaStream_t stream);
+int launch_fixed_add_f32(const unsigned long long* src, float* dst, int64_t T, int H, int D, cudaStream_t stream);
 
 // EAGLE-3 cached attention diagonals (cached.cu).  Each cache block is [T, Hkv, D] bf16 at its
 // own address; lse is [H, T] fp32.  diag_merge: o32 holds block 0's normalised fp32 output;
@@ -85,9 +103,10 @@ struct CacheBlocks {
 };
 int launch_diag_merge(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
                       const float* o32, float* lse, void* out, cudaStream_t stream);
+// Block 0's dq comes as fp32 (dq_acc) or, in deterministic mode, as 64-bit fixed point (dq_fixed).
 int launch_diag_grad(const void* q, const CacheBlocks& cb, int nb, int64_t T, int H, int Hkv, int D, float scale,
-                     const void* dout, const void* out, const float* lse, const float* dq_acc, void* dq,
-                     cudaStream_t stream);
+                     const void* dout, const void* out, const float* lse, const float* dq_acc,
+                     const unsigned long long* dq_fixed, void* dq, cudaStream_t stream);
 // Standalone merge of (block_out, block_lse) into a running fp32 (out, lse).
 int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
                  float* weight_out, int64_t seqlen, int32_t heads, int32_t head_dim, cudaStream_t stream);

@@ -107,6 +107,40 @@ __global__ void __launch_bounds__(256) convert_kernel(const float4* __restrict__
   }
 }
 
+// 64-bit fixed point in units of 2^-32: the integer rounds to the nearest fp32, and the power-of-two
+// scale is exact.
+__device__ __forceinline__ float fixed_to_float(unsigned long long x) {
+  return __ll2float_rn((long long)x) * 2.3283064365386963e-10f;
+}
+
+// One thread per pair of adjacent head dims (never split across a quarter: D/4 is even).
+__global__ void __launch_bounds__(256) fixed_to_bf16_kernel(const unsigned long long* __restrict__ src,
+                                                            __nv_bfloat162* __restrict__ dst, int64_t T, int H,
+                                                            int D, int64_t tpad) {
+  const int64_t n2 = T * H * D / 2;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += (int64_t)gridDim.x * blockDim.x) {
+    const int d = (int)(2 * i % D);
+    const int64_t th = 2 * i / D;
+    const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(src + fixed_index(th / H, (int)(th % H), d, tpad, D));
+    dst[i] = __floats2bfloat162_rn(fixed_to_float(v.x), fixed_to_float(v.y));
+  }
+}
+
+__global__ void __launch_bounds__(256) fixed_add_f32_kernel(const unsigned long long* __restrict__ src,
+                                                            float2* __restrict__ dst, int64_t T, int H, int D,
+                                                            int64_t tpad) {
+  const int64_t n2 = T * H * D / 2;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += (int64_t)gridDim.x * blockDim.x) {
+    const int d = (int)(2 * i % D);
+    const int64_t th = 2 * i / D;
+    const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(src + fixed_index(th / H, (int)(th % H), d, tpad, D));
+    float2 o = dst[i];
+    o.x += fixed_to_float(v.x);
+    o.y += fixed_to_float(v.y);
+    dst[i] = o;
+  }
+}
+
 }  // namespace
 
 int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
@@ -131,12 +165,12 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
 }
 
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
-                          int32_t heads, int32_t head_dim, float* rows, float* dq_acc,
+                          int32_t heads, int32_t head_dim, float* rows, void* dq_zero, size_t zero_bytes,
                           cudaStream_t stream) {
   const int64_t n = total * heads;
   if (n == 0) return 0;
-  if (dq_acc) {
-    cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)n * head_dim * sizeof(float), stream);
+  if (dq_zero) {
+    cudaError_t e = cudaMemsetAsync(dq_zero, 0, zero_bytes, stream);
     if (e != cudaSuccess) return (int)e;
   }
   const int64_t blocks = (n + 7) / 8;
@@ -146,6 +180,23 @@ int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, i
   if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, r2, total, t_pad, heads);
   else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, r2, total, t_pad, heads);
   else return (int)cudaErrorInvalidValue;
+  return (int)cudaGetLastError();
+}
+
+int launch_fixed_to_bf16(const unsigned long long* src, void* dst, int64_t T, int H, int D, cudaStream_t stream) {
+  const int64_t n2 = T * H * D / 2;
+  if (n2 == 0) return 0;
+  const int64_t blocks = std::min<int64_t>((n2 + 255) / 256, 148 * 16);
+  fixed_to_bf16_kernel<<<blocks, 256, 0, stream>>>(src, reinterpret_cast<__nv_bfloat162*>(dst), T, H, D,
+                                                   fixed_tpad(T));
+  return (int)cudaGetLastError();
+}
+
+int launch_fixed_add_f32(const unsigned long long* src, float* dst, int64_t T, int H, int D, cudaStream_t stream) {
+  const int64_t n2 = T * H * D / 2;
+  if (n2 == 0) return 0;
+  const int64_t blocks = std::min<int64_t>((n2 + 255) / 256, 148 * 16);
+  fixed_add_f32_kernel<<<blocks, 256, 0, stream>>>(src, reinterpret_cast<float2*>(dst), T, H, D, fixed_tpad(T));
   return (int)cudaGetLastError();
 }
 

@@ -181,6 +181,12 @@ int cbv_attn_merge(float* out, float* lse, const void* block_out, int32_t block_
  * packed order; lse is [num_heads, total].
  * Backward: every block is fed the MERGED out and lse (the merged-lse identity), dk/dv of
  * a key tile accumulate across all blocks that see it, dq accumulates in fp32.
+ * Deterministic backward (the `deterministic` argument of zigzag_ring_flash_attn_varlen_backward
+ * and ring_attention._fa_backward): dk and dv are always written once per key tile, but dq sums partials from every key
+ * tile that sees a row, and fp32 reduce-adds land in whatever order the tiles finish.  With
+ * deterministic = 1 every partial is rounded to 64-bit fixed point in units of 2^-32 and added as
+ * an integer, so dq is bit-identical from run to run (the workspace holds 8 instead of 4 bytes per
+ * dq element, and each partial's rounding adds at most 2^-33 absolute error).
  * Errors: causal = 0 -> CBV_ERR_NOT_CAUSAL (zig-zag is meaningless otherwise); a document
  * length not divisible by 2cp (zig-zag) or cp (contiguous) -> CBV_ERR_NOT_DIVISIBLE_2CP. */
 typedef struct cbv_ring_args {
@@ -200,6 +206,7 @@ typedef struct cbv_ring_args {
   int32_t causal;            /* must be 1 */
   int32_t window;
   int32_t schedule;          /* cbv_schedule (forward only) */
+  int32_t deterministic;     /* backward only: 1 = bit-reproducible dq (see above), 0 = fastest */
   void* out;                 /* device bf16 [total, num_heads, head_dim]: forward output, backward input */
   float* lse;                /* device f32 [num_heads, total]: forward output, backward input (merged) */
   const void* dout;          /* backward: device bf16 [total, num_heads, head_dim] */
@@ -248,6 +255,7 @@ typedef struct cbv_cached_ring_args {
   int32_t layout;              /* cbv_layout */
   float scale;
   int32_t window;
+  int32_t deterministic;       /* backward only: as cbv_ring_args.deterministic */
   void* out;                   /* device bf16 [total, num_heads, head_dim]: forward output, backward input */
   float* lse;                  /* device f32 [num_heads, total]: forward output, backward input (merged) */
   const void* dout;            /* backward: device bf16 [total, num_heads, head_dim] */
@@ -287,6 +295,8 @@ typedef struct cbv_block_bwd_args {
   float scale;
   int32_t causal;
   int32_t window;
+  int32_t deterministic;  /* 1: the block's dq is summed in 64-bit fixed point, then added to dq_acc
+                             once: bit-reproducible (as cbv_ring_args.deterministic) */
   float* dq_acc;       /* device f32 [total_q, num_heads, head_dim], += */
   float* dk_acc;       /* device f32 [total_k, num_kv_heads, head_dim], += */
   float* dv_acc;
