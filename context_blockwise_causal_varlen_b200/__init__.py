@@ -113,7 +113,7 @@ class KvpArgs(ctypes.Structure):
         ("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
         ("block_tables", ctypes.c_void_p), ("shards", ctypes.c_int32), ("blocks_per_shard", ctypes.c_int32),
         ("kv_mode", ctypes.c_int32), ("seg_size", ctypes.c_int32), ("scale", ctypes.c_float),
-        ("global_q_offset", ctypes.c_int32), ("sliding_window", ctypes.c_int32),
+        ("global_q_offset", ctypes.c_int32), ("sliding_window", ctypes.c_int32), ("tp_out", ctypes.c_int32),
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("shard_out", ctypes.c_void_p),
         ("shard_lse", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
@@ -480,8 +480,9 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
 
 def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_ROBIN, seg_size: int = 512,
                           scale=None, global_q_offset: int = 0, sliding_window: int = 0, per_shard: bool = False,
-                          return_lse: bool = True):
-    """Paged KV-parallel prefill; q ``[HQ, S, D]`` -> ``out [HQ, S, D]`` (+ lse, + per-shard partials)."""
+                          return_lse: bool = True, tp_out: bool = False):
+    """Paged KV-parallel prefill; q ``[HQ, S, D]`` -> ``out [HQ, S, D]`` (``[HQ, D, S]`` with ``tp_out``)
+    (+ lse, + per-shard partials)."""
     if not q.is_cuda or q.dtype != torch.bfloat16:
         raise CbvError(-3, "q must be a CUDA bfloat16 tensor")
     k_cache, v_cache = _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache")
@@ -489,7 +490,7 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
     nb, HKV, bs, _ = k_cache.shape
     bt = block_tables.to(device=q.device, dtype=torch.int32).contiguous()
     R, bps = bt.shape
-    out = torch.empty((HQ, S, D), dtype=torch.bfloat16, device=q.device)
+    out = torch.empty((HQ, D, S) if tp_out else (HQ, S, D), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((HQ, S), dtype=torch.float32, device=q.device) if return_lse else None
     so = torch.empty((R, HQ, S, D), dtype=torch.float32, device=q.device) if per_shard else None
     sl = torch.empty((R, HQ, S), dtype=torch.float32, device=q.device) if per_shard else None
@@ -497,7 +498,8 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
                 num_heads=HQ, num_kv_heads=HKV, head_dim=D, k_cache=_ptr(k_cache), v_cache=_ptr(v_cache),
                 num_blocks=nb, block_size=bs, block_tables=_ptr(bt), shards=R, blocks_per_shard=bps,
                 kv_mode=int(kv_mode), seg_size=int(seg_size), scale=_scale(scale),
-                global_q_offset=int(global_q_offset), sliding_window=int(sliding_window), out=_ptr(out),
+                global_q_offset=int(global_q_offset), sliding_window=int(sliding_window), tp_out=int(bool(tp_out)),
+                out=_ptr(out),
                 lse=_ptr(lse), shard_out=_ptr(so), shard_lse=_ptr(sl))
     if q.stride(2) != 1:
         raise CbvError(-4, "q's last dimension must be contiguous")

@@ -545,8 +545,9 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   if (!a->shard_out) {
     p.out = a->out;
     p.out_mode = kOutBf16;
-    p.out_stride_t = D;
+    p.out_stride_t = a->tp_out ? 1 : D;
     p.out_stride_h = (int64_t)a->q_len * D;
+    p.out_stride_d = a->tp_out ? a->q_len : 1;
     p.lse = a->lse ? a->lse : lse_scratch;
     p.lse_stride_h = a->q_len;
     p.lse_stride_t = 1;
@@ -576,6 +577,7 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
     e = cudaMemcpyAsync(a->lse, lse_scratch, rows * sizeof(float), cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "copying lse");
   }
+  if (a->tp_out) return launch_rc(launch_convert_bf16_transposed(acc, a->out, H, a->q_len, D, s), "output conversion");
   return launch_rc(launch_convert_bf16(acc, a->out, (int64_t)rows * D, 1.f, s), "output conversion");
 }
 

@@ -406,7 +406,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        if (p.out_mode == kOutBf16) {
+        if (p.out_mode == kOutBf16 && p.out_stride_d > 1) {
+          // transposed output: lanes hold consecutive rows, so each store covers 32 adjacent rows
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + shard_off * p.out_shard_stride +
+                               orow * p.out_stride_t + (int64_t)head * p.out_stride_h + (int64_t)c * p.out_stride_d;
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            dst[(int64_t)e * p.out_stride_d] = __float2bfloat16_rn(__uint_as_float(o[e]) * inv_l);
+        } else if (p.out_mode == kOutBf16) {
           __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + shard_off * p.out_shard_stride + orow * p.out_stride_t +
                                (int64_t)head * p.out_stride_h + c;
 #pragma unroll

@@ -29,6 +29,7 @@ struct FwdParams {
   int32_t window;
   void* out;
   int64_t out_stride_t, out_stride_h;  // elements
+  int64_t out_stride_d;  // bf16 out only: 0 or 1 = head dims contiguous; > 1 = transposed ([H, D, S]) output
   float* lse;
   int64_t lse_stride_h, lse_stride_t;  // elements
   int32_t out_mode;
@@ -77,6 +78,8 @@ int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, i
                           cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
+// fp32 [H, S, D] -> bf16 [H, D, S] (the prefill's transposed output).
+int launch_convert_bf16_transposed(const float* src, void* dst, int H, int64_t S, int D, cudaStream_t stream);
 // The fixed-point dq accumulator of the deterministic backward is [H][4][t_pad][D/4]: each of the
 // four dQ readout warps owns a quarter of the head dims, and its slice of consecutive q rows is
 // contiguous, so one bulk reduce adds it.  t_pad = fixed_tpad(T) leaves room for a full 64-row

@@ -141,6 +141,27 @@ __global__ void __launch_bounds__(256) fixed_add_f32_kernel(const unsigned long 
   }
 }
 
+// [H, S, D] fp32 -> [H, D, S] bf16 through a 32 x 32 shared-memory tile: reads run along D,
+// writes along S, both coalesced.  Block (32, 8); grid (ceil(S/32), D/32, H).
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const float* __restrict__ src,
+                                                             __nv_bfloat16* __restrict__ dst, int64_t S, int D) {
+  __shared__ float tile[32][33];
+  const int64_t s0 = (int64_t)blockIdx.x * 32;
+  const int d0 = blockIdx.y * 32;
+  const int64_t h = blockIdx.z;
+  const float* in = src + h * S * D;
+  __nv_bfloat16* outp = dst + h * S * D;
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int64_t s = s0 + r;
+    if (s < S) tile[r][threadIdx.x] = in[s * D + d0 + threadIdx.x];
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int64_t s = s0 + threadIdx.x;
+    if (s < S) outp[(int64_t)(d0 + r) * S + s] = __float2bfloat16_rn(tile[threadIdx.x][r]);
+  }
+}
+
 }  // namespace
 
 int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
@@ -197,6 +218,13 @@ int launch_fixed_add_f32(const unsigned long long* src, float* dst, int64_t T, i
   if (n2 == 0) return 0;
   const int64_t blocks = std::min<int64_t>((n2 + 255) / 256, 148 * 16);
   fixed_add_f32_kernel<<<blocks, 256, 0, stream>>>(src, reinterpret_cast<float2*>(dst), T, H, D, fixed_tpad(T));
+  return (int)cudaGetLastError();
+}
+
+int launch_convert_bf16_transposed(const float* src, void* dst, int H, int64_t S, int D, cudaStream_t stream) {
+  if ((int64_t)H * S == 0) return 0;
+  const dim3 grid((unsigned)((S + 31) / 32), (unsigned)(D / 32), (unsigned)H);
+  transpose_bf16_kernel<<<grid, dim3(32, 8), 0, stream>>>(src, static_cast<__nv_bfloat16*>(dst), S, D);
   return (int)cudaGetLastError();
 }
 

@@ -334,7 +334,8 @@ typedef struct cbv_kvp_args {
   float scale;
   int32_t global_q_offset;
   int32_t sliding_window;     /* 0 = disabled */
-  void* out;                  /* device bf16 [num_heads, q_len, head_dim] (merged result) */
+  int32_t tp_out;             /* 0: out is [num_heads, q_len, head_dim]; 1: transposed, [num_heads, head_dim, q_len] */
+  void* out;                  /* device bf16 merged result, laid out as tp_out says */
   float* lse;                 /* device f32 [num_heads, q_len] or NULL */
   float* shard_out;           /* NULL, or device f32 [shards, num_heads, q_len, head_dim] per-shard partials */
   float* shard_lse;           /* with shard_out: device f32 [shards, num_heads, q_len] */

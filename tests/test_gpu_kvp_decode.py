@@ -101,3 +101,23 @@ def test_decode_rejects_more_than_one_query_per_sequence():
     with pytest.raises(cbv.CbvError) as e:
         cbv.varlen_decode(dev(q), dev(k), dev(v), torch.tensor([0, 1, 3, 4]), torch.tensor([0, 3, 6, 10]))
     assert e.value.status == "Q_LEN_NOT_ONE"
+
+
+@pytest.mark.parametrize("per_shard", [False, True])
+@pytest.mark.parametrize("D,S", [(128, 300), (64, 1), (64, 97)])
+def test_kvp_transposed_output_is_the_transpose(per_shard, D, S):
+    # tp_out: out is [HQ, D, S], element for element the transpose of the [HQ, S, D] output
+    R, bps, bs, hq, hkv = 4, 8, 32, 4, 2
+    q, kc, vc, perm = _paged(23, R, bps, bs, hq, hkv, D, S)
+    bt = torch.from_numpy(PG.shard_block_tables(perm, R, PG.ROUND_ROBIN))
+    gqo = R * bps * bs - S
+    kw = dict(seg_size=256, scale=0.1, global_q_offset=gqo, sliding_window=500, per_shard=per_shard)
+    a = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), bt, **kw)
+    b = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), bt, tp_out=True, **kw)
+    sync()
+    assert b[0].shape == (hq, D, S)
+    assert torch.equal(b[0], a[0].transpose(1, 2))
+    assert torch.equal(b[1], a[1])
+    K, V = PG.global_kv(f64(kc), f64(vc), bt.numpy(), bs, PG.ROUND_ROBIN)
+    ro, _ = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=500)
+    check_out(host(b[0]).transpose(0, 2, 1), ro)
