@@ -472,6 +472,32 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_workload(kind: str, seed: int, rank: int):
+    """The batch one rank runs.  Replicas: every rank draws its own packed batch (seed + rank) of the
+    same total size, so per-rank work is fixed as ranks are added (weak scaling); the long-document
+    workloads are one fixed document."""
+    from synth.workloads import long_doc, packed_zigzag
+
+    if kind == "packed":
+        return packed_zigzag(seed + rank)
+    if kind == "long_doc":
+        return long_doc()
+    return long_doc(total=16384, cp=8, heads=16)
+
+
+def reduce_over_ranks(dist, torch, device, ms: float, flops: float, world: int):
+    """Whole-job timing of replicas: (the slowest rank's step time, the flops of all ranks).
+    Every rank takes the same collective steps (two all-reduces) in the same order."""
+    if world <= 1:
+        return ms, flops
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    f = torch.tensor([flops], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
 # ----------------------------------------------------------------------------- main arm
 def main():
     args = parse_args()
@@ -482,7 +508,6 @@ def main():
     import torch.distributed as dist
 
     import context_blockwise_causal_varlen_b200 as cbv
-    from synth.workloads import long_doc, packed_zigzag
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -495,12 +520,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     pk, pk_kind = peaks()
 
-    if args.workload == "packed":
-        w = packed_zigzag(args.seed + rank)
-    elif args.workload == "long_doc":
-        w = long_doc()
-    else:
-        w = long_doc(total=16384, cp=8, heads=16)
+    w = rank_workload(args.workload, args.seed, rank)
     cu = w.cu_seqlens
     S, H, D, cp = w.total, w.heads, w.head_dim, w.cp
     q, k, v, do = make_ring_inputs(cu, H, D, args.seed + rank, device)
@@ -541,22 +561,17 @@ def main():
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / args.steps
+    # each replica's batch has its own documents, hence its own visible-pair count
+    ms, total_flops = reduce_over_ranks(dist, torch, device, ms, f_fwd + f_bwd, world)
     if world > 1:
-        tt = torch.tensor([ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
         dist.barrier()
     fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["f0"], ev["f1"])]))
     bwd_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["f1"], ev["b1"])]))
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e_ms, h2d, d2h = e2e_pipelined(cbv, torch, (q, k, v, do), cu, cp, max(6, args.steps // 2), 2)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms, _ = reduce_over_ranks(dist, torch, device, e2e_ms, 0.0, world)
 
-    total_flops = (f_fwd + f_bwd) * world
     value = total_flops / (ms * 1e-3) / 1e12
     if rank == 0:
         # the dominant kernel: the block backward (10 of the 14 flops per pair)
