@@ -735,7 +735,9 @@ static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows, dq_buf, dq_bytes, s),
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows,
+                                            det ? nullptr : static_cast<float*>(dq_buf), det ? dq_buf : nullptr,
+                                            det ? dq_bytes : 0, s),
                       "backward preprocess")))
     return rc;
   *dq_acc_out = det ? nullptr : static_cast<float*>(dq_buf);
@@ -825,7 +827,8 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
-  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, rows, dq_fixed, fix_bytes, s),
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, rows, nullptr, dq_fixed,
+                                            fix_bytes, s),
                       "backward preprocess")))
     return rc;
   if ((rc = launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "backward launch"))) return rc;

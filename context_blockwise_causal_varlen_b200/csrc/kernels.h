@@ -71,11 +71,11 @@ int launch_fwd_pingpong(const FwdParams& p, int head_dim, bool paged, int grid, 
 int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream);
 
 // Per (token, head): Delta = rowsum(dout * out) and lse * log2(e), written [H, t_pad]
-// (t_pad = total rounded up to a multiple of 4); optionally zero the dq accumulator
-// (dq_zero, zero_bytes).
+// (t_pad = total rounded up to a multiple of 4).  Optionally zeroes a dq accumulator: an fp32
+// [T, H, D] one in the same pass (dq_f32_zero), or any other (dq_other_zero, other_bytes) by memset.
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
-                          int32_t heads, int32_t head_dim, float* rows, void* dq_zero, size_t zero_bytes,
-                          cudaStream_t stream);
+                          int32_t heads, int32_t head_dim, float* rows, float* dq_f32_zero, void* dq_other_zero,
+                          size_t other_bytes, cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
 // fp32 [H, S, D] -> bf16 [H, D, S] (the prefill's transposed output).

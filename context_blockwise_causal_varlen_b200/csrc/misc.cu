@@ -75,28 +75,43 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ out, flo
 }
 
 // Backward preprocess: Delta_i = <dO_i, O_i> with the merged (bf16) output, and the
-// merged lse in log2 units, both laid out [H, t_pad] for the backward's row loads.
+// merged lse in log2 units, both laid out [H, t_pad] for the backward's row loads; with
+// dq_zero, the row's fp32 dq accumulator is zeroed in the same pass.  D/8 lanes per
+// (token, head) row with 16-byte accesses; rows are numbered head-major, so consecutive rows
+// read consecutive lse entries and write consecutive row pairs.
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ dout,
                                                     const __nv_bfloat16* __restrict__ out,
                                                     const float* __restrict__ lse, float2* __restrict__ rows,
-                                                    int64_t total, int64_t t_pad, int heads) {
-  constexpr int E = D / 32;
-  const int64_t rowid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (rowid >= total * heads) return;
-  const __nv_bfloat16* a = dout + rowid * D + lane * E;
-  const __nv_bfloat16* b = out + rowid * D + lane * E;
+                                                    float* __restrict__ dq_zero, int64_t total, int64_t t_pad,
+                                                    int heads) {
+  constexpr int L = D / 8;  // lanes per row
+  const int64_t rowid = ((int64_t)blockIdx.x * 256 + threadIdx.x) / L;
+  const int c = (threadIdx.x % L) * 8;
+  const bool valid = rowid < total * heads;
+  const int64_t h = valid ? rowid / total : 0;
+  const int64_t tok = valid ? rowid % total : 0;
+  const int64_t off = (tok * heads + h) * D + c;
+  const uint4 ua = __ldg(reinterpret_cast<const uint4*>(dout + off));
+  const uint4 ub = __ldg(reinterpret_cast<const uint4*>(out + off));
+  const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
   float s = 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) s += __bfloat162float(a[e]) * __bfloat162float(b[e]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
-    const int64_t tok = rowid / heads;
-    const int h = (int)(rowid % heads);
-    rows[(int64_t)h * t_pad + tok] = make_float2(lse[(int64_t)h * total + tok] * 1.4426950408889634f, s);
+  for (int j = 0; j < 4; ++j) {
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&wa[j]);
+    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&wb[j]);
+    s = fmaf(__low2float(x), __low2float(y), s);
+    s = fmaf(__high2float(x), __high2float(y), s);
   }
+#pragma unroll
+  for (int o = L / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (!valid) return;
+  if (dq_zero) {
+    float4* z = reinterpret_cast<float4*>(dq_zero + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (c == 0) rows[h * t_pad + tok] = make_float2(lse[h * total + tok] * 1.4426950408889634f, s);
 }
 
 __global__ void __launch_bounds__(256) convert_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
@@ -186,20 +201,20 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
 }
 
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
-                          int32_t heads, int32_t head_dim, float* rows, void* dq_zero, size_t zero_bytes,
-                          cudaStream_t stream) {
+                          int32_t heads, int32_t head_dim, float* rows, float* dq_f32_zero, void* dq_other_zero,
+                          size_t other_bytes, cudaStream_t stream) {
   const int64_t n = total * heads;
   if (n == 0) return 0;
-  if (dq_zero) {
-    cudaError_t e = cudaMemsetAsync(dq_zero, 0, zero_bytes, stream);
+  if (dq_other_zero) {
+    cudaError_t e = cudaMemsetAsync(dq_other_zero, 0, other_bytes, stream);
     if (e != cudaSuccess) return (int)e;
   }
-  const int64_t blocks = (n + 7) / 8;
+  const int64_t blocks = (n * (head_dim / 8) + 255) / 256;
   auto d = reinterpret_cast<const __nv_bfloat16*>(dout);
   auto o = reinterpret_cast<const __nv_bfloat16*>(out);
   float2* r2 = reinterpret_cast<float2*>(rows);
-  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, r2, total, t_pad, heads);
-  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, r2, total, t_pad, heads);
+  if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, r2, dq_f32_zero, total, t_pad, heads);
+  else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, r2, dq_f32_zero, total, t_pad, heads);
   else return (int)cudaErrorInvalidValue;
   return (int)cudaGetLastError();
 }
