@@ -554,10 +554,12 @@ def main():
     clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.begin()
+    n0 = cbv.launch_count()
     t0.record()
     for _ in range(args.steps):
         step(record=True)
     t1.record()
+    launches = cbv.launch_count() - n0
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / args.steps
@@ -593,7 +595,7 @@ def main():
             "phases_ms": {"fwd": fwd_ms, "bwd": bwd_ms},
             "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * 4,
+            "gpu_launches": launches,
             "clocks": clk,
             "balance": {"zigzag_pairs_per_rank": cbv.rank_pair_counts(cu, cp, "zigzag").tolist(),
                         "contiguous_pairs_per_rank": cbv.rank_pair_counts(cu, cp, "contiguous").tolist()},

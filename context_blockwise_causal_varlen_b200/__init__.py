@@ -148,7 +148,7 @@ class CachedRingArgs(ctypes.Structure):
 
 
 EXPORTS = [
-    "cbv_last_error_message", "cbv_abi_version", "cbv_read_status",
+    "cbv_last_error_message", "cbv_abi_version", "cbv_read_status", "cbv_launch_count",
     "cbv_local_cu_seqlens", "cbv_half_cu_seqlens", "cbv_get_half_index", "cbv_get_half_lse", "cbv_rank_tokens",
     "cbv_rank_pair_counts", "cbv_ring_step",
     "cbv_block_fwd_workspace_size", "cbv_attn_block_fwd", "cbv_attn_merge",
@@ -164,6 +164,7 @@ EXPORTS = [
 def _declare(L):
     L.cbv_last_error_message.restype = ctypes.c_char_p
     L.cbv_abi_version.restype = ctypes.c_int
+    L.cbv_launch_count.restype = ctypes.c_size_t
     L.cbv_read_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
     L.cbv_local_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i32p]
     L.cbv_half_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, c_i32p]
@@ -237,6 +238,11 @@ def _layout(layout) -> int:
     if isinstance(layout, str):
         return {"zigzag": ZIGZAG, "contiguous": CONTIGUOUS}[layout]
     return int(layout)
+
+
+def launch_count() -> int:
+    """Kernels the library has launched from this thread so far (diagnostic)."""
+    return int(lib().cbv_launch_count())
 
 
 def read_status(workspace: torch.Tensor) -> int:

@@ -125,33 +125,51 @@ int check_max_seqlen(const int32_t* cu, int32_t num_docs, int32_t max_seqlen) {
   return CBV_OK;
 }
 
-int upload(void* dst, const void* src, size_t bytes, cudaStream_t s) {
-  if (bytes == 0) return CBV_OK;
-  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
-  return e == cudaSuccess ? CBV_OK : cuda_fail(e, "uploading the schedule");
-}
-
 int zero_status(void* ws, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, s);
   return e == cudaSuccess ? CBV_OK : cuda_fail(e, "clearing the status word");
 }
 
+// A schedule in the workspace: the expanded task list (written on the device) and one image of
+// groups | tiles | segs (uploaded), each part 16-byte aligned.
 struct PlanDev {
   TileTask* tasks = nullptr;
   Seg* segs = nullptr;
+  PlanGroup* groups = nullptr;
+  TileTask* tiles = nullptr;
+  unsigned char* image = nullptr;
+  size_t off_tiles = 0, off_segs = 0, image_bytes = 0;
 };
+
+size_t up16(size_t x) { return (x + 15) / 16 * 16; }
 
 PlanDev carve_plan(Carve& c, const Plan& p) {
   PlanDev d;
   d.tasks = static_cast<TileTask*>(c.take(std::max<size_t>(1, p.tasks.size()) * sizeof(TileTask)));
-  d.segs = static_cast<Seg*>(c.take(std::max<size_t>(1, p.segs.size()) * sizeof(Seg)));
+  d.off_tiles = up16(p.groups.size() * sizeof(PlanGroup));
+  d.off_segs = d.off_tiles + up16(p.tiles.size() * sizeof(TileTask));
+  d.image_bytes = d.off_segs + up16(p.segs.size() * sizeof(Seg));
+  d.image = static_cast<unsigned char*>(c.take(std::max<size_t>(16, d.image_bytes)));
+  if (d.image) {
+    d.groups = reinterpret_cast<PlanGroup*>(d.image);
+    d.tiles = reinterpret_cast<TileTask*>(d.image + d.off_tiles);
+    d.segs = reinterpret_cast<Seg*>(d.image + d.off_segs);
+  }
   return d;
 }
 
+// Uploads the compact schedule inside kernel launch parameters (no copy engine, no host wait)
+// and expands the task list on the device.
 int upload_plan(const PlanDev& d, const Plan& p, cudaStream_t s) {
-  int rc = upload(d.tasks, p.tasks.data(), p.tasks.size() * sizeof(TileTask), s);
-  if (rc) return rc;
-  return upload(d.segs, p.segs.data(), p.segs.size() * sizeof(Seg), s);
+  if (p.tasks.empty()) return CBV_OK;
+  std::vector<unsigned char> img(d.image_bytes, 0);
+  memcpy(img.data(), p.groups.data(), p.groups.size() * sizeof(PlanGroup));
+  memcpy(img.data() + d.off_tiles, p.tiles.data(), p.tiles.size() * sizeof(TileTask));
+  memcpy(img.data() + d.off_segs, p.segs.data(), p.segs.size() * sizeof(Seg));
+  int e = launch_inline_copy(d.image, img.data(), img.size(), s);
+  if (e) return cuda_fail(e, "uploading the schedule");
+  e = launch_expand_tasks(d.groups, (int)p.groups.size(), d.tiles, d.tasks, (int)p.tasks.size(), s);
+  return e ? cuda_fail(e, "expanding the schedule") : CBV_OK;
 }
 
 int launch_rc(int e, const char* what) { return e == 0 ? CBV_OK : cuda_fail(e, what); }
@@ -238,6 +256,8 @@ extern "C" {
 
 const char* cbv_last_error_message(void) { return g_err.c_str(); }
 int cbv_abi_version(void) { return CBV_ABI_VERSION; }
+
+size_t cbv_launch_count(void) { return cbv::launch_count(); }
 
 int cbv_read_status(const void* workspace, int* status_out, void* stream) {
   if (!workspace || !status_out) return fail(CBV_ERR_BAD_ARG, "NULL argument");

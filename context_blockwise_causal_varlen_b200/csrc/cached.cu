@@ -211,7 +211,7 @@ int merge_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, fl
   const int64_t blocks = (lanes + kThreads - 1) / kThreads;
   diag_merge_kernel<D, NB><<<blocks, kThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q), cb, T, H, Hkv,
                                                              scale, o32, lse, static_cast<__nv_bfloat16*>(out));
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 template <int D, int NB>
@@ -230,7 +230,7 @@ int grad_nb(const void* q, const CacheBlocks& cb, int64_t T, int H, int Hkv, flo
   auto c = [](const void* p) { return static_cast<const __nv_bfloat16*>(p); };
   kern<<<blocks, kThreads, smem, stream>>>(c(q), cb, T, H, Hkv, scale, c(dout), c(out), lse, dq_acc, dq_fixed,
                                            static_cast<__nv_bfloat16*>(dq));
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 template <int D>

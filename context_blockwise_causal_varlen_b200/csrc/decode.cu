@@ -276,7 +276,7 @@ int launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return (int)e;
   dim3 grid(p.num_seqs, p.hkv / p.heads_per_cta);
   kern<<<grid, kDecThreads, smem, stream>>>(p);
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 }  // namespace

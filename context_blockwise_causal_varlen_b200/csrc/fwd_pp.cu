@@ -462,7 +462,7 @@ int launch_pp_t(const FwdParams& p, int grid, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
   kern<<<grid, kThreads, smem, stream>>>(p);
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 }  // namespace

@@ -9,6 +9,11 @@
 
 namespace cbv {
 
+// Every kernel launch of the library ends with `return launched();`: it counts the launch for
+// the calling thread (cbv_launch_count) and returns the launch's error code.
+int launched();
+size_t launch_count();
+
 // Output modes of the forward kernel's epilogue.
 enum OutMode : int32_t {
   kOutBf16 = 0,   // write normalised out (bf16) and lse
@@ -76,6 +81,15 @@ int launch_bwd(const BwdParams& p, int head_dim, int grid, cudaStream_t stream);
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
                           int32_t heads, int32_t head_dim, float* rows, float* dq_f32_zero, void* dq_other_zero,
                           size_t other_bytes, cudaStream_t stream);
+// Host -> device copy of a small host buffer without a copy engine: the bytes travel inside the
+// launch parameters of one kernel per 30 KB.  A cudaMemcpyAsync from pageable host memory
+// would block the calling thread until the stream had drained and queue behind any large
+// transfer on the copy engine; this neither blocks nor queues.  dst 16-byte aligned.
+int launch_inline_copy(void* dst, const void* src, size_t bytes, cudaStream_t stream);
+// The task list from its compact form (plan.h: PlanGroup): task i of group g is tile
+// first_tile + (i - first_task) % ntiles with head (i - first_task) / ntiles.
+int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* tiles, TileTask* tasks, int ntasks,
+                        cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
 // fp32 [H, S, D] -> bf16 [H, D, S] (the prefill's transposed output).

@@ -1,5 +1,7 @@
 // Memory-bound helper kernels: the standalone online-softmax merge, the backward
 // preprocess (Delta = rowsum(dO * O)) and the fp32 -> bf16 conversion.
+#include <cstring>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -177,6 +179,36 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(const float* __rest
   }
 }
 
+constexpr int kInlineBytes = 30 * 1024;
+struct InlineChunk {
+  uint4* dst;
+  uint32_t n16;  // 16-byte words
+  uint32_t pad;
+  uint4 data[kInlineBytes / 16];
+};
+
+__global__ void __launch_bounds__(256) inline_copy_kernel(const __grid_constant__ InlineChunk c) {
+  for (uint32_t i = threadIdx.x; i < c.n16; i += blockDim.x) c.dst[i] = c.data[i];
+}
+
+__global__ void __launch_bounds__(256) expand_tasks_kernel(const PlanGroup* __restrict__ groups, int ngroups,
+                                                           const TileTask* __restrict__ tiles,
+                                                           TileTask* __restrict__ tasks, int ntasks) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < ntasks; i += gridDim.x * blockDim.x) {
+    int lo = 0, hi = ngroups - 1;  // the last group whose first task is <= i
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) / 2;
+      if (groups[mid].first_task <= i) lo = mid;
+      else hi = mid - 1;
+    }
+    const PlanGroup g = groups[lo];
+    const int local = i - g.first_task;
+    TileTask t = tiles[g.first_tile + local % g.ntiles];
+    t.head = local / g.ntiles;
+    tasks[i] = t;
+  }
+}
+
 }  // namespace
 
 int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
@@ -197,7 +229,7 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
   } else {
     return (int)cudaErrorInvalidValue;
   }
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, int64_t total, int64_t t_pad,
@@ -216,7 +248,7 @@ int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, i
   if (head_dim == 128) delta_kernel<128><<<blocks, 256, 0, stream>>>(d, o, lse, r2, dq_f32_zero, total, t_pad, heads);
   else if (head_dim == 64) delta_kernel<64><<<blocks, 256, 0, stream>>>(d, o, lse, r2, dq_f32_zero, total, t_pad, heads);
   else return (int)cudaErrorInvalidValue;
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 int launch_fixed_to_bf16(const unsigned long long* src, void* dst, int64_t T, int H, int D, cudaStream_t stream) {
@@ -225,7 +257,7 @@ int launch_fixed_to_bf16(const unsigned long long* src, void* dst, int64_t T, in
   const int64_t blocks = std::min<int64_t>((n2 + 255) / 256, 148 * 16);
   fixed_to_bf16_kernel<<<blocks, 256, 0, stream>>>(src, reinterpret_cast<__nv_bfloat162*>(dst), T, H, D,
                                                    fixed_tpad(T));
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 int launch_fixed_add_f32(const unsigned long long* src, float* dst, int64_t T, int H, int D, cudaStream_t stream) {
@@ -233,14 +265,50 @@ int launch_fixed_add_f32(const unsigned long long* src, float* dst, int64_t T, i
   if (n2 == 0) return 0;
   const int64_t blocks = std::min<int64_t>((n2 + 255) / 256, 148 * 16);
   fixed_add_f32_kernel<<<blocks, 256, 0, stream>>>(src, reinterpret_cast<float2*>(dst), T, H, D, fixed_tpad(T));
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 int launch_convert_bf16_transposed(const float* src, void* dst, int H, int64_t S, int D, cudaStream_t stream) {
   if ((int64_t)H * S == 0) return 0;
   const dim3 grid((unsigned)((S + 31) / 32), (unsigned)(D / 32), (unsigned)H);
   transpose_bf16_kernel<<<grid, dim3(32, 8), 0, stream>>>(src, static_cast<__nv_bfloat16*>(dst), S, D);
+  return launched();
+}
+
+namespace {
+thread_local size_t g_launches = 0;
+}
+
+int launched() {
+  ++g_launches;
   return (int)cudaGetLastError();
+}
+
+size_t launch_count() { return g_launches; }
+
+int launch_inline_copy(void* dst, const void* src, size_t bytes, cudaStream_t stream) {
+  InlineChunk c;
+  const unsigned char* p = static_cast<const unsigned char*>(src);
+  for (size_t off = 0; off < bytes; off += kInlineBytes) {
+    const size_t n = std::min<size_t>(kInlineBytes, bytes - off);
+    c.dst = reinterpret_cast<uint4*>(static_cast<unsigned char*>(dst) + off);
+    c.n16 = (uint32_t)((n + 15) / 16);
+    c.pad = 0;
+    memset(c.data, 0, (size_t)c.n16 * 16);
+    memcpy(c.data, p + off, n);
+    inline_copy_kernel<<<1, 256, 0, stream>>>(c);
+    const int e = launched();
+    if (e) return e;
+  }
+  return 0;
+}
+
+int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* tiles, TileTask* tasks, int ntasks,
+                        cudaStream_t stream) {
+  if (ntasks == 0 || ngroups == 0) return 0;
+  const int blocks = std::min((ntasks + 255) / 256, 148 * 4);
+  expand_tasks_kernel<<<blocks, 256, 0, stream>>>(groups, ngroups, tiles, tasks, ntasks);
+  return launched();
 }
 
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream) {
@@ -249,7 +317,7 @@ int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaS
   const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 148 * 16);
   convert_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst), n4,
                                              mul);
-  return (int)cudaGetLastError();
+  return launched();
 }
 
 }  // namespace cbv

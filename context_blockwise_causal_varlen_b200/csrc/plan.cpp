@@ -63,11 +63,11 @@ void coalesce_tail(std::vector<Seg>& segs, size_t first) {
 // descending total work, inside a group head by head (heads of one GQA group are
 // adjacent), inside a head tiles by descending work.  Consecutive CTAs then reuse the
 // same k/v (forward) or q/dO and dq rows (backward) from L2, and the largest pieces
-// start first.
-void expand_heads(std::vector<TileTask>& tiles, int32_t heads) {
+// start first.  Fills plan.tasks and its compact form (plan.tiles, plan.groups).
+void expand_heads(Plan& plan, int32_t heads) {
   std::map<int32_t, std::vector<TileTask>> groups;
   std::map<int32_t, int64_t> total;
-  for (const TileTask& t : tiles) {
+  for (const TileTask& t : plan.tasks) {
     groups[t.head].push_back(t);
     total[t.head] += t.work;
   }
@@ -75,17 +75,24 @@ void expand_heads(std::vector<TileTask>& tiles, int32_t heads) {
   for (auto& kv : groups) order.push_back(kv.first);
   std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return total[a] > total[b]; });
   std::vector<TileTask> out;
-  out.reserve(tiles.size() * (size_t)heads);
+  out.reserve(plan.tasks.size() * (size_t)heads);
+  plan.tiles.clear();
+  plan.groups.clear();
   for (int32_t g : order) {
     auto& v = groups[g];
     std::stable_sort(v.begin(), v.end(), [](const TileTask& a, const TileTask& b) { return a.work > b.work; });
+    plan.groups.push_back({(int32_t)out.size(), (int32_t)plan.tiles.size(), (int32_t)v.size(), 0});
+    for (TileTask t : v) {
+      t.head = 0;
+      plan.tiles.push_back(t);
+    }
     for (int32_t h = 0; h < heads; ++h)
       for (TileTask t : v) {
         t.head = h;
         out.push_back(t);
       }
   }
-  tiles.swap(out);
+  plan.tasks.swap(out);
 }
 
 }  // namespace
@@ -266,7 +273,7 @@ Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       plan.tasks.push_back(t);
     }
   }
-  expand_heads(plan.tasks, heads);
+  expand_heads(plan, heads);
   return plan;
 }
 
@@ -315,7 +322,7 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       plan.tasks.push_back(t);
     }
   }
-  expand_heads(plan.tasks, kv_heads);
+  expand_heads(plan, kv_heads);
   return plan;
 }
 
@@ -343,7 +350,7 @@ Plan plan_block_fwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qba
       plan.tasks.push_back(t);
     }
   }
-  expand_heads(plan.tasks, heads);
+  expand_heads(plan, heads);
   return plan;
 }
 
@@ -371,7 +378,7 @@ Plan plan_block_bwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qba
       plan.tasks.push_back(t);
     }
   }
-  expand_heads(plan.tasks, kv_heads);
+  expand_heads(plan, kv_heads);
   return plan;
 }
 
@@ -414,7 +421,7 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
       plan.tasks.push_back(t);
     }
   }
-  expand_heads(plan.tasks, heads);
+  expand_heads(plan, heads);
   return plan;
 }
 

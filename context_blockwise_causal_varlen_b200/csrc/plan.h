@@ -67,9 +67,18 @@ std::vector<ChunkPair> ring_chunk_pairs(const int32_t* cu, int32_t num_docs, int
                                         int32_t window, int32_t only_step /* -1 = all */);
 
 // ---------------------------------------------------------------- tile schedules
+// Tasks come in groups (e.g. one per document): inside a group, head by head, the group's tiles
+// in order.  Task i of a group is tile first_tile + i % ntiles for head i / ntiles, so the
+// tiles and this table describe the task list compactly (the device expands it).
+struct PlanGroup {
+  int32_t first_task, first_tile, ntiles, pad;
+};
+
 struct Plan {
-  std::vector<TileTask> tasks;
+  std::vector<TileTask> tasks;  // expanded: one per tile and head, in launch order
   std::vector<Seg> segs;
+  std::vector<TileTask> tiles;  // compact form of `tasks`: the tiles of every group, in order
+  std::vector<PlanGroup> groups;
 };
 
 // Forward over the ring: one task per 128-row q tile (inside one chunk, i.e. one virtual

@@ -91,6 +91,11 @@ int cbv_abi_version(void);
    kernel gave up a wait, CBV_OK otherwise. */
 int cbv_read_status(const void* workspace, int* status_out, void* stream);
 
+/* Number of kernels the library has launched from the calling thread since it was loaded
+ * (every call's schedule upload, helpers and attention kernels included).  A diagnostic: the
+ * difference across a stretch of calls is exactly what those calls enqueued. */
+size_t cbv_launch_count(void);
+
 /* ========================================================================= planner (host only)
  * Integer, exact; all arrays are host memory.  cu_seqlens is GLOBAL, int32 [num_docs+1],
  * natural packed order.  NeMo AutoModel zigzag_ring_attention: module docstring

@@ -226,3 +226,12 @@ def test_cached_ring_workspace_holds_the_fp32_block_output():
     a, _ = _cached_args(cu=np.array([0, 0], np.int32))
     assert cbv.lib().cbv_cached_ring_fwd(ctypes.byref(a), None) == 0
     assert cbv.lib().cbv_cached_ring_bwd(ctypes.byref(a), None) == 0
+
+
+def test_argument_errors_launch_nothing():
+    n0 = cbv.launch_count()
+    a, _ = _ring_args(head_dim=96)
+    assert cbv.STATUS[cbv.lib().cbv_zigzag_ring_fwd(ctypes.byref(a), None)] == "UNSUPPORTED_HEAD_DIM"
+    a, _ = _ring_args(cu=np.array([0], np.int32))
+    assert cbv.lib().cbv_zigzag_ring_bwd(ctypes.byref(a), None) == 0
+    assert cbv.launch_count() == n0

@@ -108,3 +108,17 @@ def test_status_word_is_clear_after_a_run():
     cu, q, k, v, _ = _case(5, [256], 2, 2, 128)
     _, _, ws = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, 2, return_workspace=True)
     assert cbv.read_status(ws) == 0
+
+
+def test_each_call_launches_its_schedule_upload_and_kernels():
+    # forward: schedule image (one launch per 30 KB) + task expansion + the forward kernel;
+    # backward: the same two + Delta + the backward kernel + the dq conversion
+    cu, q, k, v, do = _case(3, [264, 520, 128], 2, 2, 128)
+    tq, tk, tv, tdo = dev(q), dev(k), dev(v), dev(do)
+    n0 = cbv.launch_count()
+    out, lse = cbv.zigzag_ring_fwd(tq, tk, tv, cu, 2)
+    n1 = cbv.launch_count()
+    cbv.zigzag_ring_bwd(tdo, tq, tk, tv, out, lse, cu, 2)
+    n2 = cbv.launch_count()
+    sync()
+    assert n1 - n0 == 3 and n2 - n1 == 5
