@@ -22,17 +22,25 @@ int64_t sum_capped(int64_t a, int64_t b, int64_t window) {
   return s;
 }
 
-// visible (q, k) pairs between q positions [qp, qp+nq) and k positions [kp, kp+nk)
+// sum over q in [q0, q1) of clamp(q - a, 0, n): a ramp that starts after q = a and saturates at n
+int64_t ramp_sum(int64_t q0, int64_t q1, int64_t a, int64_t n) {
+  int64_t s = 0;
+  const int64_t lo = std::max(q0, a + 1), hi = std::min(q1, a + n);
+  if (hi > lo) s += (hi - lo) * ((lo - a) + (hi - 1 - a)) / 2;
+  const int64_t lo2 = std::max(q0, a + n);
+  if (q1 > lo2) s += (q1 - lo2) * n;
+  return s;
+}
+
+// visible (q, k) pairs between q positions [qp, qp+nq) and k positions [kp, kp+nk): with the
+// causal or window test, the pairs with 0 <= q - k (and q - k < window), counted as the pairs with
+// q - k >= 0 minus those with q - k >= window; each count is a ramp sum over q
 int64_t visible_pairs(int64_t qp, int64_t nq, int64_t kp, int64_t nk, bool causal, int64_t window) {
-  int64_t total = 0;
-  for (int64_t i = 0; i < nq; ++i) {
-    int64_t q = qp + i;
-    int64_t lo = kp, hi = kp + nk - 1;
-    if (causal || window > 0) hi = std::min(hi, q);
-    if (window > 0) lo = std::max(lo, q - window + 1);
-    if (hi >= lo) total += hi - lo + 1;
-  }
-  return total;
+  if (nq <= 0 || nk <= 0) return 0;
+  if (!causal && window <= 0) return nq * nk;
+  const int64_t ahead = ramp_sum(qp, qp + nq, kp - 1, nk);
+  if (window <= 0) return ahead;
+  return ahead - ramp_sum(qp, qp + nq, kp - 1 + window, nk);
 }
 
 int32_t weight(int64_t pairs) { return (int32_t)std::min<int64_t>(pairs / 256 + 1, INT32_MAX); }
