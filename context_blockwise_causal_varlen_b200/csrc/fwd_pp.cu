@@ -14,6 +14,10 @@
 // The two q tiles A and B of a CTA belong to the same head and stream the same k/v
 // tiles, so the tensor core never waits for one softmax: while warpgroup A turns
 // S_A into P_A, the tensor core computes S_B or PV_B, and the other way round.
+// A task of a single q tile (a chunk's ragged last tile) splits its k tiles instead:
+// both halves hold the same q rows, A takes the even k tiles and B the odd ones, and
+// the epilogue merges the two partial softmax states with the log-sum-exp identity,
+// so the tensor core still alternates between two independent chains.
 // P never leaves TMEM: the softmax writes P (bf16, two per 32-bit column) over the
 // S columns it has just read, and PV takes its A operand from TMEM.
 //
@@ -107,7 +111,8 @@ struct PPSmem {
   static constexpr uint32_t kK = kQ + 2 * kTile; // 2 stages
   static constexpr uint32_t kV = kK + 2 * kTile; // 2 stages
   static constexpr uint32_t kBars = kV + 2 * kTile;
-  static constexpr uint32_t kEnd = kBars + 256;
+  static constexpr uint32_t kStats = kBars + 256;       // split tasks: half B's {m, l, rounded l} per row
+  static constexpr uint32_t kEnd = kStats + BM * 16;
   static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
   static_assert(kDynamic <= 232448, "shared memory budget");
 };
@@ -227,8 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       const int ntile = has_b ? 2 : 1;
       bool ok = mbar_wait_warp(&bar[pQFull], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
+      // S_x of k tile i (K stage i & 1); a split task's two halves both read q tile 0
       auto issue_s = [&](int x, int i) {
-        const uint64_t dq = sdesc_add(dQ0, x * L::kTile), dk = sdesc_add(dK0, (i & 1) * L::kTile);
+        const uint64_t dq = sdesc_add(dQ0, (has_b ? x : 0) * L::kTile), dk = sdesc_add(dK0, (i & 1) * L::kTile);
         const uint32_t ts = tmem + x * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -237,15 +243,43 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         }
         umma_commit(&bar[pSFull + x]);
       };
-      auto issue_pv = [&](int x, int i) {
+      // PV_x of k tile i (V stage i & 1); `first` starts O_x afresh
+      auto issue_pv = [&](int x, int i, bool first) {
         const uint64_t dv = sdesc_add(dV0, (i & 1) * L::kTile);
         const uint32_t tp = tmem + x * 128, to = tmem + 256 + x * D;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ts(to, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(to, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc_o, (!first || kk > 0) ? 1u : 0u);
         umma_commit(&bar[pPVDone + x]);
       };
-      if (ok && n > 0) {
+      if (!has_b) {
+        // split task: k tile i belongs to half x = i & 1 and always sits in stage i & 1
+        for (int i = 0; ok && i < min(n, 2); ++i) {
+          ok = mbar_wait_warp(&bar[pKFull + i], 0, p.status, kDevTimeoutMma);
+          tc_fence_after();
+          if (ok) {
+            issue_s(i, i);
+            umma_commit(&bar[pKEmpty + i]);
+          }
+        }
+        for (int i = 0; ok && i < n; ++i) {
+          const int x = i & 1;
+          const uint32_t ph = (i >> 1) & 1;  // half x's own tile count, and stage x's load count
+          if (!mbar_wait_warp(&bar[pVFull + x], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait_warp(&bar[pPFull + x], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(x, i, i < 2);
+          umma_commit(&bar[pVEmpty + x]);
+          if (i + 2 < n) {
+            if (!mbar_wait_warp(&bar[pKFull + x], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            // P_x lives in the columns S_x of tile i + 2 will overwrite
+            if (!mbar_wait_warp(&bar[pPVDone + x], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(x, i + 2);
+            umma_commit(&bar[pKEmpty + x]);
+          }
+        }
+      } else if (ok && n > 0) {
         ok = mbar_wait_warp(&bar[pKFull], 0, p.status, kDevTimeoutMma);
         tc_fence_after();
         if (ok) {
@@ -253,13 +287,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           umma_commit(&bar[pKEmpty]);
         }
       }
-      for (int i = 0; ok && i < n; ++i) {
+      for (int i = 0; ok && has_b && i < n; ++i) {
         const int st = i & 1;
         if (!mbar_wait_warp(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         for (int x = 0; x < ntile && ok; ++x) {
           if (!mbar_wait_warp(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(x, i);
+          issue_pv(x, i, i == 0);
           if (i + 1 < n) {
             const int st1 = (i + 1) & 1;
             if (!mbar_wait_warp(&bar[pKFull + st1], ((i + 1) >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
@@ -277,24 +311,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue (warps 2..9)
-    const int x = (warp - 2) >> 2;  // tile: 0 = A, 1 = B
+    const int x = (warp - 2) >> 2;  // tile: 0 = A, 1 = B (a split task: the two halves of one tile)
+    const bool split = !has_b;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + x * 128 + lane_base;
     const uint32_t tO = tmem + 256 + x * D + lane_base;
-    const int trow = x * BM + row;  // row within the pair
+    const int trow = (split ? 0 : x * BM) + row;  // row within the pair
     const int32_t qpos = t.pos0 + trow;
-    const int32_t xq0 = t.pos0 + x * BM, xq1 = min(t.pos0 + t.rows - 1, xq0 + BM - 1);
+    const int32_t xq0 = t.pos0 + (split ? 0 : x * BM), xq1 = min(t.pos0 + t.rows - 1, xq0 + BM - 1);
     const float sl2 = p.scale_log2;
     const int32_t W = p.window;
     float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
-    int i = 0;
-    if (x == 0 || has_b) {
+    int i = 0;  // k tiles this tile (half) has processed
+    {
       KIter it;
       KTile r;
+      int kidx = 0;
       while (next_ktile<PAGED>(p, t, qp0, qp1, it, r)) {
+        if (split && ((kidx++ & 1) != x)) continue;  // the other half's k tile
         if (!mbar_wait_warp(&bar[pSFull + x], i & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
         tc_fence_after();
         uint32_t s[BN];
@@ -373,6 +410,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       }
     }
     // ---------------------------------------------------------------- epilogue
+    // split task: half B hands its softmax state to half A, which merges the two
+    // (every softmax warp reaches the barrier once, whatever happened before)
+    float wa_o = 1.f, wb_o = 0.f;  // weights of O_A and O_B in the merged accumulator
+    if (split) {
+      float4* stats = reinterpret_cast<float4*>(sm + L::kStats);
+      if (x == 1) stats[row] = make_float4(m, l, lr, 0.f);
+      named_bar_sync(1, 256);
+      if (x == 0) {
+        const float4 b = stats[row];
+        const float mm = fmaxf(m, b.x);
+        wa_o = (m == -INFINITY) ? 0.f : ex2_approx(m - mm);
+        wb_o = (b.x == -INFINITY) ? 0.f : ex2_approx(b.x - mm);
+        l = l * wa_o + b.y * wb_o;
+        lr = lr * wa_o + b.z * wb_o;
+        m = mm;
+      }
+    }
     if (ok && (x == 0 || has_b) && mbar_wait_warp(&bar[pODone], 0, p.status, kDevTimeoutEpilogue)) {
       tc_fence_after();
       const bool has = (l > 0.f) && (m != -INFINITY);
@@ -401,6 +455,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         uint32_t o[32];
         tmem_ld32(tO + c, o);
         tmem_ld_wait();
+        if (split) {
+          uint32_t ob[32];
+          tmem_ld32(tO + D + c, ob);  // O_B, the same rows
+          tmem_ld_wait();
+          // a half without k tiles (weight 0) never wrote its accumulator: select, do not multiply
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            o[e] = __float_as_uint((wa_o != 0.f ? __uint_as_float(o[e]) * wa_o : 0.f) +
+                                   (wb_o != 0.f ? __uint_as_float(ob[e]) * wb_o : 0.f));
+        }
         if (!valid) continue;
         if (!has) {
 #pragma unroll
@@ -448,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       }
       if (valid) *lse_ptr = lse_new;
     }
+
   }
 
   tc_fence_before();
