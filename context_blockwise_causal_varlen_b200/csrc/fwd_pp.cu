@@ -51,10 +51,13 @@ struct KIter {
   Seg seg;
 };
 
-// global position of shard-local token t of a paged KV cache
+// global position of shard-local token t of a paged KV cache (block_size is a power of two:
+// the call accepts only divisors of 128)
 __device__ __forceinline__ int32_t kvp_position(const FwdParams& p, int32_t shard, int32_t t) {
-  if (p.kv_mode == kKvRoundRobin)
-    return ((t / p.block_size) * p.shards + shard) * p.block_size + t % p.block_size;
+  if (p.kv_mode == kKvRoundRobin) {
+    const int lbs = __ffs(p.block_size) - 1;
+    return ((((t >> lbs) * p.shards + shard)) << lbs) + (t & (p.block_size - 1));
+  }
   return shard * p.n_local + t;
 }
 
@@ -349,10 +352,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           for (int c = 0; c < BN; ++c)
             if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
         } else if (need_mask) {
-          // round-robin pages: position = page base + offset inside the page
+          // round-robin pages: position = page base + offset inside the page (shifts: the
+          // block size is a power of two)
+          const int lbs = __ffs(p.block_size) - 1;
+          const int32_t page_stride = p.shards << lbs, in_page = p.block_size - 1;
 #pragma unroll
           for (int c = 0; c < BN; ++c) {
-            const int32_t kpos = r.kpos0 + (c / p.block_size) * p.shards * p.block_size + (c % p.block_size);
+            const int32_t kpos = r.kpos0 + (c >> lbs) * page_stride + (c & in_page);
             bool vis = c < r.nvalid;
             if (cz) vis = vis && (kpos <= qpos);
             if (W > 0) vis = vis && (qpos - kpos < W);
