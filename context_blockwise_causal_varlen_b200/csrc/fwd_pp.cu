@@ -206,9 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
             for (int h = 0; h < QH; ++h) tma_load_3d(dst + h * 16384, map, full, h * 64, kvh, r.k_row);
           } else {
             // one box per page of block_size tokens, found through the shard's block table
-            const int bs = p.block_size;
-            for (int pg = 0; pg < BN / bs; ++pg) {
-              const int blk = min((r.k_row + pg * bs) / bs, p.blocks_per_shard - 1);
+            const int bs = p.block_size, lbs = __ffs(bs) - 1;
+            for (int pg = 0; pg < (BN >> lbs); ++pg) {
+              const int blk = min((r.k_row >> lbs) + pg, p.blocks_per_shard - 1);  // k_row: a multiple of 128
               const int page = __ldg(&p.block_tables[(int64_t)r.shard * p.blocks_per_shard + blk]);
               for (int h = 0; h < QH; ++h) tma_load_4d(dst + h * 16384 + pg * bs * 128, map, full, h * 64, 0, kvh, page);
             }
@@ -366,9 +366,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           }
         }
         // row maximum of the raw scores (the scale is positive, so it commutes)
-        float mraw = -INFINITY;
+        // eight independent chains (the max is exact in any order), so the reduction sits on the
+        // softmax's critical path for about 11 dependent steps instead of 64
+        float mq[8];
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) mraw = max3f(mraw, __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        for (int j = 0; j < 8; ++j) mq[j] = max3f(-INFINITY, __uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1]));
+#pragma unroll
+        for (int c = 16; c < BN; c += 16)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mq[j] = max3f(mq[j], __uint_as_float(s[c + 2 * j]), __uint_as_float(s[c + 2 * j + 1]));
+        const float mraw = max3f(max3f(mq[0], mq[1], mq[2]), max3f(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
         const float mx = mraw * sl2;  // log2 units
         float m_use = m, alpha = 1.f;
         bool rescale_o = false;
