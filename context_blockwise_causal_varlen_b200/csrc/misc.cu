@@ -22,13 +22,17 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ out, flo
                                                     const void* __restrict__ block_out,
                                                     const float* __restrict__ block_lse, float* __restrict__ weight,
                                                     int64_t seqlen, int heads) {
-  constexpr int E = D / 32;
-  const int64_t rowid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (rowid >= seqlen * heads) return;
-  const int64_t tok = rowid / heads;
-  const int h = (int)(rowid % heads);
-  const int64_t li = (int64_t)h * seqlen + tok;
+  // D/8 lanes per (token, head) row, 8 elements each; rows numbered head-major so that
+  // consecutive rows read and write consecutive lse entries
+  constexpr int L = D / 8;
+  const int64_t rowid = ((int64_t)blockIdx.x * 256 + threadIdx.x) / L;
+  const int c = (threadIdx.x % L) * 8;
+  // every lane of a row reads lse[li] before one of them overwrites it: no early exit, and a
+  // warp barrier between the reads and the write
+  const bool valid = rowid < seqlen * heads;
+  const int64_t r = valid ? rowid : 0;
+  const int64_t h = r / seqlen, tok = r % seqlen;
+  const int64_t li = r;  // == h * seqlen + tok
   const float a = lse[li];
   const float b = block_lse[li];
   const float m = fmaxf(a, b);
@@ -44,33 +48,32 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ out, flo
     wb = __expf(b - nl);
     w = wb;  // sigmoid(b - a) with the pre-merge lse
   }
-  float* o = out + rowid * D + lane * E;
-  float x[E];
-  if constexpr (E == 4) {
-    const float4 v = *reinterpret_cast<const float4*>(o);
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-  } else {
-    const float2 v = *reinterpret_cast<const float2*>(o);
-    x[0] = v.x; x[1] = v.y;
-  }
-  float y[E];
+  const int64_t off = (tok * heads + h) * D + c;
+  float4* o = reinterpret_cast<float4*>(out + off);
+  float4 x0 = o[0], x1 = o[1];
+  float y[8];
   if (BF16_IN) {
-    const __nv_bfloat16* bo = reinterpret_cast<const __nv_bfloat16*>(block_out) + rowid * D + lane * E;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(block_out) + off));
+    const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int e = 0; e < E; ++e) y[e] = __bfloat162float(bo[e]);
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&wds[j]);
+      y[2 * j] = __low2float(v);
+      y[2 * j + 1] = __high2float(v);
+    }
   } else {
-    const float* bo = reinterpret_cast<const float*>(block_out) + rowid * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) y[e] = bo[e];
+    const float4* bo = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(block_out) + off);
+    const float4 v0 = __ldg(bo), v1 = __ldg(bo + 1);
+    y[0] = v0.x, y[1] = v0.y, y[2] = v0.z, y[3] = v0.w, y[4] = v1.x, y[5] = v1.y, y[6] = v1.z, y[7] = v1.w;
   }
-#pragma unroll
-  for (int e = 0; e < E; ++e) x[e] = x[e] * wa + y[e] * wb;
-  if constexpr (E == 4) {
-    *reinterpret_cast<float4*>(o) = make_float4(x[0], x[1], x[2], x[3]);
-  } else {
-    *reinterpret_cast<float2*>(o) = make_float2(x[0], x[1]);
+  x0 = make_float4(x0.x * wa + y[0] * wb, x0.y * wa + y[1] * wb, x0.z * wa + y[2] * wb, x0.w * wa + y[3] * wb);
+  x1 = make_float4(x1.x * wa + y[4] * wb, x1.y * wa + y[5] * wb, x1.z * wa + y[6] * wb, x1.w * wa + y[7] * wb);
+  if (valid) {
+    o[0] = x0;
+    o[1] = x1;
   }
-  if (lane == 0) {
+  __syncwarp();
+  if (valid && c == 0) {
     lse[li] = nl;
     if (weight) weight[li] = w;
   }
@@ -215,7 +218,7 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
                  float* weight_out, int64_t seqlen, int32_t heads, int32_t head_dim, cudaStream_t stream) {
   const int64_t rows = seqlen * heads;
   if (rows == 0) return 0;
-  const int64_t blocks = (rows + 7) / 8;
+  const int64_t blocks = (rows * (head_dim / 8) + 255) / 256;
   if (head_dim == 128) {
     if (block_out_is_f32)
       merge_kernel<128, false><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
