@@ -673,6 +673,8 @@ int make_bwd_maps(BwdParams* p, const void* q, const void* dout, const void* k, 
   if ((rc = map_thd(&p->tm_do, dout, total_q, H, D, (int64_t)H * D, D, 64))) return rc;
   if ((rc = map_thd(&p->tm_k, k, total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
   if ((rc = map_thd(&p->tm_v, v, total_k, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  if ((rc = map_thd(&p->tm_k8, k, total_k, Hkv, D, (int64_t)Hkv * D, D, 8))) return rc;
+  if ((rc = map_thd(&p->tm_v8, v, total_k, Hkv, D, (int64_t)Hkv * D, D, 8))) return rc;
   uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)std::max<int64_t>(total_q, 1)};
   uint64_t st[2] = {(uint64_t)D, (uint64_t)H * D};
   uint32_t box[3] = {(uint32_t)D / 4, 1, 16};  // one warp's head-dim slice x 16 q rows

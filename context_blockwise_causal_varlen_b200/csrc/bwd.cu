@@ -52,7 +52,8 @@ struct QIter {
 // Enumerates the q tiles (over the GQA group's q heads and all segments) that see
 // at least one key of the tile.  Every role runs its own copy.
 __device__ __forceinline__ bool next_qtile(const BwdParams& p, const TileTask& t, int kvh, QIter& it, QTile& r) {
-  const int32_t kp0 = t.pos0, kp1 = t.pos0 + t.rows - 1;
+  // key positions span [kp0, kp1]: with a second range, its last key (it lies after the first)
+  const int32_t kp0 = t.pos0, kp1 = t.split1 ? max(t.pos0 + t.rows, t.pos1 + t.rows1) - 1 : t.pos0 + t.rows - 1;
   const int32_t W = p.window;
   while (true) {
     if (it.hs >= p.heads_per_kv) return false;  // exhausted (and stays so when called again)
@@ -65,7 +66,9 @@ __device__ __forceinline__ bool next_qtile(const BwdParams& p, const TileTask& t
       if (t.nseg == 0) return false;
       it.seg = p.segs[t.seg0 + it.si];
       it.si++;
-      const bool cz = (it.seg.flags & kSegCausal) || W > 0;
+      // a tile of two key ranges tests causality on every segment: a segment that lies wholly
+      // after one range's keys can still precede the other's (the test is a no-op elsewhere)
+      const bool cz = (it.seg.flags & kSegCausal) || W > 0 || t.split1;
       int32_t cmin = 0, cmax = it.seg.rows - 1;
       if (cz) cmin = max(cmin, kp0 - it.seg.pos0);
       if (W > 0) cmax = min(cmax, kp1 + W - 1 - it.seg.pos0);
@@ -82,7 +85,7 @@ __device__ __forceinline__ bool next_qtile(const BwdParams& p, const TileTask& t
     r.q_row = it.seg.row0 + c0;
     r.qpos0 = it.seg.pos0 + c0;
     r.head = kvh * p.heads_per_kv + it.hs;
-    r.causal = it.seg.flags & kSegCausal;
+    r.causal = (it.seg.flags & kSegCausal) || t.split1;
     const bool cz = r.causal || W > 0;
     const int32_t qa = r.qpos0, qb = r.qpos0 + r.nvalid - 1;
     const bool all_vis = (r.nvalid == BM) && (t.rows == BN) && (!cz || qa >= kp1) && (W <= 0 || qb - kp0 < W);
@@ -190,8 +193,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       tma_prefetch_desc(&p.tm_q);
       mbar_arrive_expect_tx(&bar[bKVFull], 2 * L::kKV);
       for (int h = 0; h < KH; ++h) {
-        tma_load_3d(sK + h * 16384, &p.tm_k, &bar[bKVFull], h * 64, kvh, t.row0);
-        tma_load_3d(sV + h * 16384, &p.tm_v, &bar[bKVFull], h * 64, kvh, t.row0);
+        if (!t.split1) {
+          tma_load_3d(sK + h * 16384, &p.tm_k, &bar[bKVFull], h * 64, kvh, t.row0);
+          tma_load_3d(sV + h * 16384, &p.tm_v, &bar[bKVFull], h * 64, kvh, t.row0);
+        } else {
+          // two key ranges: 8-row pieces (1 KB of the 128B-swizzled tile each, so the swizzle
+          // pattern stays aligned); every tile row is loaded, from one range or the other
+          for (int g = 0; g < BN / 8; ++g) {
+            const int32_t row = g * 8 < t.split1 ? t.row0 + g * 8 : t.row1 + (g * 8 - t.split1);
+            tma_load_3d(sK + h * 16384 + g * 1024, &p.tm_k8, &bar[bKVFull], h * 64, kvh, row);
+            tma_load_3d(sV + h * 16384 + g * 1024, &p.tm_v8, &bar[bKVFull], h * 64, kvh, row);
+          }
+        }
       }
     }
     if (lane == 0) {
@@ -301,8 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const int quarter = warp & 3;
     const int krow = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int32_t kpos = t.pos0 + krow;
-    const bool kvalid = krow < t.rows;
+    const bool second = t.split1 && krow >= t.split1;  // this key row belongs to the second range
+    const int32_t kpos = second ? t.pos1 + (krow - t.split1) : t.pos0 + krow;
+    const bool kvalid = second ? krow - t.split1 < t.rows1 : krow < t.rows;
+    const int32_t kglobal = second ? t.row1 + (krow - t.split1) : t.row0 + krow;
     const int32_t W = p.window;
     const float sl2 = p.scale_log2;
     const uint32_t pt_buf[2] = {smem_u32(sPt), smem_u32(sm + L::kPt1)};
@@ -405,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_base;
         const float mul = which == 0 ? 1.f : p.scale;
         void* dst_base = which == 0 ? p.dv : p.dk;
-        const int64_t off = (int64_t)(t.row0 + krow) * p.dkv_stride_t + (int64_t)kvh * p.dkv_stride_h;
+        const int64_t off = (int64_t)kglobal * p.dkv_stride_t + (int64_t)kvh * p.dkv_stride_h;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];

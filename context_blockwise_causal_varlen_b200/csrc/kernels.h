@@ -50,7 +50,9 @@ struct BwdParams {
   CUtensorMap tm_do;    // (D, H, T) bf16, box (64, 1, 64)
   CUtensorMap tm_k;     // (D, Hkv, T) bf16, box (64, 1, 128)
   CUtensorMap tm_v;
-  CUtensorMap tm_dq;    // (D, H, T) fp32, box (D, 1, 64), no swizzle (reduce-add target)
+  CUtensorMap tm_k8;    // the same, box (64, 1, 8): tiles of two key ranges load in 8-row pieces
+  CUtensorMap tm_v8;
+  CUtensorMap tm_dq;    // (D, H, T) fp32, box (D/4, 1, 16), no swizzle (reduce-add target)
   const TileTask* tasks;
   const Seg* segs;
   int32_t num_tasks;

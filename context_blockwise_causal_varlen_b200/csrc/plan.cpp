@@ -312,7 +312,15 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
     }
     coalesce_tail(plan.segs, seg0);
     const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    // Zig-zag without a window: a rank's two chunks of a document, f < cp and b = 2cp-1-f, end in
+    // equally ragged key tiles.  When the two tails fit in one tile they share it: the keys of
+    // chunk b are seen only by q rows of chunks >= b, all of them among chunk f's segments, so
+    // the tile walks chunk f's segments and masks by position.  Chunk b's tail gets no task.
+    const int32_t tail = c % tile_n;
+    const bool pair_tails = layout == kZigZag && window <= 0 && tail > 0 && tail <= tile_n / 2;
     for (int32_t t0 = 0; t0 < c; t0 += tile_n) {
+      const bool is_tail = t0 + tile_n > c;
+      if (pair_tails && is_tail && y >= cp) continue;  // rides in chunk f's tail tile
       TileTask t{};
       t.row0 = cu[d] + y * c + t0;
       t.rows = std::min(tile_n, c - t0);
@@ -321,10 +329,17 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
       t.nseg = nseg;
       t.aux = -1;
       t.head = d;
+      if (pair_tails && is_tail) {
+        t.row1 = cu[d] + (nchunk - 1 - y) * c + t0;
+        t.pos1 = t.row1;
+        t.rows1 = tail;
+        t.split1 = (tail + 7) / 8 * 8;
+      }
       int64_t w = 0;
       for (int32_t i = 0; i < nseg; ++i) {
         const Seg& s = plan.segs[seg0 + i];
         w += visible_pairs(s.pos0, s.rows, t.pos0, t.rows, s.flags & kSegCausal, window);
+        if (t.split1) w += visible_pairs(s.pos0, s.rows, t.pos1, t.rows1, s.flags & kSegCausal, window);
       }
       t.work = weight(w);
       plan.tasks.push_back(t);

@@ -27,6 +27,10 @@ struct TileTask {
   int32_t aux;   // paged prefill: shard of the single-shard variant (-1 = all shards)
   int32_t head;  // head (q head in the forward, kv head in the backward); one task per tile and head
   int32_t work;  // estimated visible pairs / 256 (scheduling weight)
+  // backward only: a second key range in the same tile (split1 > 0).  Tile rows [0, split1)
+  // hold rows row0.. (valid: the first `rows`), tile rows [split1, 128) hold rows row1..
+  // (valid: the first rows1, positions pos1..).  split1 is a multiple of 8.
+  int32_t row1, pos1, rows1, split1;
 };
 
 // A streamed range: rows [row0, row0 + rows) attended by (or attending) the tile.
