@@ -31,7 +31,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "causal varlen attn TFLOP/s fwd+bwd (zig-zag ring, packed varlen)"
+METRIC = "causal varlen attn TFLOP/s fwd & fwd+bwd; decode HBM GB/s; % of B200 roofline"
+MEASURES = "fwd+bwd TFLOP/s of the zig-zag ring (fused schedule), visible pairs only; fwd, decode GB/s and the other workloads under extra"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -465,7 +466,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "cp": w.cp, "heads": w.heads, "head_dim": w.head_dim,
+            "config": {"workload": w.name, "measures": MEASURES, "cp": w.cp, "heads": w.heads, "head_dim": w.head_dim,
                        "l2": "inputs larger than L2 not applicable (CPU)"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": int(threads), "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -583,7 +584,8 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "tokens": S, "docs": len(cu) - 1, "cp": cp, "heads": H, "head_dim": D,
+            "config": {"workload": w.name, "measures": MEASURES, "tokens": S, "docs": len(cu) - 1, "cp": cp,
+                       "heads": H, "head_dim": D,
                        "layout": "zigzag", "schedule": "fused", "visible_pairs_per_head": pairs,
                        "l2": f"inputs larger than L2 (q, k, v, dout {4 * S * H * D * 2 / 1e6:.0f} MB)",
                        "parallelism": f"replicas x{world}"},
