@@ -17,7 +17,8 @@
  *   - Tensors are plain pointers.  "device" pointers are CUDA global memory of the
  *     current device; "host" pointers are ordinary CPU memory read during the call
  *     and not retained.  The caller owns all memory; the library allocates nothing
- *     and keeps no state between calls.  Scratch memory comes from a caller-owned
+ *     and keeps no state between calls (apart from the per-thread count of its kernel
+ *     launches, cbv_launch_count).  Scratch memory comes from a caller-owned
  *     device `workspace` whose size the matching *_workspace_size() call reports
  *     (cbv_zigzag_ring_fwd_noalloc, at the end, is the one call with built-in scratch).
  *   - bf16 means IEEE bfloat16 (torch.bfloat16); token-major layouts are
@@ -34,6 +35,10 @@
  *     stream) unless stated otherwise, and returns CBV_OK (0) or a negative
  *     cbv_status; cbv_last_error_message() then describes the failure.  Argument
  *     errors are detected on the host before anything is launched.
+ *   - No call copies host memory to the device with a copy engine.  The tile schedules
+ *     built on the host travel inside kernel launch parameters, so a call neither waits
+ *     for its stream nor queues behind the caller's own transfers.  A fixed-shape sequence
+ *     of calls can be captured in a CUDA graph and replayed on new tensor contents.
  *   - Kernels never wait without a bound: a stalled pipeline records a code in the
  *     workspace status word and exits; cbv_read_status() returns CBV_ERR_TIMEOUT.
  *   - Argument structs start with struct_size and abi_version so that fields are
