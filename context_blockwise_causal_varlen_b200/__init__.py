@@ -222,6 +222,16 @@ def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
     return t.contiguous()
 
 
+def _given(t, like_shape, dtype, device, name):
+    """A caller-provided output: the kernels write exactly this shape, contiguous, so check it."""
+    if t is None:
+        return None
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.device == device and t.dtype == dtype
+            and tuple(t.shape) == tuple(like_shape) and t.is_contiguous()):
+        raise CbvError(-2, f"{name} must be a contiguous {dtype} CUDA tensor of shape {tuple(like_shape)} on {device}")
+    return t
+
+
 def _workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
@@ -312,6 +322,8 @@ def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, l
     q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
     S, H, D = q.shape
     cu = _host_i32(cu_seqlens)
+    out = _given(out, q.shape, q.dtype, q.device, "out")
+    lse = _given(lse, (H, S), torch.float32, q.device, "lse")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
     a = RingArgs(**_header(RingArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), total=S, num_heads=H, num_kv_heads=k.shape[1],
@@ -331,6 +343,9 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
     dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
     S, H, D = q.shape
     cu = _host_i32(cu_seqlens)
+    dq = _given(dq, q.shape, q.dtype, q.device, "dq")
+    dk = _given(dk, k.shape, k.dtype, q.device, "dk")
+    dv = _given(dv, v.shape, v.dtype, q.device, "dv")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -381,6 +396,8 @@ def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window
     ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
     S, H, _ = q.shape
     cu = _host_i32(cu_seqlens)
+    out = _given(out, q.shape, q.dtype, q.device, "out")
+    lse = _given(lse, (H, S), torch.float32, q.device, "lse")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse is None else lse
     a, keep = _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse)
@@ -398,6 +415,7 @@ def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, sc
     dout, q, out = _bf16(dout, "dout"), _bf16(q, "q"), _bf16(out, "out")
     ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
     cu = _host_i32(cu_seqlens)
+    dq = _given(dq, q.shape, q.dtype, q.device, "dq")
     dq = torch.empty_like(q) if dq is None else dq
     stacked = isinstance(cache_k, torch.Tensor)
     if dcache_k is None:
@@ -469,6 +487,9 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
     qb = None if q_pos_base is None else _host_i32(q_pos_base)
     kb = None if k_pos_base is None else _host_i32(k_pos_base)
     f32 = dict(dtype=torch.float32, device=q.device)
+    dq_acc = _given(dq_acc, (Sq, H, D), torch.float32, q.device, "dq_acc")
+    dk_acc = _given(dk_acc, (Sk, Hkv, D), torch.float32, q.device, "dk_acc")
+    dv_acc = _given(dv_acc, (Sk, Hkv, D), torch.float32, q.device, "dv_acc")
     dq_acc = torch.zeros((Sq, H, D), **f32) if dq_acc is None else dq_acc
     dk_acc = torch.zeros((Sk, Hkv, D), **f32) if dk_acc is None else dk_acc
     dv_acc = torch.zeros((Sk, Hkv, D), **f32) if dv_acc is None else dv_acc
@@ -527,6 +548,7 @@ def varlen_decode(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, validate=None
         validate = not torch.cuda.is_current_stream_capturing()
     cq = cu_seqlens_q.to(device=q.device, dtype=torch.int32).contiguous()
     ck = cu_seqlens_k.to(device=q.device, dtype=torch.int32).contiguous()
+    out = _given(out, q.shape, q.dtype, q.device, "out")
     out = torch.empty_like(q) if out is None else out
     a = DecodeArgs(**_header(DecodeArgs), q=_ptr(q), k=_ptr(k), v=_ptr(v), out=_ptr(out), cu_seqlens_q=_ptr(cq),
                    cu_seqlens_k=_ptr(ck), num_seqs=ck.numel() - 1, total_q=q.shape[0], total_k=k.shape[0],

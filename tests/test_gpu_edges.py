@@ -172,3 +172,22 @@ def test_ring_step_replays_from_a_cuda_graph():
         check_rel(host(dq), rq, what="dq")
         check_rel(host(dk), rk, what="dk")
         check_rel(host(dv), rv, what="dv")
+
+
+def test_wrong_output_tensors_are_refused_before_any_launch():
+    cu = cu_from_lengths([64, 64])
+    q, k, v, do = (dev(x) for x in gen(64, *[(128, 2, 64)] * 4))
+    n0 = cbv.launch_count()
+    for kw in ({"out": torch.empty((128, 2, 32), dtype=torch.bfloat16, device="cuda")},
+               {"lse": torch.empty((128, 2), dtype=torch.float32, device="cuda")},
+               {"out": torch.empty((128, 2, 64), dtype=torch.float32, device="cuda")}):
+        with pytest.raises(cbv.CbvError):
+            cbv.zigzag_ring_fwd(q, k, v, cu, 2, **kw)
+    out, lse = cbv.zigzag_ring_fwd(q, k, v, cu, 2)
+    n1 = cbv.launch_count()
+    with pytest.raises(cbv.CbvError):
+        cbv.zigzag_ring_bwd(do, q, k, v, out, lse, cu, 2, dk=torch.empty((128, 1, 64), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(cbv.CbvError):
+        # the right shape, but not contiguous
+        cbv.attn_block_bwd(do, q, k, v, out, lse, cu, cu, dq_acc=torch.zeros((2, 128, 64), device="cuda").transpose(0, 1))
+    assert n1 - n0 == 3 and cbv.launch_count() == n1  # only the good forward launched anything
