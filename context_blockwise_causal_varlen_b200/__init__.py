@@ -222,6 +222,14 @@ def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
     return t.contiguous()
 
 
+def _shape(t, shape, name, dtype=None):
+    """An input the kernels read as exactly this shape (and dtype): check it before any launch."""
+    if tuple(t.shape) != tuple(shape) or (dtype is not None and t.dtype != dtype):
+        want = f"{tuple(shape)}" + (f" {dtype}" if dtype is not None else "")
+        raise CbvError(-2, f"{name} has shape {tuple(t.shape)} {t.dtype}, expected {want}")
+    return t
+
+
 def _given(t, like_shape, dtype, device, name):
     """A caller-provided output: the kernels write exactly this shape, contiguous, so check it."""
     if t is None:
@@ -321,6 +329,8 @@ def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, l
     """Ring forward over ``cp`` virtual ranks: ``(out [S,H,D] bf16, lse [H,S] f32)``."""
     q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
     S, H, D = q.shape
+    _shape(k, (S, k.shape[1], D), "k")
+    _shape(v, k.shape, "v")
     cu = _host_i32(cu_seqlens)
     out = _given(out, q.shape, q.dtype, q.device, "out")
     lse = _given(lse, (H, S), torch.float32, q.device, "lse")
@@ -342,6 +352,11 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
     64-bit fixed point, bit-identical from run to run."""
     dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
     S, H, D = q.shape
+    _shape(k, (S, k.shape[1], D), "k")
+    _shape(v, k.shape, "v")
+    _shape(dout, q.shape, "dout")
+    _shape(out, q.shape, "out")
+    _shape(lse, (H, S), "lse", torch.float32)
     cu = _host_i32(cu_seqlens)
     dq = _given(dq, q.shape, q.dtype, q.device, "dq")
     dk = _given(dk, k.shape, k.dtype, q.device, "dk")
@@ -395,6 +410,11 @@ def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window
     q = _bf16(q, "q")
     ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
     S, H, _ = q.shape
+    for i, (bk, bv) in enumerate(zip(ck, cv)):
+        _shape(bk, (S, ck[0].shape[1], q.shape[2]), f"cache_k[{i}]")
+        _shape(bv, bk.shape, f"cache_v[{i}]")
+    if len(ck) != len(cv):
+        raise CbvError(-2, "cache_k and cache_v have different block counts")
     cu = _host_i32(cu_seqlens)
     out = _given(out, q.shape, q.dtype, q.device, "out")
     lse = _given(lse, (H, S), torch.float32, q.device, "lse")
@@ -415,6 +435,15 @@ def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, sc
     dout, q, out = _bf16(dout, "dout"), _bf16(q, "q"), _bf16(out, "out")
     ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
     cu = _host_i32(cu_seqlens)
+    S, H, D = q.shape
+    for i, (bk, bv) in enumerate(zip(ck, cv)):
+        _shape(bk, (S, ck[0].shape[1], D), f"cache_k[{i}]")
+        _shape(bv, bk.shape, f"cache_v[{i}]")
+    if len(ck) != len(cv):
+        raise CbvError(-2, "cache_k and cache_v have different block counts")
+    _shape(dout, q.shape, "dout")
+    _shape(out, q.shape, "out")
+    _shape(lse, (H, S), "lse", torch.float32)
     dq = _given(dq, q.shape, q.dtype, q.device, "dq")
     dq = torch.empty_like(q) if dq is None else dq
     stacked = isinstance(cache_k, torch.Tensor)
@@ -444,6 +473,8 @@ def attn_block_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int = 0, sca
     """One varlen block: ``(out, lse)``; with ``merge=True`` merges into the running f32 ``(out, lse)`` in place."""
     q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
     Sq, H, D = q.shape
+    _shape(k, (k.shape[0], k.shape[1], D), "k")
+    _shape(v, k.shape, "v")
     cq, ck = _host_i32(cu_seqlens_q), _host_i32(cu_seqlens_k)
     qb = None if q_pos_base is None else _host_i32(q_pos_base)
     kb = None if k_pos_base is None else _host_i32(k_pos_base)
@@ -451,6 +482,8 @@ def attn_block_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int = 0, sca
         out_dtype = torch.float32
         if out is None or lse is None:
             raise CbvError(-1, "merge=True needs the running out (f32) and lse")
+    out = _given(out, (Sq, H, D), out_dtype, q.device, "out")
+    lse = _given(lse, (H, Sq), torch.float32, q.device, "lse")
     if out is None:
         out = torch.empty((Sq, H, D), dtype=out_dtype, device=q.device)
     if lse is None:
@@ -469,6 +502,10 @@ def attn_block_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int = 0, sca
 def attn_merge(out, lse, block_out, block_lse, return_weight: bool = False):
     """In-place online-softmax merge of ``(block_out, block_lse)`` into the f32 running ``(out, lse)``."""
     S, H, D = out.shape
+    _given(out, (S, H, D), torch.float32, out.device, "out")
+    _given(lse, (H, S), torch.float32, out.device, "lse")
+    _shape(block_out, (S, H, D), "block_out")
+    _shape(block_lse, (H, S), "block_lse", torch.float32)
     w = torch.empty((H, S), dtype=torch.float32, device=out.device) if return_weight else None
     dt = DTYPE_F32 if block_out.dtype == torch.float32 else DTYPE_BF16
     _check(lib().cbv_attn_merge(_ptr(out), _ptr(lse), _ptr(block_out.contiguous()), dt, _ptr(block_lse.contiguous()),
@@ -483,6 +520,11 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
     dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
     Sq, H, D = q.shape
     Sk, Hkv, _ = k.shape
+    _shape(v, k.shape, "v")
+    _shape(k, (Sk, Hkv, D), "k")
+    _shape(dout, q.shape, "dout")
+    _shape(out, q.shape, "out")
+    _shape(lse, (H, Sq), "lse", torch.float32)
     cq, ck = _host_i32(cu_seqlens_q), _host_i32(cu_seqlens_k)
     qb = None if q_pos_base is None else _host_i32(q_pos_base)
     kb = None if k_pos_base is None else _host_i32(k_pos_base)
@@ -515,6 +557,8 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
     k_cache, v_cache = _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache")
     HQ, S, D = q.shape
     nb, HKV, bs, _ = k_cache.shape
+    _shape(k_cache, (nb, HKV, bs, D), "k_cache")
+    _shape(v_cache, k_cache.shape, "v_cache")
     bt = block_tables.to(device=q.device, dtype=torch.int32).contiguous()
     R, bps = bt.shape
     out = torch.empty((HQ, D, S) if tp_out else (HQ, S, D), dtype=torch.bfloat16, device=q.device)
@@ -544,6 +588,8 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
 def varlen_decode(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, validate=None, out=None, workspace=None):
     """One query per sequence, GQA, offsets read on the device: ``out [total_q, HQ, D]`` bf16."""
     q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    _shape(k, (k.shape[0], k.shape[1], q.shape[2]), "k")
+    _shape(v, k.shape, "v")
     if validate is None:
         validate = not torch.cuda.is_current_stream_capturing()
     cq = cu_seqlens_q.to(device=q.device, dtype=torch.int32).contiguous()
