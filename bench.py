@@ -47,6 +47,9 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--workload", choices=["packed", "long_doc", "long_doc_small"], default="packed",
                    help="ring workload of the timed step (the headline is `packed`; the others are for profiling)")
+    p.add_argument("--only", choices=["long_doc", "deterministic", "cached", "paged", "decode", "merge"], default=None,
+                   help="run one of the sub-benchmarks alone and print its result (for profiling); no headline line")
+    p.add_argument("--decode-seqs", type=int, default=8192, help="sequences of the decode sub-benchmark")
     return p.parse_args()
 
 
@@ -271,8 +274,9 @@ def e2e_pipelined(cbv, torch, inputs, cu, cp, steps, warmup):
     return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
-def extra_benchmarks(device, pk, pk_kind):
-    """The other workloads, one line each (not the headline)."""
+def extra_benchmarks(device, pk, pk_kind, only=None, decode_seqs=8192):
+    """The other workloads, one line each (not the headline); `only` selects one of them."""
+    run = lambda name: only is None or only == name
     import torch
 
     import context_blockwise_causal_varlen_b200 as cbv
@@ -281,123 +285,129 @@ def extra_benchmarks(device, pk, pk_kind):
 
     res = {}
     tf_peak = pk["bf16_tflops"]
-    # long single document, zig-zag and contiguous, full causal and sliding window
-    for layout, window in (("zigzag", 0), ("contiguous", 0), ("zigzag", 4096)):
-        w = long_doc(window=window)
-        q, k, v, do = make_ring_inputs(w.cu_seqlens, w.heads, w.head_dim, 7, device)
-        pairs = visible_pairs(w.cu_seqlens, window)
+    if run("long_doc"):
+        # long single document, zig-zag and contiguous, full causal and sliding window
+        for layout, window in (("zigzag", 0), ("contiguous", 0), ("zigzag", 4096)):
+            w = long_doc(window=window)
+            q, k, v, do = make_ring_inputs(w.cu_seqlens, w.heads, w.head_dim, 7, device)
+            pairs = visible_pairs(w.cu_seqlens, window)
+            st = {}
+
+            def fwd():
+                st["o"], st["l"] = cbv.zigzag_ring_fwd(q, k, v, w.cu_seqlens, w.cp, window=window, layout=layout)
+
+            def bwd():
+                cbv.zigzag_ring_bwd(do, q, k, v, st["o"], st["l"], w.cu_seqlens, w.cp, window=window, layout=layout)
+
+            fwd()
+            t_f = timed(fwd, 5, 2)
+            t_b = timed(bwd, 5, 2)
+            f_fwd = 4 * w.head_dim * w.heads * pairs
+            f_bwd = 10 * w.head_dim * w.heads * pairs
+            key = f"long_doc_S65536_cp8_H16_{layout}" + (f"_W{window}" if window else "")
+            res[key] = {"fwd_tflops": f_fwd / t_f / 1e9, "bwd_tflops": f_bwd / t_b / 1e9,
+                        "fwd_bwd_tflops": (f_fwd + f_bwd) / (t_f + t_b) / 1e9,
+                        "fwd_bwd_frac": (f_fwd + f_bwd) / (t_f + t_b) / 1e9 / tf_peak, "ms": t_f + t_b}
+            del q, k, v, do, st
+            torch.cuda.empty_cache()
+    if run("deterministic"):
+        # deterministic backward (dq summed in 64-bit fixed point) against the default, packed workload
+        w = packed_zigzag()
+        q, k, v, do = make_ring_inputs(w.cu_seqlens, w.heads, w.head_dim, 41, device)
+        o, l = cbv.zigzag_ring_fwd(q, k, v, w.cu_seqlens, w.cp)
+        t_fast = timed(lambda: cbv.zigzag_ring_bwd(do, q, k, v, o, l, w.cu_seqlens, w.cp), 8, 3)
+        t_det = timed(lambda: cbv.zigzag_ring_bwd(do, q, k, v, o, l, w.cu_seqlens, w.cp, deterministic=True), 8, 3)
+        f_bwd = 10 * w.head_dim * w.heads * visible_pairs(w.cu_seqlens)
+        res[f"deterministic_bwd_{w.name}"] = {"bwd_tflops": f_bwd / t_det / 1e9, "ms": t_det, "default_ms": t_fast}
+        del q, k, v, do, o, l
+        torch.cuda.empty_cache()
+    if run("cached"):
+        # EAGLE-3 cached ring on the packed workload: the sequence block plus 3 cache diagonals.  The
+        # diagonals' cost is the time above the plain ring on the same sequence block, set against the
+        # bytes that the two diagonal kernels must move (and the fp32 block output they add).
+        w = packed_zigzag()
+        nb, S, H, D = 4, w.total, w.heads, w.head_dim
+        q = torch_normal_bf16((S, H, D), 31, device)
+        ck = torch_normal_bf16((nb, S, H, D), 32, device)
+        cv = torch_normal_bf16((nb, S, H, D), 33, device)
+        do = torch_normal_bf16((S, H, D), 34, device)
         st = {}
 
-        def fwd():
-            st["o"], st["l"] = cbv.zigzag_ring_fwd(q, k, v, w.cu_seqlens, w.cp, window=window, layout=layout)
+        def cfwd():
+            st["o"], st["l"] = cbv.cached_ring_fwd(q, ck, cv, w.cu_seqlens, w.cp)
 
-        def bwd():
-            cbv.zigzag_ring_bwd(do, q, k, v, st["o"], st["l"], w.cu_seqlens, w.cp, window=window, layout=layout)
+        def cbwd():
+            cbv.cached_ring_bwd(do, q, ck, cv, st["o"], st["l"], w.cu_seqlens, w.cp)
 
-        fwd()
-        t_f = timed(fwd, 5, 2)
-        t_b = timed(bwd, 5, 2)
-        f_fwd = 4 * w.head_dim * w.heads * pairs
-        f_bwd = 10 * w.head_dim * w.heads * pairs
-        key = f"long_doc_S65536_cp8_H16_{layout}" + (f"_W{window}" if window else "")
-        res[key] = {"fwd_tflops": f_fwd / t_f / 1e9, "bwd_tflops": f_bwd / t_b / 1e9,
-                    "fwd_bwd_tflops": (f_fwd + f_bwd) / (t_f + t_b) / 1e9,
-                    "fwd_bwd_frac": (f_fwd + f_bwd) / (t_f + t_b) / 1e9 / tf_peak, "ms": t_f + t_b}
-        del q, k, v, do, st
+        def pfwd():
+            st["po"], st["pl"] = cbv.zigzag_ring_fwd(q, ck[0], cv[0], w.cu_seqlens, w.cp)
+
+        def pbwd():
+            cbv.zigzag_ring_bwd(do, q, ck[0], cv[0], st["po"], st["pl"], w.cu_seqlens, w.cp)
+
+        cfwd()
+        pfwd()
+        t_cf, t_cb = timed(cfwd, 8, 3), timed(cbwd, 8, 3)
+        t_pf, t_pb = timed(pfwd, 8, 3), timed(pbwd, 8, 3)
+        e = S * H * D
+        diag_kv = 2 * (nb - 1) * S * H * D * 2
+        b_fwd = e * 2 + e * 4 + diag_kv + S * H * 8 + e * 2 + e * 2  # q, o32, k/v diagonals, lse r/w, out, o32's extra write
+        b_bwd = 3 * e * 2 + 2 * diag_kv + S * H * 4  # q, dO, out; k/v diagonals read, their gradients written; lse
+        pairs = visible_pairs(w.cu_seqlens)
+        f_all = 14 * D * H * pairs
+        res[f"cached_ring_{w.name}_NB{nb}"] = {
+            "fwd_bwd_tflops": f_all / (t_cf + t_cb) / 1e9, "ms": t_cf + t_cb, "plain_ms": t_pf + t_pb,
+            "diag_fwd_ms": t_cf - t_pf, "diag_bwd_ms": t_cb - t_pb,
+            "diag_fwd_gbs": b_fwd / max(t_cf - t_pf, 1e-6) / 1e6, "diag_bwd_gbs": b_bwd / max(t_cb - t_pb, 1e-6) / 1e6}
+        del q, ck, cv, do, st
         torch.cuda.empty_cache()
-    # deterministic backward (dq summed in 64-bit fixed point) against the default, packed workload
-    w = packed_zigzag()
-    q, k, v, do = make_ring_inputs(w.cu_seqlens, w.heads, w.head_dim, 41, device)
-    o, l = cbv.zigzag_ring_fwd(q, k, v, w.cu_seqlens, w.cp)
-    t_fast = timed(lambda: cbv.zigzag_ring_bwd(do, q, k, v, o, l, w.cu_seqlens, w.cp), 8, 3)
-    t_det = timed(lambda: cbv.zigzag_ring_bwd(do, q, k, v, o, l, w.cu_seqlens, w.cp, deterministic=True), 8, 3)
-    f_bwd = 10 * w.head_dim * w.heads * visible_pairs(w.cu_seqlens)
-    res[f"deterministic_bwd_{w.name}"] = {"bwd_tflops": f_bwd / t_det / 1e9, "ms": t_det, "default_ms": t_fast}
-    del q, k, v, do, o, l
-    torch.cuda.empty_cache()
-    # EAGLE-3 cached ring on the packed workload: the sequence block plus 3 cache diagonals.  The
-    # diagonals' cost is the time above the plain ring on the same sequence block, set against the
-    # bytes that the two diagonal kernels must move (and the fp32 block output they add).
-    w = packed_zigzag()
-    nb, S, H, D = 4, w.total, w.heads, w.head_dim
-    q = torch_normal_bf16((S, H, D), 31, device)
-    ck = torch_normal_bf16((nb, S, H, D), 32, device)
-    cv = torch_normal_bf16((nb, S, H, D), 33, device)
-    do = torch_normal_bf16((S, H, D), 34, device)
-    st = {}
-
-    def cfwd():
-        st["o"], st["l"] = cbv.cached_ring_fwd(q, ck, cv, w.cu_seqlens, w.cp)
-
-    def cbwd():
-        cbv.cached_ring_bwd(do, q, ck, cv, st["o"], st["l"], w.cu_seqlens, w.cp)
-
-    def pfwd():
-        st["po"], st["pl"] = cbv.zigzag_ring_fwd(q, ck[0], cv[0], w.cu_seqlens, w.cp)
-
-    def pbwd():
-        cbv.zigzag_ring_bwd(do, q, ck[0], cv[0], st["po"], st["pl"], w.cu_seqlens, w.cp)
-
-    cfwd()
-    pfwd()
-    t_cf, t_cb = timed(cfwd, 8, 3), timed(cbwd, 8, 3)
-    t_pf, t_pb = timed(pfwd, 8, 3), timed(pbwd, 8, 3)
-    e = S * H * D
-    diag_kv = 2 * (nb - 1) * S * H * D * 2
-    b_fwd = e * 2 + e * 4 + diag_kv + S * H * 8 + e * 2 + e * 2  # q, o32, k/v diagonals, lse r/w, out, o32's extra write
-    b_bwd = 3 * e * 2 + 2 * diag_kv + S * H * 4  # q, dO, out; k/v diagonals read, their gradients written; lse
-    pairs = visible_pairs(w.cu_seqlens)
-    f_all = 14 * D * H * pairs
-    res[f"cached_ring_{w.name}_NB{nb}"] = {
-        "fwd_bwd_tflops": f_all / (t_cf + t_cb) / 1e9, "ms": t_cf + t_cb, "plain_ms": t_pf + t_pb,
-        "diag_fwd_ms": t_cf - t_pf, "diag_bwd_ms": t_cb - t_pb,
-        "diag_fwd_gbs": b_fwd / max(t_cf - t_pf, 1e-6) / 1e6, "diag_bwd_gbs": b_bwd / max(t_cb - t_pb, 1e-6) / 1e6}
-    del q, ck, cv, do, st
-    torch.cuda.empty_cache()
-    # paged KV-parallel prefill, round-robin shards
-    for window in (0, 8192):
-        w = paged_prefill(window=window)
-        q = torch_normal_bf16((w.hq, w.q_len, w.head_dim), 11, device)
-        kc = torch_normal_bf16((w.kv_len // w.block_size, w.hkv, w.block_size, w.head_dim), 12, device)
-        vc = torch_normal_bf16(kc.shape, 13, device)
-        perm = w.perm.astype(np.int64)
-        bt = torch.from_numpy(np.stack([perm[r::w.shards] for r in range(w.shards)]).astype(np.int32)).to(device)
-        fn = lambda: cbv.kvp_segmented_prefill(q, kc, vc, bt, cbv.KV_ROUND_ROBIN, w.seg_size, None,
-                                               w.global_q_offset, window, return_lse=False)
+    if run("paged"):
+        # paged KV-parallel prefill, round-robin shards
+        for window in (0, 8192):
+            w = paged_prefill(window=window)
+            q = torch_normal_bf16((w.hq, w.q_len, w.head_dim), 11, device)
+            kc = torch_normal_bf16((w.kv_len // w.block_size, w.hkv, w.block_size, w.head_dim), 12, device)
+            vc = torch_normal_bf16(kc.shape, 13, device)
+            perm = w.perm.astype(np.int64)
+            bt = torch.from_numpy(np.stack([perm[r::w.shards] for r in range(w.shards)]).astype(np.int32)).to(device)
+            fn = lambda: cbv.kvp_segmented_prefill(q, kc, vc, bt, cbv.KV_ROUND_ROBIN, w.seg_size, None,
+                                                   w.global_q_offset, window, return_lse=False)
+            t = timed(fn, 10, 3)
+            qpos = w.global_q_offset + np.arange(w.q_len)
+            vis = np.minimum(qpos + 1, window) if window else qpos + 1
+            flops = 4 * w.head_dim * w.hq * int(vis.sum())
+            res[f"paged_prefill_S4096_KV32768_rr" + (f"_W{window}" if window else "")] = {
+                "tflops": flops / t / 1e9, "frac": flops / t / 1e9 / tf_peak, "ms": t}
+            del q, kc, vc
+            torch.cuda.empty_cache()
+    if run("decode"):
+        # one-query GQA varlen decode
+        w = varlen_decode(num_seqs=decode_seqs)
+        cu_k = torch.from_numpy(w.cu_seqlens_k).to(device)
+        cu_q = torch.arange(w.num_seqs + 1, dtype=torch.int32, device=device)
+        tk = int(w.cu_seqlens_k[-1])
+        q = torch_normal_bf16((w.num_seqs, w.hq, w.head_dim), 21, device)
+        k = torch_normal_bf16((tk, w.hkv, w.head_dim), 22, device)
+        v = torch_normal_bf16((tk, w.hkv, w.head_dim), 23, device)
+        out = torch.empty_like(q)
+        ws = torch.empty(256, dtype=torch.uint8, device=device)
+        fn = lambda: cbv.varlen_decode(q, k, v, cu_q, cu_k, validate=False, out=out, workspace=ws)
         t = timed(fn, 10, 3)
-        qpos = w.global_q_offset + np.arange(w.q_len)
-        vis = np.minimum(qpos + 1, window) if window else qpos + 1
-        flops = 4 * w.head_dim * w.hq * int(vis.sum())
-        res[f"paged_prefill_S4096_KV32768_rr" + (f"_W{window}" if window else "")] = {
-            "tflops": flops / t / 1e9, "frac": flops / t / 1e9 / tf_peak, "ms": t}
-        del q, kc, vc
+        nbytes = 2 * tk * w.hkv * w.head_dim * 2 + 2 * q.numel() * 2 + 2 * cu_k.numel() * 4
+        res[f"varlen_decode_N{w.num_seqs}_HQ32_HKV4"] = {"gbs": nbytes / t / 1e6, "frac": nbytes / t / 1e6 / pk["hbm_gbs"],
+                                                "ms": t, "bytes": nbytes}
+        del q, k, v, out
         torch.cuda.empty_cache()
-    # one-query GQA varlen decode
-    w = varlen_decode()
-    cu_k = torch.from_numpy(w.cu_seqlens_k).to(device)
-    cu_q = torch.arange(w.num_seqs + 1, dtype=torch.int32, device=device)
-    tk = int(w.cu_seqlens_k[-1])
-    q = torch_normal_bf16((w.num_seqs, w.hq, w.head_dim), 21, device)
-    k = torch_normal_bf16((tk, w.hkv, w.head_dim), 22, device)
-    v = torch_normal_bf16((tk, w.hkv, w.head_dim), 23, device)
-    out = torch.empty_like(q)
-    ws = torch.empty(256, dtype=torch.uint8, device=device)
-    fn = lambda: cbv.varlen_decode(q, k, v, cu_q, cu_k, validate=False, out=out, workspace=ws)
-    t = timed(fn, 10, 3)
-    nbytes = 2 * tk * w.hkv * w.head_dim * 2 + 2 * q.numel() * 2 + 2 * cu_k.numel() * 4
-    res["varlen_decode_N8192_HQ32_HKV4"] = {"gbs": nbytes / t / 1e6, "frac": nbytes / t / 1e6 / pk["hbm_gbs"],
-                                            "ms": t, "bytes": nbytes}
-    del q, k, v, out
-    torch.cuda.empty_cache()
-    # standalone merge at the packed workload's shapes
-    S, H, D = 16384, 32, 128
-    o = torch.randn((S, H, D), device=device)
-    l = torch.randn((H, S), device=device)
-    bo = torch.randn((S, H, D), device=device).to(torch.bfloat16)
-    bl = torch.randn((H, S), device=device)
-    t = timed(lambda: cbv.attn_merge(o, l, bo, bl), 20, 3)
-    nbytes = S * H * (D * 4 * 2 + D * 2 + 3 * 4)
-    res["merge_S16384_H32_D128"] = {"gbs": nbytes / t / 1e6, "frac": nbytes / t / 1e6 / pk["hbm_gbs"], "ms": t}
+    if run("merge"):
+        # standalone merge at the packed workload's shapes
+        S, H, D = 16384, 32, 128
+        o = torch.randn((S, H, D), device=device)
+        l = torch.randn((H, S), device=device)
+        bo = torch.randn((S, H, D), device=device).to(torch.bfloat16)
+        bl = torch.randn((H, S), device=device)
+        t = timed(lambda: cbv.attn_merge(o, l, bo, bl), 20, 3)
+        nbytes = S * H * (D * 4 * 2 + D * 2 + 3 * 4)
+        res["merge_S16384_H32_D128"] = {"gbs": nbytes / t / 1e6, "frac": nbytes / t / 1e6 / pk["hbm_gbs"], "ms": t}
     res["peak_kind"] = pk_kind
     return res
 
@@ -520,6 +530,11 @@ def main():
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     pk, pk_kind = peaks()
+    if args.only:
+        print(json.dumps(extra_benchmarks(device, pk, pk_kind, only=args.only, decode_seqs=args.decode_seqs)), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     w = rank_workload(args.workload, args.seed, rank)
     cu = w.cu_seqlens
