@@ -47,7 +47,8 @@ def parse_args():
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     p.add_argument("--workload", choices=["packed", "long_doc", "long_doc_small"], default="packed",
                    help="ring workload of the timed step (the headline is `packed`; the others are for profiling)")
-    p.add_argument("--only", choices=["long_doc", "deterministic", "cached", "paged", "decode", "merge"], default=None,
+    p.add_argument("--only", choices=["long_doc", "rank_balance", "deterministic", "cached", "paged", "decode", "merge"],
+                   default=None,
                    help="run one of the sub-benchmarks alone and print its result (for profiling); no headline line")
     p.add_argument("--decode-seqs", type=int, default=8192, help="sequences of the decode sub-benchmark")
     return p.parse_args()
@@ -310,6 +311,37 @@ def extra_benchmarks(device, pk, pk_kind, only=None, decode_seqs=8192):
                         "fwd_bwd_frac": (f_fwd + f_bwd) / (t_f + t_b) / 1e9 / tf_peak, "ms": t_f + t_b}
             del q, k, v, do, st
             torch.cuda.empty_cache()
+    if run("rank_balance"):
+        # each virtual rank's forward work alone (its q rows against the keys they see, one block
+        # call with explicit positions), long document: zig-zag ranks do equal work, contiguous
+        # ranks a growing share (the last about 2x the mean)
+        w = long_doc()
+        S, H, D, cp = w.total, w.heads, w.head_dim, w.cp
+        q, k, v, _ = make_ring_inputs(w.cu_seqlens, H, D, 9, device)
+        bal = {}
+        for layout in ("zigzag", "contiguous"):
+            times = []
+            for r in range(cp):
+                if layout == "zigzag":
+                    c = S // (2 * cp)
+                    parts = [(r * c, c), ((2 * cp - 1 - r) * c, c)]
+                else:
+                    c = S // cp
+                    parts = [(r * c, c)]
+                qr = torch.cat([q[a:a + n] for a, n in parts]).contiguous()
+                kr = torch.cat([k[:a + n] for a, n in parts]).contiguous()
+                vr = torch.cat([v[:a + n] for a, n in parts]).contiguous()
+                cu_q = np.cumsum([0] + [n for _, n in parts]).astype(np.int32)
+                cu_k = np.cumsum([0] + [a + n for a, n in parts]).astype(np.int32)
+                qb = np.array([a for a, _ in parts], np.int32)
+                kb = np.zeros(len(parts), np.int32)
+                fn = lambda: cbv.attn_block_fwd(qr, kr, vr, cu_q, cu_k, q_pos_base=qb, k_pos_base=kb)
+                times.append(timed(fn, 4, 2))
+                del qr, kr, vr
+            bal[layout] = {"rank_ms": times, "max_over_mean": max(times) / (sum(times) / len(times))}
+        res[f"rank_balance_{w.name}_fwd"] = bal
+        del q, k, v
+        torch.cuda.empty_cache()
     if run("deterministic"):
         # deterministic backward (dq summed in 64-bit fixed point) against the default, packed workload
         w = packed_zigzag()
