@@ -167,10 +167,9 @@ int upload_plan(const PlanDev& d, const Plan& p, cudaStream_t s) {
   memcpy(img.data(), p.groups.data(), p.groups.size() * sizeof(PlanGroup));
   memcpy(img.data() + d.off_tiles, p.tiles.data(), p.tiles.size() * sizeof(TileTask));
   memcpy(img.data() + d.off_segs, p.segs.data(), p.segs.size() * sizeof(Seg));
-  int e = launch_inline_copy(d.image, img.data(), img.size(), s);
-  if (e) return cuda_fail(e, "uploading the schedule");
-  e = launch_expand_tasks(d.groups, (int)p.groups.size(), d.tiles, d.tasks, (int)p.tasks.size(), s);
-  return e ? cuda_fail(e, "expanding the schedule") : CBV_OK;
+  const int e = launch_schedule(d.image, img.data(), img.size(), d.off_tiles, (int)p.groups.size(), d.tasks,
+                                (int)p.tasks.size(), s);
+  return e ? cuda_fail(e, "uploading the schedule") : CBV_OK;
 }
 
 int launch_rc(int e, const char* what) { return e == 0 ? CBV_OK : cuda_fail(e, what); }

@@ -194,6 +194,38 @@ __global__ void __launch_bounds__(256) inline_copy_kernel(const __grid_constant_
   for (uint32_t i = threadIdx.x; i < c.n16; i += blockDim.x) c.dst[i] = c.data[i];
 }
 
+// The usual case, a schedule image that fits one payload: one launch both writes the image to
+// the workspace (block 0) and expands the task list, reading the groups and tiles straight from
+// its own parameters.
+struct ScheduleChunk {
+  uint4* dst;                // the image's place in the workspace
+  TileTask* tasks;           // the expanded task list
+  uint32_t n16;              // image size, 16-byte words
+  uint32_t off_tiles;        // byte offset of the tiles in the image (the groups start at 0)
+  int32_t ngroups, ntasks;
+  uint4 data[kInlineBytes / 16];
+};
+
+__global__ void __launch_bounds__(256) schedule_kernel(const __grid_constant__ ScheduleChunk c) {
+  if (blockIdx.x == 0)
+    for (uint32_t i = threadIdx.x; i < c.n16; i += blockDim.x) c.dst[i] = c.data[i];
+  const PlanGroup* groups = reinterpret_cast<const PlanGroup*>(c.data);
+  const TileTask* tiles = reinterpret_cast<const TileTask*>(reinterpret_cast<const unsigned char*>(c.data) + c.off_tiles);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < c.ntasks; i += gridDim.x * blockDim.x) {
+    int lo = 0, hi = c.ngroups - 1;  // the last group whose first task is <= i
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) / 2;
+      if (groups[mid].first_task <= i) lo = mid;
+      else hi = mid - 1;
+    }
+    const PlanGroup g = groups[lo];
+    const int local = i - g.first_task;
+    TileTask t = tiles[g.first_tile + local % g.ntiles];
+    t.head = local / g.ntiles;
+    c.tasks[i] = t;
+  }
+}
+
 __global__ void __launch_bounds__(256) expand_tasks_kernel(const PlanGroup* __restrict__ groups, int ngroups,
                                                            const TileTask* __restrict__ tiles,
                                                            TileTask* __restrict__ tasks, int ntasks) {
@@ -304,6 +336,29 @@ int launch_inline_copy(void* dst, const void* src, size_t bytes, cudaStream_t st
     if (e) return e;
   }
   return 0;
+}
+
+int launch_schedule(void* image_dst, const void* image, size_t bytes, size_t off_tiles, int ngroups, TileTask* tasks,
+                    int ntasks, cudaStream_t stream) {
+  if (ntasks == 0 || ngroups == 0) return 0;
+  if (bytes > (size_t)kInlineBytes || bytes % 16) {  // larger images: copy in pieces, then expand
+    int e = launch_inline_copy(image_dst, image, bytes, stream);
+    if (e) return e;
+    return launch_expand_tasks(static_cast<const PlanGroup*>(image_dst), ngroups,
+                               reinterpret_cast<const TileTask*>(static_cast<unsigned char*>(image_dst) + off_tiles),
+                               tasks, ntasks, stream);
+  }
+  ScheduleChunk c;
+  c.dst = static_cast<uint4*>(image_dst);
+  c.tasks = tasks;
+  c.n16 = (uint32_t)(bytes / 16);
+  c.off_tiles = (uint32_t)off_tiles;
+  c.ngroups = ngroups;
+  c.ntasks = ntasks;
+  memcpy(c.data, image, bytes);
+  const int blocks = std::min((ntasks + 255) / 256, 148 * 4);
+  schedule_kernel<<<blocks, 256, 0, stream>>>(c);
+  return launched();
 }
 
 int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* tiles, TileTask* tasks, int ntasks,

@@ -111,8 +111,8 @@ def test_status_word_is_clear_after_a_run():
 
 
 def test_each_call_launches_its_schedule_upload_and_kernels():
-    # forward: schedule image (one launch per 30 KB) + task expansion + the forward kernel;
-    # backward: the same two + Delta + the backward kernel + the dq conversion
+    # forward: the schedule (image and task expansion in one launch while the image fits 30 KB) + the
+    # forward kernel; backward: the schedule + Delta + the backward kernel + the dq conversion
     cu, q, k, v, do = _case(3, [264, 520, 128], 2, 2, 128)
     tq, tk, tv, tdo = dev(q), dev(k), dev(v), dev(do)
     n0 = cbv.launch_count()
@@ -121,4 +121,4 @@ def test_each_call_launches_its_schedule_upload_and_kernels():
     cbv.zigzag_ring_bwd(tdo, tq, tk, tv, out, lse, cu, 2)
     n2 = cbv.launch_count()
     sync()
-    assert n1 - n0 == 3 and n2 - n1 == 5
+    assert n1 - n0 == 2 and n2 - n1 == 4
