@@ -191,3 +191,24 @@ def test_wrong_output_tensors_are_refused_before_any_launch():
         # the right shape, but not contiguous
         cbv.attn_block_bwd(do, q, k, v, out, lse, cu, cu, dq_acc=torch.zeros((2, 128, 64), device="cuda").transpose(0, 1))
     assert n1 - n0 == 2 and cbv.launch_count() == n1  # only the good forward launched anything
+
+
+def test_many_tiny_documents_take_the_large_schedule_path():
+    # 600 documents of 16 tokens: thousands of tiles, a schedule image far over one launch's 30 KB of
+    # parameters, so it is uploaded in pieces and expanded by a second kernel
+    cu = cu_from_lengths([16] * 600)
+    S, H, D = int(cu[-1]), 2, 64
+    q, k, v, do = gen(65, (S, H, D), (S, H, D), (S, H, D), (S, H, D))
+    n0 = cbv.launch_count()
+    out, lse = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, 2)
+    n1 = cbv.launch_count()
+    dq, dk, dv = cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out, lse, cu, 2)
+    sync()
+    assert n1 - n0 > 2  # the schedule took more than the one-launch path
+    ro, rl = A.attention_fwd(f64(q), f64(k), f64(v), cu, cu, D ** -0.5, causal=True)
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+    rq, rk, rv = A.attention_bwd(f64(do), f64(q), f64(k), f64(v), host(out), host(lse), cu, cu, D ** -0.5, causal=True)
+    check_rel(host(dq), rq, what="dq")
+    check_rel(host(dk), rk, what="dk")
+    check_rel(host(dv), rv, what="dv")
