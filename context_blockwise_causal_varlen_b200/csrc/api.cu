@@ -500,23 +500,51 @@ static int kvp_checks(const cbv_kvp_args* a) {
   return CBV_OK;
 }
 
-static size_t kvp_layout(const cbv_kvp_args* a, Plan* plan_out) {
+// Tasks of a prefill are about equal in size, so a last wave of CTAs that is at most half full
+// costs as much time as a full one.  Those tail tasks run instead as two halves each, cut where
+// the visible work is split evenly (TileTask::split1), so the last wave is full and half as
+// long; merge_halves_kernel combines the halves' partial (out, lse).  Returns how many tasks at
+// the end of the list run that way (0 without a device to ask, or when the tail is too light
+// to repay the merge).
+constexpr int64_t kMinSplitWork = 16 * 128;  // 16 k tiles of a 256-row task, in TileTask::work units
+static int kvp_tail_tasks(const Plan& plan) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const int nt = (int)plan.tasks.size();
+  if (sms <= 0 || nt == 0) return 0;
+  const int tail = nt % sms;
+  if (tail == 0 || 2 * tail > sms) return 0;
+  int64_t w = 0;
+  for (int i = nt - tail; i < nt; ++i) w += plan.tasks[i].work;
+  return w >= kMinSplitWork * tail ? tail : 0;
+}
+
+static size_t kvp_layout(const cbv_kvp_args* a, Plan* plan_out, int* tail_out) {
   const int n_local = a->blocks_per_shard * a->block_size;
   Plan plan = plan_kvp(a->q_len, a->num_heads, a->shards, n_local, a->seg_size, (KvMode)a->kv_mode, a->block_size,
                        a->global_q_offset, a->sliding_window, a->shard_out != nullptr, kPairRows);
+  const int tail = a->shard_out ? 0 : kvp_tail_tasks(plan);
   Carve c(nullptr);
   c.take(kStatusBytes);
   carve_plan(c, plan);
   const size_t rows = (size_t)a->num_heads * a->q_len;
   if (!a->lse || a->shard_out) c.take(rows * sizeof(float));                // lse scratch / merged lse
   if (a->shard_out) c.take(rows * a->head_dim * sizeof(float));             // merged fp32 out
+  if (tail) {
+    c.take(2 * rows * a->head_dim * sizeof(float));                         // the halves' partial out
+    c.take(2 * rows * sizeof(float));                                       // and lse
+  }
   if (plan_out) *plan_out = std::move(plan);
+  if (tail_out) *tail_out = tail;
   return c.off;
 }
 
 size_t cbv_kvp_workspace_size(const cbv_kvp_args* a) {
   if (kvp_checks(a)) return 0;
-  return kvp_layout(a, nullptr);
+  return kvp_layout(a, nullptr, nullptr);
 }
 
 int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
@@ -525,7 +553,8 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   if (a->q_len == 0) return CBV_OK;  // no query rows: nothing to write
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Plan plan;
-  const size_t need = kvp_layout(a, &plan);
+  int tail = 0;
+  const size_t need = kvp_layout(a, &plan, &tail);
   if (!a->workspace || a->workspace_bytes < need) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", need);
   Carve c(a->workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
@@ -533,6 +562,8 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   const size_t rows = (size_t)a->num_heads * a->q_len;
   float* lse_scratch = (!a->lse || a->shard_out) ? static_cast<float*>(c.take(rows * sizeof(float))) : nullptr;
   float* acc = a->shard_out ? static_cast<float*>(c.take(rows * a->head_dim * sizeof(float))) : nullptr;
+  float* part = tail ? static_cast<float*>(c.take(2 * rows * a->head_dim * sizeof(float))) : nullptr;
+  float* part_lse = tail ? static_cast<float*>(c.take(2 * rows * sizeof(float))) : nullptr;
   const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads, bs = a->block_size;
   FwdParams p{};
   if ((rc = map_thd(&p.tm_q, a->q, a->q_len, H, D, a->q_stride_token, a->q_stride_head, 128))) return rc;
@@ -571,7 +602,19 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
     p.lse = a->lse ? a->lse : lse_scratch;
     p.lse_stride_h = a->q_len;
     p.lse_stride_t = 1;
-    return launch_rc(launch_fwd_pingpong(p, D, true, grid, s), "prefill launch");
+    const int full = grid - tail;
+    // the tail tasks: two CTAs each, in the same launch, so the halves take SMs as they free up
+    p.split_halves = tail > 0;
+    p.split_from = full;
+    p.half_out = part;
+    p.half_lse = part_lse;
+    p.half_rows = (int64_t)rows;
+    p.half_q_len = a->q_len;
+    if ((rc = launch_rc(launch_fwd_pingpong(p, D, true, full + 2 * tail, s), "prefill launch"))) return rc;
+    if (!tail) return CBV_OK;
+    return launch_rc(launch_merge_halves(pd.tasks + full, tail, part, part_lse, H, a->q_len, D, a->out, p.out_stride_h,
+                                         p.out_stride_t, p.out_stride_d, a->lse, s),
+                     "prefill tail merge");
   }
   // per-shard partials, then an explicit online-softmax merge of the shards
   p.out = a->shard_out;

@@ -147,7 +147,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const TileTask t = p.tasks[blockIdx.x];
+  int tix = (int)blockIdx.x, half = -1;
+  if (p.split_halves && tix >= p.split_from) {
+    half = (tix - p.split_from) & 1;
+    tix = p.split_from + ((tix - p.split_from) >> 1);
+  }
+  TileTask t = p.tasks[tix];
+  if (half >= 0) {
+    // one half of a split task: its share of the segments, written to output slot 0 or 1
+    const int cut = min(max(t.split1, 0), t.nseg);
+    if (half == 0) {
+      t.nseg = cut;
+    } else {
+      t.seg0 += cut;
+      t.nseg -= cut;
+    }
+    t.aux = half;
+  }
   const int head = t.head;
   const int kvh = head / p.heads_per_kv;
   const bool has_b = t.rows > BM;
@@ -424,6 +440,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       }
     }
     // ---------------------------------------------------------------- epilogue
+    // where this CTA writes: the call's output, or for one half of a split task its fp32 slot
+    const bool hx = half >= 0;
+    const int o_mode = hx ? (int)kOutF32 : p.out_mode;
+    void* const o_base = hx ? static_cast<void*>(p.half_out) : p.out;
+    const int64_t o_t = hx ? (int64_t)D : p.out_stride_t, o_h = hx ? p.half_q_len * D : p.out_stride_h;
+    const int64_t o_d = hx ? 1 : p.out_stride_d, o_sh = hx ? p.half_rows * D : p.out_shard_stride;
+    float* const l_base = hx ? p.half_lse : p.lse;
+    const int64_t l_h = hx ? p.half_q_len : p.lse_stride_h, l_t = hx ? 1 : p.lse_stride_t;
+    const int64_t l_sh = hx ? p.half_rows : p.lse_shard_stride;
     // split task: half B hands its softmax state to half A, which merges the two
     // (every softmax warp reaches the barrier once, whatever happened before)
     float wa_o = 1.f, wb_o = 0.f;  // weights of O_A and O_B in the merged accumulator
@@ -449,9 +474,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       const bool valid = trow < t.rows;
       const int64_t orow = (int64_t)(t.row0 + trow);
       const int64_t shard_off = t.aux >= 0 ? (int64_t)t.aux : 0;  // per-shard outputs
-      float* lse_ptr = p.lse + shard_off * p.lse_shard_stride + (int64_t)head * p.lse_stride_h + orow * p.lse_stride_t;
+      float* lse_ptr = l_base + shard_off * l_sh + (int64_t)head * l_h + orow * l_t;
       float wa = 0.f, wb = 1.f, lse_new = lse_b;
-      if (p.out_mode == kOutMerge && valid) {
+      if (o_mode == kOutMerge && valid) {
         const float lse_a = *lse_ptr;
         const float mm = fmaxf(lse_a, lse_b);
         if (mm == -INFINITY) {
@@ -484,16 +509,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        if (p.out_mode == kOutBf16 && p.out_stride_d > 1) {
+        if (o_mode == kOutBf16 && o_d > 1) {
           // transposed output: lanes hold consecutive rows, so each store covers 32 adjacent rows
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + shard_off * p.out_shard_stride +
-                               orow * p.out_stride_t + (int64_t)head * p.out_stride_h + (int64_t)c * p.out_stride_d;
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o_base) + shard_off * o_sh +
+                               orow * o_t + (int64_t)head * o_h + (int64_t)c * o_d;
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            dst[(int64_t)e * p.out_stride_d] = __float2bfloat16_rn(__uint_as_float(o[e]) * inv_l);
-        } else if (p.out_mode == kOutBf16) {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + shard_off * p.out_shard_stride + orow * p.out_stride_t +
-                               (int64_t)head * p.out_stride_h + c;
+            dst[(int64_t)e * o_d] = __float2bfloat16_rn(__uint_as_float(o[e]) * inv_l);
+        } else if (o_mode == kOutBf16) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(o_base) + shard_off * o_sh + orow * o_t +
+                               (int64_t)head * o_h + c;
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 v;
@@ -504,8 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
             *reinterpret_cast<uint4*>(dst + e) = v;
           }
         } else {
-          float* dst = reinterpret_cast<float*>(p.out) + shard_off * p.out_shard_stride + orow * p.out_stride_t +
-                     (int64_t)head * p.out_stride_h + c;
+          float* dst = reinterpret_cast<float*>(o_base) + shard_off * o_sh + orow * o_t +
+                     (int64_t)head * o_h + c;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             float4 v;
@@ -513,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
             v.y = __uint_as_float(o[e + 1]) * inv_l;
             v.z = __uint_as_float(o[e + 2]) * inv_l;
             v.w = __uint_as_float(o[e + 3]) * inv_l;
-            if (p.out_mode == kOutMerge) {
+            if (o_mode == kOutMerge) {
               const float4 a = *reinterpret_cast<const float4*>(dst + e);
               v.x = a.x * wa + v.x * wb;
               v.y = a.y * wa + v.y * wb;

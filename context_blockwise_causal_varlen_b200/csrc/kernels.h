@@ -39,6 +39,14 @@ struct FwdParams {
   int64_t lse_stride_h, lse_stride_t;  // elements
   int32_t out_mode;
   int64_t out_shard_stride, lse_shard_stride;  // per-shard outputs (task.aux = shard >= 0)
+  // with split_halves, the tasks from split_from on run as two halves each: CTA split_from + 2j
+  // takes segments [0, split1) of task split_from + j and CTA split_from + 2j + 1 the rest.  A
+  // half writes its normalised partial (out, lse) in fp32 to slot 0 or 1 of half_out
+  // [2][H][S][D] and half_lse [2][H][S] (half_rows = H * S, half_q_len = S).
+  int32_t split_halves, split_from;
+  float* half_out;
+  float* half_lse;
+  int64_t half_rows, half_q_len;
   // paged KV
   const int32_t* block_tables;  // [shards, blocks_per_shard]
   int32_t blocks_per_shard, block_size, shards, kv_mode, n_local;
@@ -98,6 +106,13 @@ int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* ti
                         cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
+// The two halves of each of `ntasks` split prefill tasks (q tiles of up to 256 rows), whose
+// partial (out, lse) sit in slots 0 and 1 of part [2][H][S][D] and part_lse [2][H][S], merged into
+// the bf16 out (element (h, t, d) at h * out_stride_h + t * out_stride_t + d * out_stride_d) and,
+// when lse is not null, lse [H][S].
+int launch_merge_halves(const TileTask* tasks, int ntasks, const float* part, const float* part_lse, int heads,
+                        int64_t q_len, int head_dim, void* out, int64_t out_stride_h, int64_t out_stride_t,
+                        int64_t out_stride_d, float* lse, cudaStream_t stream);
 // fp32 [H, S, D] -> bf16 [H, D, S] (the prefill's transposed output).
 int launch_convert_bf16_transposed(const float* src, void* dst, int H, int64_t S, int D, cudaStream_t stream);
 // The fixed-point dq accumulator of the deterministic backward is [H][4][t_pad][D/4]: each of the

@@ -244,6 +244,55 @@ __global__ void __launch_bounds__(256) expand_tasks_kernel(const PlanGroup* __re
   }
 }
 
+// The two halves of a split prefill task attend disjoint parts of the keys for the same q rows.
+// Their normalised partials combine by the log-sum-exp identity (update_out_and_lse):
+// lse = log(e^lse0 + e^lse1) and out = e^(lse0 - lse) out0 + e^(lse1 - lse) out1, rounded
+// to the bf16 output (head-major rows; a head-dim stride > 1 gives the transposed layout).
+// A half at -inf has weight 0; both at -inf give out = 0 and lse = -inf.
+template <int D>
+__global__ void __launch_bounds__(256) merge_halves_kernel(const TileTask* __restrict__ tasks,
+                                                           const float* __restrict__ part,
+                                                           const float* __restrict__ part_lse, int64_t part_stride,
+                                                           int64_t lse_part_stride, int64_t q_len,
+                                                           __nv_bfloat16* __restrict__ out, int64_t out_stride_h,
+                                                           int64_t out_stride_t, int64_t out_stride_d,
+                                                           float* __restrict__ lse) {
+  constexpr int L = D / 8;         // lanes per row, 8 elements each
+  constexpr int kRows = 256 / L;   // rows per block
+  const TileTask t = tasks[blockIdx.x];
+  const int r = blockIdx.y * kRows + (int)threadIdx.x / L;
+  if (r >= t.rows) return;
+  const int c = ((int)threadIdx.x % L) * 8;
+  const int64_t row = (int64_t)t.row0 + r;
+  const int64_t li = (int64_t)t.head * q_len + row;
+  const float l0 = part_lse[li], l1 = part_lse[lse_part_stride + li];
+  const float m = fmaxf(l0, l1);
+  float w0 = 0.f, w1 = 0.f, nl = -INFINITY;
+  if (m != -INFINITY) {
+    nl = m + __logf(__expf(l0 - m) + __expf(l1 - m));
+    w0 = __expf(l0 - nl);
+    w1 = __expf(l1 - nl);
+  }
+  const float4* a = reinterpret_cast<const float4*>(part + li * D + c);
+  const float4* b = reinterpret_cast<const float4*>(part + part_stride + li * D + c);
+  const float4 a0 = __ldg(a), a1 = __ldg(a + 1), b0 = __ldg(b), b1 = __ldg(b + 1);
+  const float v[8] = {a0.x * w0 + b0.x * w1, a0.y * w0 + b0.y * w1, a0.z * w0 + b0.z * w1, a0.w * w0 + b0.w * w1,
+                      a1.x * w0 + b1.x * w1, a1.y * w0 + b1.y * w1, a1.z * w0 + b1.z * w1, a1.w * w0 + b1.w * w1};
+  __nv_bfloat16* dst = out + (int64_t)t.head * out_stride_h + row * out_stride_t;
+  if (out_stride_d <= 1) {
+    uint4 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    u.z = pack_bf16x2(v[4], v[5]);
+    u.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(dst + c) = u;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[(int64_t)(c + e) * out_stride_d] = __float2bfloat16_rn(v[e]);
+  }
+  if (c == 0 && lse) lse[li] = nl;
+}
+
 }  // namespace
 
 int launch_merge(float* out, float* lse, const void* block_out, int32_t block_out_is_f32, const float* block_lse,
@@ -261,6 +310,24 @@ int launch_merge(float* out, float* lse, const void* block_out, int32_t block_ou
       merge_kernel<64, false><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
     else
       merge_kernel<64, true><<<blocks, 256, 0, stream>>>(out, lse, block_out, block_lse, weight_out, seqlen, heads);
+  } else {
+    return (int)cudaErrorInvalidValue;
+  }
+  return launched();
+}
+
+int launch_merge_halves(const TileTask* tasks, int ntasks, const float* part, const float* part_lse, int heads,
+                        int64_t q_len, int head_dim, void* out, int64_t out_stride_h, int64_t out_stride_t,
+                        int64_t out_stride_d, float* lse, cudaStream_t stream) {
+  if (ntasks <= 0) return 0;
+  const int64_t part_stride = (int64_t)heads * q_len * head_dim, lse_part_stride = (int64_t)heads * q_len;
+  auto o = static_cast<__nv_bfloat16*>(out);
+  if (head_dim == 128) {
+    merge_halves_kernel<128><<<dim3((unsigned)ntasks, 256 / 16), 256, 0, stream>>>(
+        tasks, part, part_lse, part_stride, lse_part_stride, q_len, o, out_stride_h, out_stride_t, out_stride_d, lse);
+  } else if (head_dim == 64) {
+    merge_halves_kernel<64><<<dim3((unsigned)ntasks, 256 / 32), 256, 0, stream>>>(
+        tasks, part, part_lse, part_stride, lse_part_stride, q_len, o, out_stride_h, out_stride_t, out_stride_d, lse);
   } else {
     return (int)cudaErrorInvalidValue;
   }

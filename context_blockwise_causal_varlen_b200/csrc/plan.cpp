@@ -441,6 +441,32 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
       int64_t lo = window > 0 ? std::max<int64_t>(0, pos0 - window + 1) : 0;
       int64_t span = (int64_t)pos0 + rows - lo;
       t.work = weight((int64_t)rows * span / (per_shard ? shards : 1));
+      // where to cut the segment list for two halves of about equal work: count the 128-key
+      // tiles of each segment this tile sees (the kernel's own skip rule)
+      int64_t total = 0;
+      std::vector<int64_t> seen(t.nseg);
+      for (int32_t i = 0; i < t.nseg; ++i) {
+        const Seg& g = plan.segs[t.seg0 + i];
+        const int32_t r = g.flags >> kSegShardShift;
+        int64_t n = 0;
+        for (int32_t c0 = 0; c0 < g.rows; c0 += 128) {
+          const int32_t nv = std::min(128, g.rows - c0);
+          const int64_t kp0 = kvp_position(r, g.row0 + c0, n_local, block_size, shards, mode);
+          const int64_t kp1 = kvp_position(r, g.row0 + c0 + nv - 1, n_local, block_size, shards, mode);
+          if (kp0 > (int64_t)pos0 + rows - 1) continue;
+          if (window > 0 && kp1 < (int64_t)pos0 - window + 1) continue;
+          ++n;
+        }
+        seen[i] = n;
+        total += n;
+      }
+      int64_t acc = 0;
+      t.split1 = t.nseg > 1 ? 1 : t.nseg;
+      for (int32_t i = 0; i + 1 < t.nseg; ++i) {
+        acc += seen[i];
+        t.split1 = i + 1;
+        if (2 * acc >= total) break;
+      }
       plan.tasks.push_back(t);
     }
   }

@@ -27,9 +27,11 @@ struct TileTask {
   int32_t aux;   // paged prefill: shard of the single-shard variant (-1 = all shards)
   int32_t head;  // head (q head in the forward, kv head in the backward); one task per tile and head
   int32_t work;  // estimated visible pairs / 256 (scheduling weight)
-  // backward only: a second key range in the same tile (split1 > 0).  Tile rows [0, split1)
+  // backward: a second key range in the same tile (split1 > 0).  Tile rows [0, split1)
   // hold rows row0.. (valid: the first `rows`), tile rows [split1, 128) hold rows row1..
   // (valid: the first rows1, positions pos1..).  split1 is a multiple of 8.
+  // paged prefill forward: split1 is the segment where the task is cut when it runs as two
+  // halves of about equal visible work.
   int32_t row1, pos1, rows1, split1;
 };
 

@@ -121,3 +121,24 @@ def test_kvp_transposed_output_is_the_transpose(per_shard, D, S):
     K, V = PG.global_kv(f64(kc), f64(vc), bt.numpy(), bs, PG.ROUND_ROBIN)
     ro, _ = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=500)
     check_out(host(b[0]).transpose(0, 2, 1), ro)
+
+
+@pytest.mark.parametrize("window,tp_out", [(0, False), (3000, True)])
+def test_kvp_tail_tasks_split_in_halves(window, tp_out):
+    # 11 q tile pairs x 16 heads = 176 tasks: 148 fill one wave and the other 28 run as two halves
+    # each (cut along the segment list), merged afterwards; every pair and head is sampled
+    R, bps, bs, hq, hkv, D, S = 4, 64, 32, 16, 4, 128, 11 * 256
+    q, kc, vc, perm = _paged(60, R, bps, bs, hq, hkv, D, S)
+    bt = PG.shard_block_tables(perm, R, PG.ROUND_ROBIN)
+    gqo = R * bps * bs - S
+    n0 = cbv.launch_count()
+    out, lse = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), seg_size=512, scale=0.1,
+                                         global_q_offset=gqo, sliding_window=window, tp_out=tp_out)
+    sync()
+    assert cbv.launch_count() - n0 == 3  # schedule, the prefill (whole tasks and halves), the merge
+    rows = np.unique(np.concatenate([[p, p + 1, p + 127, p + 128, p + 255] for p in range(0, S, 256)]))
+    K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, PG.ROUND_ROBIN)
+    ro, rl = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=window, rows=rows)
+    got = host(out).transpose(0, 2, 1) if tp_out else host(out)
+    check_out(got[:, rows], ro[:, rows])
+    check_lse(host(lse)[:, rows], rl[:, rows])
