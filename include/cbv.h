@@ -352,6 +352,11 @@ typedef struct cbv_kvp_args {
   void* workspace;
   size_t workspace_bytes;
 } cbv_kvp_args;
+/* Workspace bytes for a call with these arguments on the current device.  The size depends on
+ * the device's SM count: when the last wave of the prefill's tasks would fill at most half the
+ * SMs, those tasks run as two halves each, and the halves' fp32 partial results (8 bytes per
+ * element of out, 8 per lse entry) live in the workspace.  Query it on the device that runs
+ * the call; a smaller workspace makes the call return CBV_ERR_WORKSPACE_TOO_SMALL. */
 size_t cbv_kvp_workspace_size(const cbv_kvp_args* a);
 int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream);
 
