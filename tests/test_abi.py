@@ -235,3 +235,55 @@ def test_argument_errors_launch_nothing():
     a, _ = _ring_args(cu=np.array([0], np.int32))
     assert cbv.lib().cbv_zigzag_ring_bwd(ctypes.byref(a), None) == 0
     assert cbv.launch_count() == n0
+
+
+def _block_args(**kw):
+    cq = np.array([0, 64, 160], np.int32)
+    ck = np.array([0, 96, 200], np.int32)
+    a = cbv.BlockFwdArgs(struct_size=ctypes.sizeof(cbv.BlockFwdArgs), abi_version=cbv.ABI_VERSION, q=256, k=512,
+                         v=768, total_q=160, total_k=200, num_heads=4, num_kv_heads=2, head_dim=128, num_docs=2,
+                         cu_seqlens_q=cq.ctypes.data_as(cbv.c_i32p), cu_seqlens_k=ck.ctypes.data_as(cbv.c_i32p),
+                         causal=1, out_dtype=cbv.DTYPE_BF16, out=1024, lse=2048)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, (cq, ck)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("merge", 1, "BAD_DTYPE"),       # merging needs the f32 running out
+    ("out_dtype", 7, "BAD_DTYPE"),
+    ("q", 8, "MISALIGNED"),
+    ("out", 1032, "MISALIGNED"),
+    ("workspace", None, "WORKSPACE_TOO_SMALL"),
+])
+def test_block_forward_argument_errors(field, value, status):
+    # fake device addresses: every one of these is refused on the host, before any CUDA call
+    a, keep = _block_args(**{field: value})
+    rc = cbv.lib().cbv_attn_block_fwd(ctypes.byref(a), None)
+    assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
+
+
+def _kvp_args(**kw):
+    a = cbv.KvpArgs(struct_size=ctypes.sizeof(cbv.KvpArgs), abi_version=cbv.ABI_VERSION, q=256, q_stride_head=16 * 128,
+                    q_stride_token=128, q_len=16, num_heads=4, num_kv_heads=2, head_dim=128, k_cache=512, v_cache=768,
+                    num_blocks=8, block_size=32, shards=2, blocks_per_shard=4, kv_mode=cbv.KV_ROUND_ROBIN,
+                    seg_size=128, global_q_offset=100, out=1024)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("kv_mode", 5, "BAD_ARG"),
+    ("global_q_offset", -1, "BAD_ARG"),
+    ("shard_out", 4096, "BAD_ARG"),   # per-shard out without per-shard lse
+    ("q", 8, "MISALIGNED"),
+    ("q_stride_token", 132, "MISALIGNED"),
+    ("shards", 0, "BAD_SHAPE"),
+    ("num_kv_heads", 3, "GQA_MISMATCH"),
+    ("workspace", None, "WORKSPACE_TOO_SMALL"),
+])
+def test_prefill_argument_errors(field, value, status):
+    a = _kvp_args(**{field: value})
+    rc = cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)
+    assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
