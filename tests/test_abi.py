@@ -287,3 +287,22 @@ def test_prefill_argument_errors(field, value, status):
     a = _kvp_args(**{field: value})
     rc = cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)
     assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("dout", None, "BAD_ARG"),
+    ("dq_acc", 4104, "MISALIGNED"),
+    ("head_dim", 256, "UNSUPPORTED_HEAD_DIM"),
+    ("total_k", 150, "BAD_CU_SEQLENS"),   # the key offsets run past the key rows
+    ("workspace", None, "WORKSPACE_TOO_SMALL"),
+])
+def test_block_backward_argument_errors(field, value, status):
+    cq = np.array([0, 64, 160], np.int32)
+    ck = np.array([0, 96, 200], np.int32)
+    a = cbv.BlockBwdArgs(struct_size=ctypes.sizeof(cbv.BlockBwdArgs), abi_version=cbv.ABI_VERSION, dout=256, q=512,
+                         k=768, v=1024, out=1280, lse=1536, total_q=160, total_k=200, num_heads=4, num_kv_heads=2,
+                         head_dim=128, num_docs=2, cu_seqlens_q=cq.ctypes.data_as(cbv.c_i32p),
+                         cu_seqlens_k=ck.ctypes.data_as(cbv.c_i32p), causal=1, dq_acc=2048, dk_acc=2304, dv_acc=2560)
+    setattr(a, field, value)
+    rc = cbv.lib().cbv_attn_block_bwd(ctypes.byref(a), None)
+    assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
