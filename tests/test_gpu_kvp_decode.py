@@ -142,3 +142,20 @@ def test_kvp_tail_tasks_split_in_halves(window, tp_out):
     got = host(out).transpose(0, 2, 1) if tp_out else host(out)
     check_out(got[:, rows], ro[:, rows])
     check_lse(host(lse)[:, rows], rl[:, rows])
+
+
+def test_kvp_every_task_split_when_fewer_than_half_the_sms():
+    # one q tile pair x 16 heads = 16 tasks, fewer than half the SMs: every task runs as two halves
+    R, bps, bs, hq, hkv, D, S = 4, 32, 32, 16, 4, 128, 256
+    q, kc, vc, perm = _paged(61, R, bps, bs, hq, hkv, D, S)
+    bt = PG.shard_block_tables(perm, R, PG.CONTIGUOUS)
+    gqo = R * bps * bs - S
+    n0 = cbv.launch_count()
+    out, lse = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), kv_mode=cbv.KV_CONTIGUOUS,
+                                         seg_size=256, scale=0.1, global_q_offset=gqo, sliding_window=3000)
+    sync()
+    assert cbv.launch_count() - n0 == 3
+    K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, PG.CONTIGUOUS)
+    ro, rl = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=3000)
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
