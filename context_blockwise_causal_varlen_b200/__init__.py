@@ -147,10 +147,22 @@ class CachedRingArgs(ctypes.Structure):
     ]
 
 
+class RowRun(ctypes.Structure):
+    _fields_ = [("doc", ctypes.c_int32), ("row0", ctypes.c_int32), ("rows", ctypes.c_int32), ("pos0", ctypes.c_int32),
+                ("local0", ctypes.c_int32)]
+
+
+class RingBlock(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32), ("step", ctypes.c_int32), ("src", ctypes.c_int32), ("kind", ctypes.c_int32),
+                ("causal", ctypes.c_int32), ("q_half", ctypes.c_int32), ("k_half", ctypes.c_int32),
+                ("q_run0", ctypes.c_int32), ("q_nruns", ctypes.c_int32), ("k_run0", ctypes.c_int32),
+                ("k_nruns", ctypes.c_int32)]
+
+
 EXPORTS = [
     "cbv_last_error_message", "cbv_abi_version", "cbv_read_status", "cbv_launch_count",
     "cbv_local_cu_seqlens", "cbv_half_cu_seqlens", "cbv_get_half_index", "cbv_get_half_lse", "cbv_rank_tokens",
-    "cbv_rank_pair_counts", "cbv_ring_step",
+    "cbv_rank_pair_counts", "cbv_ring_step", "cbv_plan_zigzag",
     "cbv_block_fwd_workspace_size", "cbv_attn_block_fwd", "cbv_attn_merge",
     "cbv_zigzag_ring_fwd_workspace_size", "cbv_zigzag_ring_fwd", "cbv_zigzag_ring_bwd_workspace_size",
     "cbv_zigzag_ring_bwd", "cbv_block_bwd_workspace_size", "cbv_attn_block_bwd",
@@ -173,6 +185,8 @@ def _declare(L):
     L.cbv_rank_tokens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i32p]
     L.cbv_rank_pair_counts.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i64p]
     L.cbv_ring_step.argtypes = [ctypes.c_int32] * 4 + [c_i32p, c_i32p]
+    L.cbv_plan_zigzag.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(RingBlock),
+                                  ctypes.c_int32, c_i32p, ctypes.POINTER(RowRun), ctypes.c_int32, c_i32p]
     for name, st in (("block_fwd", BlockFwdArgs), ("zigzag_ring_fwd", RingArgs), ("zigzag_ring_bwd", RingArgs),
                      ("block_bwd", BlockBwdArgs), ("kvp", KvpArgs), ("decode", DecodeArgs),
                      ("cached_ring_fwd", CachedRingArgs), ("cached_ring_bwd", CachedRingArgs)):
@@ -321,6 +335,28 @@ def ring_step(rank: int, step: int, cp: int, layout="zigzag") -> tuple[int, int]
     src, kind = ctypes.c_int32(0), ctypes.c_int32(0)
     _check(lib().cbv_ring_step(rank, step, cp, _layout(layout), ctypes.byref(src), ctypes.byref(kind)))
     return src.value, kind.value
+
+
+def plan_zigzag(cu_seqlens, cp: int, layout="zigzag") -> list[dict]:
+    """Per-step block descriptors of the ring (see ``cbv_plan_zigzag``): one dict per (rank, step) with
+    ``rank, step, src, kind, causal, q_half, k_half`` and ``q_runs`` / ``k_runs``, lists of
+    ``(doc, row0, rows, pos0, local0)`` runs of global rows in local order."""
+    cu = _host_i32(cu_seqlens)
+    nb, nr = ctypes.c_int32(0), ctypes.c_int32(0)
+    L = lib()
+    _check(L.cbv_plan_zigzag(_p32(cu), len(cu) - 1, cp, _layout(layout), None, 0, ctypes.byref(nb), None, 0,
+                             ctypes.byref(nr)))
+    blocks = (RingBlock * max(nb.value, 1))()
+    runs = (RowRun * max(nr.value, 1))()
+    _check(L.cbv_plan_zigzag(_p32(cu), len(cu) - 1, cp, _layout(layout), blocks, nb.value, ctypes.byref(nb), runs,
+                             nr.value, ctypes.byref(nr)))
+    out = []
+    for b in blocks[: nb.value]:
+        d = {f: getattr(b, f) for f, _ in RingBlock._fields_}
+        d["q_runs"] = [(x.doc, x.row0, x.rows, x.pos0, x.local0) for x in runs[b.q_run0: b.q_run0 + b.q_nruns]]
+        d["k_runs"] = [(x.doc, x.row0, x.rows, x.pos0, x.local0) for x in runs[b.k_run0: b.k_run0 + b.k_nruns]]
+        out.append(d)
+    return out
 
 
 # ----------------------------------------------------------------------------- attention calls

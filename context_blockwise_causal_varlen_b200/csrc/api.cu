@@ -344,6 +344,33 @@ int cbv_ring_step(int32_t rank, int32_t step, int32_t cp, int32_t layout, int32_
   return CBV_OK;
 }
 
+int cbv_plan_zigzag(const int32_t* cu, int32_t num_docs, int32_t cp, int32_t layout, cbv_ring_block* blocks,
+                    int32_t max_blocks, int32_t* num_blocks_out, cbv_row_run* runs, int32_t max_runs,
+                    int32_t* num_runs_out) {
+  if (!num_blocks_out || !num_runs_out) return fail(CBV_ERR_BAD_ARG, "NULL count");
+  if (layout != CBV_LAYOUT_ZIGZAG && layout != CBV_LAYOUT_CONTIGUOUS) return fail(CBV_ERR_BAD_ARG, "bad layout");
+  std::string e = check_cu_seqlens(cu, num_docs);
+  if (!e.empty()) return fail(CBV_ERR_BAD_CU_SEQLENS, "%s", e.c_str());
+  e = check_divisible(cu, num_docs, cp, (Layout)layout);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  std::vector<RingBlock> bl;
+  std::vector<RowRun> rr;
+  ring_blocks(cu, num_docs, cp, (Layout)layout, &bl, &rr);
+  *num_blocks_out = (int32_t)bl.size();
+  *num_runs_out = (int32_t)rr.size();
+  if (!blocks || !runs) return CBV_OK;
+  if (max_blocks < (int32_t)bl.size() || max_runs < (int32_t)rr.size())
+    return fail(CBV_ERR_BAD_ARG, "capacity too small: %zu blocks and %zu runs", bl.size(), rr.size());
+  static_assert(sizeof(cbv_ring_block) == sizeof(RingBlock) && sizeof(cbv_row_run) == sizeof(RowRun), "layouts");
+  for (size_t i = 0; i < bl.size(); ++i) {
+    const RingBlock& b = bl[i];
+    blocks[i] = cbv_ring_block{b.rank, b.step, b.src, b.kind, b.causal, b.q_half, b.k_half,
+                               b.q_run0, b.q_nruns, b.k_run0, b.k_nruns};
+  }
+  for (size_t i = 0; i < rr.size(); ++i) runs[i] = cbv_row_run{rr[i].doc, rr[i].row0, rr[i].rows, rr[i].pos0, rr[i].local0};
+  return CBV_OK;
+}
+
 // ------------------------------------------------------------------------ block forward
 static int block_fwd_checks(const cbv_block_fwd_args* a) {
   if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");

@@ -198,6 +198,58 @@ void ring_step(int32_t rank, int32_t step, int32_t cp, Layout layout, int32_t* s
   }
 }
 
+void ring_blocks(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, std::vector<RingBlock>* blocks,
+                 std::vector<RowRun>* runs) {
+  blocks->clear();
+  runs->clear();
+  const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+  // the run of chunk x of document d, which is local chunk `part` (0 front, 1 back) of its rank
+  auto chunk_run = [&](int32_t d, int32_t x, int32_t part) {
+    const int32_t c = (cu[d + 1] - cu[d]) / nchunk;
+    const int32_t row0 = cu[d] + x * c;
+    runs->push_back({d, row0, c, row0, cu[d] / cp + part * c});
+  };
+  for (int32_t r = 0; r < cp; ++r) {
+    for (int32_t s = 0; s < cp; ++s) {
+      int32_t src, kind;
+      ring_step(r, s, cp, layout, &src, &kind);
+      if (kind == kSkip) continue;
+      RingBlock b{};
+      b.rank = r;
+      b.step = s;
+      b.src = src;
+      b.kind = kind;
+      b.causal = kind == kDiag;
+      b.q_half = kind == kBackQ ? 2 : 0;
+      b.k_half = kind == kFrontK ? 1 : 0;
+      // q runs: rank r's local rows (or back halves); k runs: src's local rows (or front halves)
+      b.q_run0 = (int32_t)runs->size();
+      for (int32_t d = 0; d < num_docs; ++d) {
+        if (cu[d + 1] == cu[d]) continue;
+        if (layout == kContiguous) {
+          chunk_run(d, r, 0);
+          continue;
+        }
+        if (b.q_half != 2) chunk_run(d, r, 0);
+        chunk_run(d, 2 * cp - 1 - r, 1);
+      }
+      b.q_nruns = (int32_t)runs->size() - b.q_run0;
+      b.k_run0 = (int32_t)runs->size();
+      for (int32_t d = 0; d < num_docs; ++d) {
+        if (cu[d + 1] == cu[d]) continue;
+        if (layout == kContiguous) {
+          chunk_run(d, src, 0);
+          continue;
+        }
+        chunk_run(d, src, 0);
+        if (b.k_half != 1) chunk_run(d, 2 * cp - 1 - src, 1);
+      }
+      b.k_nruns = (int32_t)runs->size() - b.k_run0;
+      blocks->push_back(b);
+    }
+  }
+}
+
 std::vector<ChunkPair> ring_chunk_pairs(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout,
                                         int32_t window, int32_t only_step) {
   std::vector<ChunkPair> out;

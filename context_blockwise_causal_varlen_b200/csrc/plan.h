@@ -64,6 +64,21 @@ void rank_pair_counts(const int32_t* cu, int32_t num_docs, int32_t cp, Layout la
 enum BlockKind : int32_t { kDiag = 0, kFrontK = 1, kBackQ = 2, kFull = 3, kSkip = 4 };
 void ring_step(int32_t rank, int32_t step, int32_t cp, Layout layout, int32_t* src, int32_t* kind);
 
+// The blocks of the ring as the pages run them: rank r's flash call at step s, with its q
+// rows (all local rows, or the back halves), the k rows of src (all of src's local rows, or
+// its front halves), the cu_seqlens each side uses (local G/cp or halved G/(2cp)) and the
+// causal flag.  Rows are listed as runs of consecutive global rows, document by document in
+// local order (front chunk before back chunk).
+struct RowRun {
+  int32_t doc, row0, rows, pos0, local0;
+};
+struct RingBlock {
+  int32_t rank, step, src, kind, causal, q_half, k_half;
+  int32_t q_run0, q_nruns, k_run0, k_nruns;
+};
+void ring_blocks(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, std::vector<RingBlock>* blocks,
+                 std::vector<RowRun>* runs);
+
 // A pair of chunks of one document that meet in a block: q chunk x against k chunk y.
 struct ChunkPair {
   int32_t doc, rank, step, q_chunk, k_chunk, causal;

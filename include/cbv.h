@@ -132,6 +132,46 @@ int cbv_rank_pair_counts(const int32_t* cu_global, int32_t num_docs, int32_t cp,
    step <= rank), 4 skip (contiguous, step > rank). */
 int cbv_ring_step(int32_t rank, int32_t step, int32_t cp, int32_t layout, int32_t* src_out, int32_t* kind_out);
 
+/* The per-step block descriptors of the whole ring: one cbv_ring_block per (rank, step) that
+ * runs a block (rank-major, steps in order; the contiguous layout's skipped steps are left out),
+ * each the flash call of zigzag_ring_attention._block_forward / _block_backward (contiguous:
+ * ring_attention.ring_flash_attn_forward):
+ *   - step 0 (kind 0): every local q row against every local k row, causal, both sides with
+ *     the local cu_seqlens (G / cp);
+ *   - src < rank (kind 1): every local q row (local cu) against src's FRONT halves, whose
+ *     cu_seqlens are the halved ones (G / (2 cp)), not causal;
+ *   - src > rank (kind 2): the local BACK halves (halved cu; get_half_index / get_half_lse with
+ *     front = 0 select them) against every local k row of src (local cu), not causal;
+ *   - contiguous, 0 < step <= rank (kind 3): every local row against src's, not causal.
+ * The rows of a side are runs of consecutive GLOBAL rows (natural packed order), document by
+ * document in local order (a document's front chunk before its back chunk); a run's `local0`
+ * is the index of its first row in its rank's local sequence (rank for q, src for k), and
+ * `pos0` the position of its first row: positions are global rows, so pos0 == row0.  Empty
+ * documents contribute no run.
+ * Sizes: call with blocks == NULL or runs == NULL to get the counts only.  With arrays,
+ * max_blocks / max_runs are their capacities; too small -> CBV_ERR_BAD_ARG (counts still set).
+ * Errors: as the other planner calls.  (The sliding window does not change the blocks: the
+ * flash call masks by position.) */
+typedef struct cbv_row_run {
+  int32_t doc;
+  int32_t row0;   /* first global row */
+  int32_t rows;
+  int32_t pos0;   /* position of row0 (== row0) */
+  int32_t local0; /* index of row0 in the rank's local sequence */
+} cbv_row_run;
+typedef struct cbv_ring_block {
+  int32_t rank, step, src;
+  int32_t kind;    /* as cbv_ring_step */
+  int32_t causal;  /* 1 only for the step-0 block */
+  int32_t q_half;  /* 0: every local q row, cu_seqlens_q = G / cp; 2: back halves, cu_seqlens_q = G / (2 cp) */
+  int32_t k_half;  /* 0: every local k row of src, cu_seqlens_k = G / cp; 1: front halves, cu_seqlens_k = G / (2 cp) */
+  int32_t q_run0, q_nruns;  /* this block's q rows: runs[q_run0 .. q_run0 + q_nruns) */
+  int32_t k_run0, k_nruns;  /* its k rows (of src) */
+} cbv_ring_block;
+int cbv_plan_zigzag(const int32_t* cu_global, int32_t num_docs, int32_t cp, int32_t layout, cbv_ring_block* blocks,
+                    int32_t max_blocks, int32_t* num_blocks_out, cbv_row_run* runs, int32_t max_runs,
+                    int32_t* num_runs_out);
+
 /* ========================================================================= block forward
  * One flash varlen block (zigzag_ring_attention._block_forward; ring_attention._fa_forward:
  * returns (out[B,S,H,D], lse[B,H,S])).  Documents pair q rows [cu_q[d], cu_q[d+1]) with k

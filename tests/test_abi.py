@@ -12,6 +12,7 @@ import pytest
 
 import context_blockwise_causal_varlen_b200 as cbv
 from oracle import planner as P
+from oracle.ring import _block_rows
 from synth import cu_from_lengths, packed_doc_lengths, streams
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -32,7 +33,8 @@ def test_library_exports_every_declared_symbol():
 def test_struct_layouts_match_the_c_compiler():
     structs = {"cbv_block_fwd_args": cbv.BlockFwdArgs, "cbv_ring_args": cbv.RingArgs,
                "cbv_block_bwd_args": cbv.BlockBwdArgs, "cbv_kvp_args": cbv.KvpArgs, "cbv_decode_args": cbv.DecodeArgs,
-               "cbv_cached_ring_args": cbv.CachedRingArgs}
+               "cbv_cached_ring_args": cbv.CachedRingArgs, "cbv_ring_block": cbv.RingBlock,
+               "cbv_row_run": cbv.RowRun}
     src = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
     for cname, st in structs.items():
         src.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
@@ -103,6 +105,76 @@ def test_planner_on_the_packed_workload_and_long_doc():
     assert ct[0] == 33558528 and ct[-1] == 503320576
     w = cbv.rank_pair_counts(cu, 8, cbv.ZIGZAG, 4096)
     assert w.sum() == 260048896 == P.rank_pair_counts(cu, 8, P.ZIGZAG, 4096).sum()
+
+
+def _expand(runs, field):
+    """The rows of a list of runs, concatenated in order (field: 1 = global row, 4 = local index)."""
+    parts = [np.arange(r[field], r[field] + r[2]) for r in runs]
+    return np.concatenate(parts).astype(np.int64) if parts else np.zeros(0, np.int64)
+
+
+def _check_block_descriptors(cu, cp):
+    """cbv_plan_zigzag against the oracle's per-(rank, step) blocks, element by element."""
+    cu = np.asarray(cu, np.int32)
+    for layout, name in ((cbv.ZIGZAG, P.ZIGZAG), (cbv.CONTIGUOUS, P.CONTIGUOUS)):
+        div = 2 * cp if layout == cbv.ZIGZAG else cp
+        if np.any(np.diff(cu) % div):
+            with pytest.raises(cbv.CbvError) as e:
+                cbv.plan_zigzag(cu, cp, layout)
+            assert e.value.status == "NOT_DIVISIBLE_2CP"
+            continue
+        blocks = cbv.plan_zigzag(cu, cp, layout)
+        want = [(r, s) for r in range(cp) for s in range(cp) if _block_rows(cu, cp, r, s, name) is not None]
+        assert [(b["rank"], b["step"]) for b in blocks] == want
+        cu_loc, cu_half = P.local_cu_seqlens(cu, cp), P.half_cu_seqlens(cu, cp)
+        for b in blocks:
+            r, s = b["rank"], b["step"]
+            qi, kj, causal, cu_q, cu_k, src = _block_rows(cu, cp, r, s, name)
+            assert b["src"] == src and b["causal"] == int(causal)
+            # local rows (the flash call's q and k index sets) and their global rows
+            assert np.array_equal(_expand(b["q_runs"], 4), qi)
+            assert np.array_equal(_expand(b["k_runs"], 4), kj)
+            assert np.array_equal(_expand(b["q_runs"], 1), P.rank_tokens(cu, cp, r, name)[qi])
+            assert np.array_equal(_expand(b["k_runs"], 1), P.rank_tokens(cu, cp, src, name)[kj])
+            # positions are global rows; runs are documents' chunks in local order
+            for run in b["q_runs"] + b["k_runs"]:
+                d, row0, rows, pos0, _ = run
+                assert pos0 == row0 and cu[d] <= row0 and row0 + rows <= cu[d + 1]
+            # the cu_seqlens the block's flash call uses on each side
+            assert np.array_equal(cu_half if b["q_half"] == 2 else cu_loc, cu_q)
+            assert np.array_equal(cu_half if b["k_half"] == 1 else cu_loc, cu_k)
+            names = {0: "diag", 1: "front_k", 2: "back_q", 3: "full"}
+            step = P.zigzag_step if layout == cbv.ZIGZAG else P.contiguous_step
+            assert names[b["kind"]] == step(r, s, cp)[1]
+
+
+@pytest.mark.parametrize("cu", CUS)
+@pytest.mark.parametrize("cp", [1, 2, 4, 8])
+def test_block_descriptors_match_the_oracle_blocks(cu, cp):
+    _check_block_descriptors(cu, cp)
+
+
+def test_block_descriptors_of_the_tiny_and_packed_workloads():
+    _check_block_descriptors([0, 96, 256], 2)
+    for seed in range(3):
+        cu = cu_from_lengths(packed_doc_lengths(streams(seed, 6)[4], 16384, 512, 4096, 8))
+        _check_block_descriptors(cu, 4)
+    _check_block_descriptors([0, 16 * 40, 16 * 41], 8)
+
+
+def test_block_descriptor_capacity_errors():
+    cu = np.array([0, 96, 256], np.int32)
+    nb, nr = ctypes.c_int32(0), ctypes.c_int32(0)
+    L = cbv.lib()
+    assert L.cbv_plan_zigzag(cu.ctypes.data_as(cbv.c_i32p), 2, 2, 0, None, 0, ctypes.byref(nb), None, 0,
+                             ctypes.byref(nr)) == 0
+    # two documents, two chunks each per rank: the diagonals 4 q + 4 k runs, back-q 2 + 4, front-k 4 + 2
+    assert (nb.value, nr.value) == (4, 8 + 6 + 8 + 6)
+    blocks = (cbv.RingBlock * nb.value)()
+    runs = (cbv.RowRun * (nr.value - 1))()
+    rc = L.cbv_plan_zigzag(cu.ctypes.data_as(cbv.c_i32p), 2, 2, 0, blocks, nb.value, ctypes.byref(nb), runs,
+                           nr.value - 1, ctypes.byref(nr))
+    assert cbv.STATUS[rc] == "BAD_ARG"
 
 
 def _ring_args(**kw):
