@@ -167,7 +167,8 @@ EXPORTS = [
     "cbv_zigzag_ring_fwd_workspace_size", "cbv_zigzag_ring_fwd", "cbv_zigzag_ring_bwd_workspace_size",
     "cbv_zigzag_ring_bwd", "cbv_block_bwd_workspace_size", "cbv_attn_block_bwd",
     "cbv_kvp_workspace_size", "cbv_kvp_segmented_prefill", "cbv_decode_workspace_size", "cbv_varlen_decode",
-    "cbv_noalloc_scratch_bytes", "cbv_zigzag_ring_fwd_noalloc",
+    "cbv_noalloc_scratch_bytes", "cbv_zigzag_ring_fwd_noalloc", "cbv_noalloc_read_status",
+    "cbv_debug_ring_fwd_stalled",
     "cbv_cached_ring_fwd_workspace_size", "cbv_cached_ring_fwd", "cbv_cached_ring_bwd_workspace_size",
     "cbv_cached_ring_bwd",
 ]
@@ -200,6 +201,8 @@ def _declare(L):
         getattr(L, name).argtypes = [ctypes.POINTER(st), ctypes.c_void_p]
     L.cbv_noalloc_scratch_bytes.restype = ctypes.c_size_t
     L.cbv_zigzag_ring_fwd_noalloc.argtypes = [ctypes.POINTER(RingArgs), ctypes.c_void_p]
+    L.cbv_noalloc_read_status.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
+    L.cbv_debug_ring_fwd_stalled.argtypes = [ctypes.POINTER(RingArgs), ctypes.c_uint64, ctypes.c_void_p]
     L.cbv_attn_merge.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
 
@@ -360,8 +363,23 @@ def plan_zigzag(cu_seqlens, cp: int, layout="zigzag") -> list[dict]:
 
 
 # ----------------------------------------------------------------------------- attention calls
+def _given_workspace(ws, nbytes: int, device):
+    """A caller-given uint8 workspace of at least ``nbytes`` (else one is allocated).  ``ws`` may also be
+    a callable that takes the byte count and returns such a tensor."""
+    if ws is None:
+        return _workspace(nbytes, device)
+    if callable(ws):
+        ws = ws(max(int(nbytes), 256))
+    if not (isinstance(ws, torch.Tensor) and ws.is_cuda and ws.dtype == torch.uint8 and ws.is_contiguous()):
+        raise CbvError(-1, "workspace must be a contiguous uint8 CUDA tensor")
+    if ws.numel() < nbytes or ws.data_ptr() % 256:
+        raise CbvError(-11, f"workspace needs {nbytes} bytes, 256-byte aligned")
+    return ws
+
+
 def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
-                    schedule: int = SCHEDULE_FUSED, max_seqlen: int = 0, out=None, lse=None, return_workspace=False):
+                    schedule: int = SCHEDULE_FUSED, max_seqlen: int = 0, out=None, lse=None, return_workspace=False,
+                    workspace=None):
     """Ring forward over ``cp`` virtual ranks: ``(out [S,H,D] bf16, lse [H,S] f32)``."""
     q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
     S, H, D = q.shape
@@ -376,14 +394,15 @@ def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, l
                  head_dim=D, num_docs=len(cu) - 1, cu_seqlens=_p32(cu), max_seqlen=max_seqlen, cp=cp,
                  layout=_layout(layout), scale=_scale(scale), causal=1, window=int(window), schedule=int(schedule),
                  out=_ptr(out), lse=_ptr(lse))
-    ws = _workspace(lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
+    ws = _given_workspace(workspace, lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_zigzag_ring_fwd(ctypes.byref(a), _stream(q.device)))
     return (out, lse, ws) if return_workspace else (out, lse)
 
 
 def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, window: int = 0, layout="zigzag",
-                    max_seqlen: int = 0, dq=None, dk=None, dv=None, return_workspace=False, deterministic=False):
+                    max_seqlen: int = 0, dq=None, dk=None, dv=None, return_workspace=False, deterministic=False,
+                    workspace=None):
     """Ring backward fed the merged out/lse: ``(dq, dk, dv)`` bf16.  ``deterministic``: dq summed in
     64-bit fixed point, bit-identical from run to run."""
     dout, q, k, v, out = (_bf16(t, n) for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
@@ -405,7 +424,7 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
                  layout=_layout(layout), scale=_scale(scale), causal=1, window=int(window), schedule=0,
                  deterministic=int(bool(deterministic)), out=_ptr(out), lse=_ptr(lse.contiguous()), dout=_ptr(dout),
                  dq=_ptr(dq), dk=_ptr(dk), dv=_ptr(dv))
-    ws = _workspace(lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
+    ws = _given_workspace(workspace, lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_zigzag_ring_bwd(ctypes.byref(a), _stream(q.device)))
     return (dq, dk, dv, ws) if return_workspace else (dq, dk, dv)
@@ -585,7 +604,8 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
 
 def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_ROBIN, seg_size: int = 512,
                           scale=None, global_q_offset: int = 0, sliding_window: int = 0, per_shard: bool = False,
-                          return_lse: bool = True, tp_out: bool = False):
+                          return_lse: bool = True, tp_out: bool = False, out=None, lse=None, shard_out=None,
+                          shard_lse=None, workspace=None):
     """Paged KV-parallel prefill; q ``[HQ, S, D]`` -> ``out [HQ, S, D]`` (``[HQ, D, S]`` with ``tp_out``)
     (+ lse, + per-shard partials)."""
     if not q.is_cuda or q.dtype != torch.bfloat16:
@@ -597,10 +617,18 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
     _shape(v_cache, k_cache.shape, "v_cache")
     bt = block_tables.to(device=q.device, dtype=torch.int32).contiguous()
     R, bps = bt.shape
-    out = torch.empty((HQ, D, S) if tp_out else (HQ, S, D), dtype=torch.bfloat16, device=q.device)
-    lse = torch.empty((HQ, S), dtype=torch.float32, device=q.device) if return_lse else None
-    so = torch.empty((R, HQ, S, D), dtype=torch.float32, device=q.device) if per_shard else None
-    sl = torch.empty((R, HQ, S), dtype=torch.float32, device=q.device) if per_shard else None
+    oshape = (HQ, D, S) if tp_out else (HQ, S, D)
+    out = _given(out, oshape, torch.bfloat16, q.device, "out")
+    out = torch.empty(oshape, dtype=torch.bfloat16, device=q.device) if out is None else out
+    lse = _given(lse, (HQ, S), torch.float32, q.device, "lse") if return_lse else None
+    if return_lse and lse is None:
+        lse = torch.empty((HQ, S), dtype=torch.float32, device=q.device)
+    so = sl = None
+    if per_shard:
+        so = _given(shard_out, (R, HQ, S, D), torch.float32, q.device, "shard_out")
+        sl = _given(shard_lse, (R, HQ, S), torch.float32, q.device, "shard_lse")
+        so = torch.empty((R, HQ, S, D), dtype=torch.float32, device=q.device) if so is None else so
+        sl = torch.empty((R, HQ, S), dtype=torch.float32, device=q.device) if sl is None else sl
     a = KvpArgs(**_header(KvpArgs), q=_ptr(q), q_stride_head=q.stride(0), q_stride_token=q.stride(1), q_len=S,
                 num_heads=HQ, num_kv_heads=HKV, head_dim=D, k_cache=_ptr(k_cache), v_cache=_ptr(v_cache),
                 num_blocks=nb, block_size=bs, block_tables=_ptr(bt), shards=R, blocks_per_shard=bps,
@@ -610,7 +638,7 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
                 lse=_ptr(lse), shard_out=_ptr(so), shard_lse=_ptr(sl))
     if q.stride(2) != 1:
         raise CbvError(-4, "q's last dimension must be contiguous")
-    ws = _workspace(lib().cbv_kvp_workspace_size(ctypes.byref(a)), q.device)
+    ws = _given_workspace(workspace, lib().cbv_kvp_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_kvp_segmented_prefill(ctypes.byref(a), _stream(q.device)))
     res = [out]

@@ -1,6 +1,7 @@
 // The C ABI of libcbv.so (include/cbv.h): argument checks, workspace layout,
 // tensor-map encoding and the launch sequence of every call.
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -11,6 +12,7 @@
 #include <vector>
 
 #include "../../include/cbv.h"
+#include "api_internal.h"
 #include "kernels.h"
 #include "plan.h"
 #include "ptx.cuh"
@@ -20,6 +22,14 @@ using namespace cbv;
 namespace {
 
 thread_local std::string g_err;
+
+// An NVTX range around one call (visible to a profiler; close to free without one attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -180,12 +190,6 @@ int grid_of(size_t tasks, int heads) {
 }
 
 // ------------------------------------------------------------------------ ring forward
-struct RingFwdLayout {
-  Plan fused;
-  std::vector<Plan> steps;
-  size_t bytes = 0;
-};
-
 int ring_common_checks(const cbv_ring_args* a) {
   if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
   int rc = check_header(a->struct_size, sizeof(cbv_ring_args), a->abi_version);
@@ -248,7 +252,6 @@ FwdParams ring_fwd_params(const cbv_ring_args* a, int* rc) {
 }  // namespace
 
 namespace cbv {
-// Sets the text cbv_last_error_message() returns (for entry points in other files).
 void set_last_error(const char* msg) { g_err = msg; }
 }  // namespace cbv
 
@@ -397,6 +400,7 @@ size_t cbv_block_fwd_workspace_size(const cbv_block_fwd_args* a) {
 }
 
 int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_attn_block_fwd");
   int rc = block_fwd_checks(a);
   if (rc) return rc;
   if (a->total_q == 0) return CBV_OK;  // no query rows: nothing to write
@@ -445,6 +449,7 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
 // ------------------------------------------------------------------------ merge
 int cbv_attn_merge(float* out, float* lse, const void* block_out, int32_t block_out_dtype, const float* block_lse,
                    float* weight_out, int64_t seqlen, int32_t num_heads, int32_t head_dim, void* stream) {
+  NvtxRange nvtx_range("cbv_attn_merge");
   if (head_dim != 64 && head_dim != 128) return fail(CBV_ERR_UNSUPPORTED_HEAD_DIM, "head_dim %d", head_dim);
   if (seqlen < 0 || num_heads <= 0) return fail(CBV_ERR_BAD_SHAPE, "bad shape");
   if (seqlen == 0) return CBV_OK;
@@ -462,21 +467,51 @@ size_t cbv_zigzag_ring_fwd_workspace_size(const cbv_ring_args* a) {
   return ring_fwd_layout(a).bytes;
 }
 
-int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
-  int rc = ring_common_checks(a);
-  if (rc) return rc;
-  if (a->total == 0) return CBV_OK;  // no rows: nothing to write
-  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
-    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  RingFwdLayout L = ring_fwd_layout(a);
+int cbv_debug_ring_fwd_stalled(const cbv_ring_args* a, uint64_t wait_limit_ns, void* stream) {
+  NvtxRange nvtx_range("cbv_debug_ring_fwd_stalled");
+  if (wait_limit_ns < 100000ull || wait_limit_ns > 1000000000ull)
+    return fail(CBV_ERR_BAD_ARG, "wait_limit_ns must be in [1e5, 1e9]");
+  if (a && a->schedule != CBV_SCHEDULE_FUSED) return fail(CBV_ERR_BAD_ARG, "the fused schedule only");
+  RingFwdLayout L;
+  int rc = cbv::ring_fwd_plan(a, &L);
+  if (rc || a->total == 0) return rc;
   if (!a->workspace || a->workspace_bytes < L.bytes)
     return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", L.bytes);
-  Carve c(a->workspace);
+  return cbv::ring_fwd_run(a, L, a->workspace, static_cast<cudaStream_t>(stream), wait_limit_ns, 1);
+}
+
+int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_zigzag_ring_fwd");
+  RingFwdLayout L;
+  int rc = cbv::ring_fwd_plan(a, &L);
+  if (rc || a->total == 0) return rc;  // no rows: nothing to write
+  if (!a->workspace || a->workspace_bytes < L.bytes)
+    return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", L.bytes);
+  return cbv::ring_fwd_run(a, L, a->workspace, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+int cbv::ring_fwd_plan(const cbv_ring_args* a, RingFwdLayout* L) {
+  int rc = ring_common_checks(a);
+  if (rc) return rc;
+  if (a->total == 0) return CBV_OK;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  *L = ring_fwd_layout(a);
+  return CBV_OK;
+}
+
+int cbv::ring_fwd_run(const cbv_ring_args* a, const RingFwdLayout& L, void* workspace, cudaStream_t s,
+                      uint64_t wait_limit_ns, int withhold_loads) {
+  int rc;
+  Carve c(workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
   FwdParams p = ring_fwd_params(a, &rc);
   if (rc) return rc;
   p.status = status;
+  p.wait_limit_ns = wait_limit_ns;
+  p.withhold_loads = withhold_loads;
   if ((rc = zero_status(status, s))) return rc;
   const int D = a->head_dim, H = a->num_heads;
   if (a->schedule == CBV_SCHEDULE_FUSED) {
@@ -496,6 +531,9 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
   }
   float* acc = static_cast<float*>(c.take((size_t)a->total * H * D * sizeof(float)));
   for (int st = 0; st < a->cp; ++st) {
+    char name[48];
+    snprintf(name, sizeof name, "ring step %d", st);
+    NvtxRange step_range(name);
     p.tasks = pds[st].tasks;
     p.segs = pds[st].segs;
     p.num_tasks = (int)L.steps[st].tasks.size();
@@ -506,6 +544,8 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream) {
   }
   return launch_rc(launch_convert_bf16(acc, a->out, a->total * H * D, 1.f, s), "output conversion");
 }
+
+extern "C" {
 
 // ------------------------------------------------------------------------ paged KV-parallel prefill
 static int kvp_checks(const cbv_kvp_args* a) {
@@ -575,6 +615,7 @@ size_t cbv_kvp_workspace_size(const cbv_kvp_args* a) {
 }
 
 int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_kvp_segmented_prefill");
   int rc = kvp_checks(a);
   if (rc) return rc;
   if (a->q_len == 0) return CBV_OK;  // no query rows: nothing to write
@@ -678,6 +719,7 @@ size_t cbv_decode_workspace_size(const cbv_decode_args* a) {
 }
 
 int cbv_varlen_decode(const cbv_decode_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_varlen_decode");
   if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
   int rc = check_header(a->struct_size, sizeof(cbv_decode_args), a->abi_version);
   if (rc) return rc;
@@ -838,6 +880,7 @@ static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_
 }
 
 int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_zigzag_ring_bwd");
   int rc = ring_common_checks(a);
   if (rc) return rc;
   if (a->total == 0) return CBV_OK;  // no rows: nothing to write
@@ -882,6 +925,7 @@ size_t cbv_block_bwd_workspace_size(const cbv_block_bwd_args* a) {
 }
 
 int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_attn_block_bwd");
   int rc = block_bwd_checks(a);
   if (rc) return rc;
   if (a->total_q == 0 || a->total_k == 0) return CBV_OK;  // no (q, k) pair: the accumulators are unchanged
@@ -997,8 +1041,8 @@ int cached_blocks(const cbv_cached_ring_args* a, bool grads, cbv::CacheBlocks* c
   return CBV_OK;
 }
 
-size_t cached_fwd_bytes(const cbv_cached_ring_args* a, const cbv_ring_args& r) {
-  size_t b = ring_fwd_layout(&r).bytes;
+size_t cached_fwd_bytes(const cbv_cached_ring_args* a, const RingFwdLayout& L) {
+  size_t b = L.bytes;
   if (a->num_blocks > 1) b = (b + 255) / 256 * 256 + (size_t)a->total * a->num_heads * a->head_dim * sizeof(float);
   return b;
 }
@@ -1010,10 +1054,11 @@ extern "C" {
 size_t cbv_cached_ring_fwd_workspace_size(const cbv_cached_ring_args* a) {
   if (cached_checks(a)) return 0;
   cbv_ring_args r = cached_block0(a);
-  return cached_fwd_bytes(a, r);
+  return cached_fwd_bytes(a, ring_fwd_layout(&r));
 }
 
 int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_cached_ring_fwd");
   int rc = cached_checks(a);
   if (rc) return rc;
   if (a->total == 0) return CBV_OK;
@@ -1023,11 +1068,11 @@ int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream) {
   if (a->num_blocks == 1) return cbv_zigzag_ring_fwd(&r, stream);  // the sequence alone
   if (!a->q || !a->out || !a->lse) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
   if (!aligned16(a->q) || !aligned16(a->out)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
-  const size_t need = cached_fwd_bytes(a, r);
+  RingFwdLayout L = ring_fwd_layout(&r);
+  const size_t need = cached_fwd_bytes(a, L);
   if (!a->workspace || a->workspace_bytes < need) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", need);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int D = a->head_dim, H = a->num_heads;
-  RingFwdLayout L = ring_fwd_layout(&r);
   Carve c(a->workspace);
   int* status = static_cast<int*>(c.take(kStatusBytes));
   PlanDev pd = carve_plan(c, L.fused);
@@ -1056,6 +1101,7 @@ size_t cbv_cached_ring_bwd_workspace_size(const cbv_cached_ring_args* a) {
 }
 
 int cbv_cached_ring_bwd(const cbv_cached_ring_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_cached_ring_bwd");
   int rc = cached_checks(a);
   if (rc) return rc;
   if (a->total == 0) return CBV_OK;

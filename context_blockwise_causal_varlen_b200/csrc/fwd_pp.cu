@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs;
   int tix = (int)blockIdx.x, half = -1;
   if (p.split_halves && tix >= p.split_from) {
     half = (tix - p.split_from) & 1;
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (lane == 0 && !p.withhold_loads) {
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           uint64_t* full = &bar[(kv == 0 ? pKFull : pVFull) + st];
           const CUtensorMap* map = kv == 0 ? &p.tm_k : &p.tm_v;
           uint8_t* dst = (kv == 0 ? sK : sV) + st * L::kTile;
-          if (!mbar_wait(empty, ph ^ 1, p.status, kDevTimeoutTmaEmpty)) {
+          if (!mbar_wait(empty, ph ^ 1, p.status, kDevTimeoutTmaEmpty, lim)) {
             ok = false;
             break;
           }
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         while (next_ktile<PAGED>(p, t, qp0, qp1, c, r)) ++n;
       }
       const int ntile = has_b ? 2 : 1;
-      bool ok = mbar_wait_warp(&bar[pQFull], 0, p.status, kDevTimeoutMma);
+      bool ok = mbar_wait_warp(&bar[pQFull], 0, p.status, kDevTimeoutMma, lim);
       tc_fence_after();
       // S_x of k tile i (K stage i & 1); a split task's two halves both read q tile 0
       auto issue_s = [&](int x, int i) {
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       if (!has_b) {
         // split task: k tile i belongs to half x = i & 1 and always sits in stage i & 1
         for (int i = 0; ok && i < min(n, 2); ++i) {
-          ok = mbar_wait_warp(&bar[pKFull + i], 0, p.status, kDevTimeoutMma);
+          ok = mbar_wait_warp(&bar[pKFull + i], 0, p.status, kDevTimeoutMma, lim);
           tc_fence_after();
           if (ok) {
             issue_s(i, i);
@@ -284,22 +285,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         for (int i = 0; ok && i < n; ++i) {
           const int x = i & 1;
           const uint32_t ph = (i >> 1) & 1;  // half x's own tile count, and stage x's load count
-          if (!mbar_wait_warp(&bar[pVFull + x], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
-          if (!mbar_wait_warp(&bar[pPFull + x], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait_warp(&bar[pVFull + x], ph, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
+          if (!mbar_wait_warp(&bar[pPFull + x], ph, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
           tc_fence_after();
           issue_pv(x, i, i < 2);
           umma_commit(&bar[pVEmpty + x]);
           if (i + 2 < n) {
-            if (!mbar_wait_warp(&bar[pKFull + x], ph ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait_warp(&bar[pKFull + x], ph ^ 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
             // P_x lives in the columns S_x of tile i + 2 will overwrite
-            if (!mbar_wait_warp(&bar[pPVDone + x], ph, p.status, kDevTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait_warp(&bar[pPVDone + x], ph, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
             tc_fence_after();
             issue_s(x, i + 2);
             umma_commit(&bar[pKEmpty + x]);
           }
         }
       } else if (ok && n > 0) {
-        ok = mbar_wait_warp(&bar[pKFull], 0, p.status, kDevTimeoutMma);
+        ok = mbar_wait_warp(&bar[pKFull], 0, p.status, kDevTimeoutMma, lim);
         tc_fence_after();
         if (ok) {
           for (int x = 0; x < ntile; ++x) issue_s(x, 0);
@@ -308,16 +309,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       }
       for (int i = 0; ok && has_b && i < n; ++i) {
         const int st = i & 1;
-        if (!mbar_wait_warp(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
         for (int x = 0; x < ntile && ok; ++x) {
-          if (!mbar_wait_warp(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait_warp(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
           tc_fence_after();
           issue_pv(x, i, i == 0);
           if (i + 1 < n) {
             const int st1 = (i + 1) & 1;
-            if (!mbar_wait_warp(&bar[pKFull + st1], ((i + 1) >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait_warp(&bar[pKFull + st1], ((i + 1) >> 1) & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
             // P_x(i) lives in the columns S_x(i+1) will overwrite: let PV_x(i) finish reading it first
-            if (!mbar_wait_warp(&bar[pPVDone + x], i & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
+            if (!mbar_wait_warp(&bar[pPVDone + x], i & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
             tc_fence_after();
             issue_s(x, i + 1);
             if (x == ntile - 1) umma_commit(&bar[pKEmpty + st1]);
@@ -351,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       int kidx = 0;
       while (next_ktile<PAGED>(p, t, qp0, qp1, it, r)) {
         if (split && ((kidx++ & 1) != x)) continue;  // the other half's k tile
-        if (!mbar_wait_warp(&bar[pSFull + x], i & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+        if (!mbar_wait_warp(&bar[pSFull + x], i & 1, p.status, kDevTimeoutSoftmax, lim)) { ok = false; break; }
         tc_fence_after();
         uint32_t s[BN];
 #pragma unroll
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         lr = lr * alpha + rowsum_r;
         m = m_use;
         // PV of the previous k tile must be done: O is rescaled and P overwrites its input
-        if (i > 0 && !mbar_wait_warp(&bar[pPVDone + x], (i - 1) & 1, p.status, kDevTimeoutSoftmax)) { ok = false; break; }
+        if (i > 0 && !mbar_wait_warp(&bar[pPVDone + x], (i - 1) & 1, p.status, kDevTimeoutSoftmax, lim)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         m = mm;
       }
     }
-    if (ok && (x == 0 || has_b) && mbar_wait_warp(&bar[pODone], 0, p.status, kDevTimeoutEpilogue)) {
+    if (ok && (x == 0 || has_b) && mbar_wait_warp(&bar[pODone], 0, p.status, kDevTimeoutEpilogue, lim)) {
       tc_fence_after();
       const bool has = (l > 0.f) && (m != -INFINITY);
       const float inv_l = (has && lr > 0.f) ? 1.f / lr : 0.f;

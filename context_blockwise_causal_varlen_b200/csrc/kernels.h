@@ -51,6 +51,11 @@ struct FwdParams {
   const int32_t* block_tables;  // [shards, blocks_per_shard]
   int32_t blocks_per_shard, block_size, shards, kv_mode, n_local;
   int* status;  // device status word (0 = ok)
+  // diagnostics: every wait gives up after wait_limit_ns (0 = the default limit); with
+  // withhold_loads the producer issues no copy at all, so every wait runs out (the test of the
+  // timeout path: no copy or tensor-core operation is ever in flight when the kernel gives up)
+  uint64_t wait_limit_ns;
+  int32_t withhold_loads;
 };
 
 struct BwdParams {

@@ -11,22 +11,13 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
-#include "../../include/cbv.h"
-
-namespace cbv {
-void set_last_error(const char* msg);
-}
+#include "api_internal.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = (size_t)1 << 20;  // 1 MiB: status word + tile schedule
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
 
 thread_local char g_msg[256];
 
@@ -35,29 +26,18 @@ int fail(int code) {
   return code;
 }
 
-// Device address of g_scratch on the current device; looked up once per device.
+// Device address of g_scratch in the current device's context.  Looked up on every call (the
+// lookup allocates nothing), so a context torn down and created again (cudaDeviceReset) never
+// leaves a stale address behind.  The first lookup on a device loads the library's module
+// into that device's context, which must not happen inside a stream capture.
 int scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    snprintf(g_msg, sizeof g_msg, "cudaGetDevice: %s", cudaGetErrorString(e));
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+  if (e != cudaSuccess || !p) {
+    snprintf(g_msg, sizeof g_msg, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
     return fail(CBV_ERR_CUDA);
   }
-  if (dev < 0 || dev >= kMaxDevices) {
-    snprintf(g_msg, sizeof g_msg, "device %d is beyond the %d devices this library tracks", dev, kMaxDevices);
-    return fail(CBV_ERR_BAD_ARG);
-  }
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess || !p) {
-      snprintf(g_msg, sizeof g_msg, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-      return fail(CBV_ERR_CUDA);
-    }
-    g_addr[dev] = p;
-  }
-  *out = g_addr[dev];
+  *out = p;
   return CBV_OK;
 }
 
@@ -72,22 +52,44 @@ int cbv_zigzag_ring_fwd_noalloc(const cbv_ring_args* a, void* stream) {
     snprintf(g_msg, sizeof g_msg, "args is NULL");
     return fail(CBV_ERR_BAD_ARG);
   }
-  const size_t need = cbv_zigzag_ring_fwd_workspace_size(a);
-  if (need == 0) return cbv_zigzag_ring_fwd(a, stream);  // invalid arguments: same status and message
-  if (need > kScratchBytes) {
+  cbv_ring_args b = *a;
+  b.schedule = CBV_SCHEDULE_FUSED;  // the stepwise schedule's fp32 running output does not fit
+  cbv::RingFwdLayout L;
+  int rc = cbv::ring_fwd_plan(&b, &L);  // argument errors: the status and message of cbv_zigzag_ring_fwd
+  if (rc != CBV_OK || b.total == 0) return rc;
+  if (L.bytes > kScratchBytes) {
     snprintf(g_msg, sizeof g_msg,
              "this problem needs %zu bytes of scratch; the static scratch holds %zu (use cbv_zigzag_ring_fwd "
              "with a caller-provided workspace)",
-             need, kScratchBytes);
+             L.bytes, kScratchBytes);
     return fail(CBV_ERR_WORKSPACE_TOO_SMALL);
   }
   void* scratch = nullptr;
-  int rc = scratch_address(&scratch);
-  if (rc != CBV_OK) return rc;
-  cbv_ring_args b = *a;
+  if ((rc = scratch_address(&scratch)) != CBV_OK) return rc;
   b.workspace = scratch;
   b.workspace_bytes = kScratchBytes;
-  return cbv_zigzag_ring_fwd(&b, stream);
+  return cbv::ring_fwd_run(&b, L, scratch, static_cast<cudaStream_t>(stream));
+}
+
+int cbv_noalloc_read_status(int* status_out, void* stream) {
+  if (!status_out) {
+    snprintf(g_msg, sizeof g_msg, "status_out is NULL");
+    return fail(CBV_ERR_BAD_ARG);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    snprintf(g_msg, sizeof g_msg, "reading the static scratch's status word: %s", cudaGetErrorString(e));
+    return fail(CBV_ERR_CUDA);
+  }
+  *status_out = v;
+  if (v != 0) {
+    snprintf(g_msg, sizeof g_msg, "a kernel gave up a wait (code 0x%x)", v);
+    return fail(CBV_ERR_TIMEOUT);
+  }
+  return CBV_OK;
 }
 
 }  // extern "C"

@@ -71,7 +71,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Returns false if
 // the limit ran out or another thread of the grid already reported an error;
 // the first thread to time out records `code` in *status.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int code) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int code,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -79,7 +80,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*reinterpret_cast<volatile int*>(status) != 0) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       atomicCAS(status, 0, code);
       return false;
     }
@@ -88,14 +89,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
 
 // Warp-uniform variant: all 32 lanes call it together and get the same answer,
 // so a warp never splits around a warp-collective instruction after a timeout.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, int code) {
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, int code,
+                                               uint64_t limit_ns = kWaitLimitNs) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    const bool timed_out = global_timer_ns() - t0 > kWaitLimitNs;
+    const bool timed_out = global_timer_ns() - t0 > limit_ns;
     const bool give_up = timed_out || *reinterpret_cast<volatile int*>(status) != 0;
     if (__any_sync(0xffffffffu, give_up)) {
       if (timed_out && (threadIdx.x & 31) == 0) atomicCAS(status, 0, code);

@@ -429,6 +429,18 @@ typedef struct cbv_decode_args {
 size_t cbv_decode_workspace_size(const cbv_decode_args* a);
 int cbv_varlen_decode(const cbv_decode_args* a, void* stream);
 
+/* ========================================================================= diagnostics
+ * Tests of the failure path, which must fault or hang nothing.  The pages have no counterpart.
+ * cbv_debug_ring_fwd_stalled runs the fused ring forward of cbv_zigzag_ring_fwd with its copy
+ * producer told to issue no loads at all and every wait limited to wait_limit_ns (1e5..1e9 ns)
+ * instead of the usual 2 s.  Every consumer's wait then runs out before any copy or
+ * tensor-core operation is in flight: the first one to give up records its code in the status
+ * word at the start of a->workspace, the others see it and leave, and the kernel ends normally
+ * (out and lse are left unwritten).  cbv_read_status() then returns CBV_ERR_TIMEOUT with the
+ * raw code, and the stream and context remain usable.  Arguments as cbv_zigzag_ring_fwd (fused
+ * schedule only); a limit outside the range -> CBV_ERR_BAD_ARG. */
+int cbv_debug_ring_fwd_stalled(const cbv_ring_args* a, uint64_t wait_limit_ns, void* stream);
+
 /* ========================================================================= ring forward without allocation
  * The pages have no counterpart for this call; it serves callers that cannot allocate.
  * cbv_zigzag_ring_fwd takes its scratch (status word and tile schedule) from a workspace the
@@ -436,22 +448,27 @@ int cbv_varlen_decode(const cbv_decode_args* a, void* stream);
  * allocation-free serving loop with a memory budget fixed at start-up, a runtime that owns all
  * device memory through its own allocator, a plain C host with no device allocator) can use
  * this variant instead: it computes exactly what cbv_zigzag_ring_fwd computes with the fused
- * schedule, but its scratch is a fixed array of cbv_noalloc_scratch_bytes() bytes (1 MiB)
- * compiled into the library, which every GPU that loads the library holds until the process
- * exits.  a->workspace and a->workspace_bytes are ignored; inputs and outputs are still the
- * caller's.  It calls no cudaMalloc, cudaFree or allocating library routine.
- * - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *   with that device current; make that first call before any stream capture.
+ * schedule (a->schedule is ignored: the fused schedule always runs), but its scratch is a fixed
+ * array of cbv_noalloc_scratch_bytes() bytes (1 MiB) compiled into the library, which every GPU
+ * that loads the library holds until the process exits.  a->workspace and a->workspace_bytes
+ * are ignored; inputs and outputs are still the caller's.  It calls no cudaMalloc, cudaFree or
+ * allocating library routine.
+ * - Every call looks up the array's device address (cudaGetSymbolAddress) in the current
+ *   device's context; the first call on a device also loads the library's module into that
+ *   context, so make that first call before any stream capture.
  * - Every call, from any thread or stream, shares the one array, and each call overwrites what
  *   the last one left there: calls that overlap on the GPU race.  Serialise them (one stream,
  *   or events between streams).
- * - A problem whose scratch would exceed the array (cbv_zigzag_ring_fwd_workspace_size()
- *   larger than cbv_noalloc_scratch_bytes(), e.g. the stepwise schedule, which keeps an fp32
- *   running output) returns CBV_ERR_WORKSPACE_TOO_SMALL with a message; nothing is launched.
- * - Argument errors are those of cbv_zigzag_ring_fwd.
- * - cbv_read_status() cannot reach the array; a kernel timeout shows up as wrong output only. */
+ * - A problem whose tile schedule would exceed the array returns CBV_ERR_WORKSPACE_TOO_SMALL
+ *   with a message; nothing is launched.
+ * - Argument errors are those of cbv_zigzag_ring_fwd. */
 size_t cbv_noalloc_scratch_bytes(void);
 int cbv_zigzag_ring_fwd_noalloc(const cbv_ring_args* a, void* stream);
+/* The status word the last cbv_zigzag_ring_fwd_noalloc call on the current device left in the
+   static array (synchronises `stream`, which should be the stream that call used).
+   *status_out receives the raw kernel code (0 = ok); returns CBV_ERR_TIMEOUT if a kernel gave
+   up a wait, CBV_OK otherwise. */
+int cbv_noalloc_read_status(int* status_out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -378,3 +378,15 @@ def test_block_backward_argument_errors(field, value, status):
     setattr(a, field, value)
     rc = cbv.lib().cbv_attn_block_bwd(ctypes.byref(a), None)
     assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
+
+
+def test_stalled_forward_diagnostic_checks_its_limit_before_any_launch():
+    a, cu = _ring_args()
+    L = cbv.lib()
+    n0 = cbv.launch_count()
+    for lim in (0, 99_999, 2_000_000_000):
+        assert cbv.STATUS[L.cbv_debug_ring_fwd_stalled(ctypes.byref(a), lim, None)] == "BAD_ARG"
+    a.schedule = cbv.SCHEDULE_STEPWISE
+    assert cbv.STATUS[L.cbv_debug_ring_fwd_stalled(ctypes.byref(a), 1_000_000, None)] == "BAD_ARG"
+    assert cbv.launch_count() == n0
+

@@ -16,7 +16,7 @@ from oracle import decode as DEC
 from oracle import paged as PG
 from synth import torch_normal_bf16
 from synth.workloads import long_doc, packed_zigzag, paged_prefill, varlen_decode
-from tests.gpu_util import check_lse, check_out, check_rel, host
+from tests.gpu_util import GuardedWorkspaces, check_guards, check_lse, check_out, check_rel, guarded, host
 
 pytestmark = pytest.mark.gpu
 
@@ -31,15 +31,23 @@ def _f64(t):
 
 @pytest.mark.parametrize("schedule", [cbv.SCHEDULE_FUSED, cbv.SCHEDULE_STEPWISE])
 def test_packed_zigzag_full_size(schedule):
+    # every document (documents are independent) for three heads, forward and backward, with
+    # canaries around every output and workspace
     w = packed_zigzag(0)
     cu = w.cu_seqlens
+    S, H, D = w.total, w.heads, w.head_dim
     q, k, v, do = _ring_inputs(w, 0)
-    out, lse = cbv.zigzag_ring_fwd(q, k, v, cu, w.cp, schedule=schedule)
-    dq, dk, dv = cbv.zigzag_ring_bwd(do, q, k, v, out, lse, cu, w.cp)
+    (out, ob), (lse, lb) = guarded((S, H, D), torch.bfloat16), guarded((H, S), torch.float32)
+    (dq, gq), (dk, gk), (dv, gv) = (guarded((S, H, D), torch.bfloat16) for _ in range(3))
+    wss = GuardedWorkspaces()
+    cbv.zigzag_ring_fwd(q, k, v, cu, w.cp, schedule=schedule, out=out, lse=lse, workspace=wss)
+    cbv.zigzag_ring_bwd(do, q, k, v, out, lse, cu, w.cp, dq=dq, dk=dk, dv=dv, workspace=wss)
     torch.cuda.synchronize()
-    scale = w.head_dim ** -0.5
-    lengths = np.diff(cu)
-    for d in (int(np.argmin(lengths)), len(lengths) - 1):
+    for t, b, n in ((out, ob, "out"), (lse, lb, "lse"), (dq, gq, "dq"), (dk, gk, "dk"), (dv, gv, "dv")):
+        check_guards(t, b, what=n)
+    wss.check()
+    scale = D ** -0.5
+    for d in range(len(cu) - 1):
         a, b = int(cu[d]), int(cu[d + 1])
         one = np.array([0, b - a])
         for h in (0, 17, 31):
@@ -48,11 +56,10 @@ def test_packed_zigzag_full_size(schedule):
             ro, rl = A.attention_fwd(qh, kh, vh, one, one, scale)
             check_out(_f64(out[sl]), ro, what=f"out doc {d} head {h}")
             check_lse(host(lse[h:h + 1, a:b]), rl, what=f"lse doc {d} head {h}")
-            if schedule == cbv.SCHEDULE_FUSED:
-                rq, rk, rv = A.attention_bwd(dh, qh, kh, vh, ro, rl, one, one, scale)
-                check_rel(_f64(dq[sl]), rq, what=f"dq doc {d} head {h}")
-                check_rel(_f64(dk[sl]), rk, what=f"dk doc {d} head {h}")
-                check_rel(_f64(dv[sl]), rv, what=f"dv doc {d} head {h}")
+            rq, rk, rv = A.attention_bwd(dh, qh, kh, vh, _f64(out[sl]), rl, one, one, scale)
+            check_rel(_f64(dq[sl]), rq, what=f"dq doc {d} head {h}")
+            check_rel(_f64(dk[sl]), rk, what=f"dk doc {d} head {h}")
+            check_rel(_f64(dv[sl]), rv, what=f"dv doc {d} head {h}")
 
 
 @pytest.mark.parametrize("window,layout", [(0, "zigzag"), (4096, "zigzag"), (0, "contiguous")])

@@ -7,7 +7,7 @@ import context_blockwise_causal_varlen_b200 as cbv
 from oracle import decode as DEC
 from oracle import paged as PG
 from synth import block_permutation, cu_from_lengths, streams
-from tests.gpu_util import check_lse, check_out, dev, f64, gen, host, sync
+from tests.gpu_util import GuardedWorkspaces, check_guards, check_lse, check_out, dev, f64, gen, guarded, host, sync
 
 pytestmark = pytest.mark.gpu
 
@@ -29,9 +29,14 @@ def test_kvp_prefill_matches_oracle(mode, window, seg):
     K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, mode)
     ro, rl = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=window)
     kv_mode = cbv.KV_ROUND_ROBIN if mode == PG.ROUND_ROBIN else cbv.KV_CONTIGUOUS
-    out, lse = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), kv_mode=kv_mode, seg_size=seg,
-                                         scale=0.1, global_q_offset=gqo, sliding_window=window)
+    (out, ob), (lse, lb) = guarded((hq, S, D), torch.bfloat16), guarded((hq, S), torch.float32)
+    wss = GuardedWorkspaces()
+    cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), kv_mode=kv_mode, seg_size=seg,
+                              scale=0.1, global_q_offset=gqo, sliding_window=window, out=out, lse=lse, workspace=wss)
     sync()
+    check_guards(out, ob, what="out")
+    check_guards(lse, lb, what="lse")
+    wss.check()
     check_out(host(out), ro)
     check_lse(host(lse), rl)
 
@@ -43,9 +48,16 @@ def test_kvp_per_shard_partials_and_their_merge():
     gqo = 300
     (ro, rl), shards = PG.prefill_segmented(f64(q), f64(kc), f64(vc), bt, bs, 128, 0.1, gqo, window=0,
                                             mode=PG.ROUND_ROBIN, return_shards=True)
+    (so_, sob), (sl_, slb) = guarded((R, hq, S, D), torch.float32), guarded((R, hq, S), torch.float32)
+    (o_, obuf), (l_, lbuf) = guarded((hq, S, D), torch.bfloat16), guarded((hq, S), torch.float32)
+    wss = GuardedWorkspaces()
     out, lse, so, sl = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), seg_size=128,
-                                                 scale=0.1, global_q_offset=gqo, per_shard=True)
+                                                 scale=0.1, global_q_offset=gqo, per_shard=True, out=o_, lse=l_,
+                                                 shard_out=so_, shard_lse=sl_, workspace=wss)
     sync()
+    for t, b, n in ((so_, sob, "shard_out"), (sl_, slb, "shard_lse"), (o_, obuf, "out"), (l_, lbuf, "lse")):
+        check_guards(t, b, what=n)
+    wss.check()
     check_out(host(out), ro)
     check_lse(host(lse), rl)
     for r in range(R):
@@ -72,8 +84,10 @@ def test_decode_matches_oracle(hq, hkv, D):
     q, k, v = gen(31, (n, hq, D), (int(cu_k[-1]), hkv, D), (int(cu_k[-1]), hkv, D))
     cu_q = np.arange(n + 1, dtype=np.int32)
     ref = DEC.varlen_decode(f64(q), f64(k), f64(v), cu_q, cu_k, 0.1)
-    out = cbv.varlen_decode(dev(q), dev(k), dev(v), torch.from_numpy(cu_q), torch.from_numpy(cu_k), scale=0.1)
+    out, ob = guarded((n, hq, D), torch.bfloat16)
+    cbv.varlen_decode(dev(q), dev(k), dev(v), torch.from_numpy(cu_q), torch.from_numpy(cu_k), scale=0.1, out=out)
     sync()
+    check_guards(out, ob, what="decode out")
     check_out(host(out), ref)
     assert np.all(host(out)[0] == 0)  # empty key range -> zeros
 
@@ -131,10 +145,16 @@ def test_kvp_tail_tasks_split_in_halves(window, tp_out):
     q, kc, vc, perm = _paged(60, R, bps, bs, hq, hkv, D, S)
     bt = PG.shard_block_tables(perm, R, PG.ROUND_ROBIN)
     gqo = R * bps * bs - S
+    (out, ob), (lse, lb) = guarded((hq, D, S) if tp_out else (hq, S, D), torch.bfloat16), guarded((hq, S), torch.float32)
+    wss = GuardedWorkspaces()
     n0 = cbv.launch_count()
-    out, lse = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), seg_size=512, scale=0.1,
-                                         global_q_offset=gqo, sliding_window=window, tp_out=tp_out)
+    cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), seg_size=512, scale=0.1,
+                              global_q_offset=gqo, sliding_window=window, tp_out=tp_out, out=out, lse=lse,
+                              workspace=wss)
     sync()
+    check_guards(out, ob, what="out")
+    check_guards(lse, lb, what="lse")
+    wss.check()
     assert cbv.launch_count() - n0 == 3  # schedule, the prefill (whole tasks and halves), the merge
     rows = np.unique(np.concatenate([[p, p + 1, p + 127, p + 128, p + 255] for p in range(0, S, 256)]))
     K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, PG.ROUND_ROBIN)

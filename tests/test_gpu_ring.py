@@ -9,7 +9,8 @@ from oracle import planner as P
 from oracle import ring as R
 from synth import cu_from_lengths
 from synth.workloads import tiny_zigzag
-from tests.gpu_util import check_lse, check_out, check_rel, dev, f64, gen, host, sync
+from tests.gpu_util import (GuardedWorkspaces, check_guards, check_lse, check_out, check_rel, dev, f64, gen, guarded,
+                            host, sync)
 
 pytestmark = pytest.mark.gpu
 
@@ -27,9 +28,14 @@ def test_tiny_zigzag_forward(schedule, layout):
     w = tiny_zigzag()
     S = w.total
     q, k, v = gen(0, (S, w.heads, w.head_dim), (S, w.heads, w.head_dim), (S, w.heads, w.head_dim))
-    out, lse = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), w.cu_seqlens, w.cp, scale=1 / 8, layout=layout,
-                                   schedule=schedule)
+    (out, ob), (lse, lb) = guarded((S, w.heads, w.head_dim), torch.bfloat16), guarded((w.heads, S), torch.float32)
+    wss = GuardedWorkspaces()
+    cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), w.cu_seqlens, w.cp, scale=1 / 8, layout=layout, schedule=schedule,
+                        out=out, lse=lse, workspace=wss)
     sync()
+    check_guards(out, ob, what="out")
+    check_guards(lse, lb, what="lse")
+    wss.check()
     ro, rl = R.ring_fwd(f64(q), f64(k), f64(v), w.cu_seqlens, w.cp, 1 / 8,
                         layout=P.ZIGZAG if layout == "zigzag" else P.CONTIGUOUS)
     assert out.shape == (256, 2, 64) and lse.shape == (2, 256)
@@ -53,10 +59,16 @@ RING_CASES = [
 def test_ring_forward_matches_oracle(lengths, cp, H, HKV, D, window, layout):
     cu, q, k, v, _ = _case(1, lengths, H, HKV, D)
     ro, rl = A.attention_fwd(f64(q), f64(k), f64(v), cu, cu, 0.09, causal=True, window=window)
+    S, H = q.shape[0], q.shape[1]
     for schedule in (cbv.SCHEDULE_FUSED, cbv.SCHEDULE_STEPWISE):
-        out, lse = cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, cp, scale=0.09, window=window, layout=layout,
-                                       schedule=schedule)
+        (out, ob), (lse, lb) = guarded(q.shape, torch.bfloat16), guarded((H, S), torch.float32)
+        wss = GuardedWorkspaces()
+        cbv.zigzag_ring_fwd(dev(q), dev(k), dev(v), cu, cp, scale=0.09, window=window, layout=layout,
+                            schedule=schedule, out=out, lse=lse, workspace=wss)
         sync()
+        check_guards(out, ob, what="out")
+        check_guards(lse, lb, what="lse")
+        wss.check()
         check_out(host(out), ro)
         check_lse(host(lse), rl)
 
@@ -71,11 +83,20 @@ def test_ring_backward_matches_oracle(lengths, cp, H, HKV, D, window):
     ro_b = host(out_b)
     rq, rk, rv = A.attention_bwd(f64(do), f64(q), f64(k), f64(v), ro_b, rl, cu, cu, scale, causal=True, window=window)
     lse_d = torch.from_numpy(rl.astype(np.float32)).cuda()
-    dq, dk, dv = cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out_b, lse_d, cu, cp, scale=scale, window=window)
-    sync()
-    check_rel(host(dq), rq, what="dq")
-    check_rel(host(dk), rk, what="dk")
-    check_rel(host(dv), rv, what="dv")
+    (dq, gq), (dk, gk), (dv, gv) = (guarded(x.shape, torch.bfloat16) for x in (q, k, v))
+    wss = GuardedWorkspaces()
+    for det in (False, True):
+        for t in (dq, dk, dv):
+            t.fill_(float("nan"))
+        cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out_b, lse_d, cu, cp, scale=scale, window=window, dq=dq,
+                            dk=dk, dv=dv, workspace=wss, deterministic=det)
+        sync()
+        for t, b, n in ((dq, gq, "dq"), (dk, gk, "dk"), (dv, gv, "dv")):
+            check_guards(t, b, what=n)
+        wss.check()
+        check_rel(host(dq), rq, what="dq")
+        check_rel(host(dk), rk, what="dk")
+        check_rel(host(dv), rv, what="dv")
 
 
 def test_forward_then_backward_chain():
