@@ -184,6 +184,16 @@ int upload_plan(const PlanDev& d, const Plan& p, cudaStream_t s) {
 
 int launch_rc(int e, const char* what) { return e == 0 ? CBV_OK : cuda_fail(e, what); }
 
+// Streaming multiprocessors of the current device (0 if it cannot be asked).
+int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return sms;
+}
+
 int grid_of(size_t tasks, int heads) {
   const size_t g = tasks * (size_t)heads;
   return g > (size_t)INT32_MAX ? -1 : (int)g;
@@ -866,6 +876,7 @@ static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_
   p.dkv_accumulate = 0;
   p.dq_fixed = det ? static_cast<unsigned long long*>(dq_buf) : nullptr;
   p.dq_fixed_tpad = fixed_tpad(a->total);
+  p.prefetch_ahead = sm_count();
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
@@ -960,6 +971,7 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.dkv_stride_t = (int64_t)Hkv * D;
   p.dkv_stride_h = D;
   p.dkv_accumulate = 1;
+  p.prefetch_ahead = sm_count();
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;

@@ -191,6 +191,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_q);
+      if (p.prefetch_ahead > 0 && (int)blockIdx.x + p.prefetch_ahead < p.num_tasks) {
+        // warm L2 with the keys and values of the task that will likely start on an SM when this
+        // wave ends, so its start waits on L2 rather than on HBM
+        const TileTask nx = p.tasks[blockIdx.x + p.prefetch_ahead];
+        for (int h = 0; h < KH; ++h) {
+          tma_prefetch_l2_3d(&p.tm_k, h * 64, nx.head, nx.row0);
+          tma_prefetch_l2_3d(&p.tm_v, h * 64, nx.head, nx.row0);
+          if (nx.split1) {
+            tma_prefetch_l2_3d(&p.tm_k, h * 64, nx.head, nx.row1);
+            tma_prefetch_l2_3d(&p.tm_v, h * 64, nx.head, nx.row1);
+          }
+        }
+      }
       mbar_arrive_expect_tx(&bar[bKVFull], 2 * L::kKV);
       for (int h = 0; h < KH; ++h) {
         if (!t.split1) {
@@ -415,41 +428,66 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     if (ok && mbar_wait_warp(&bar[bAccDone], 0, p.status, kDevTimeoutEpilogue)) {
       tc_fence_after();
       const bool any = j > 0;
-      {
-        const int which = wg;  // warpgroup 0: dV, warpgroup 1: dK
-        const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_base;
-        const float mul = which == 0 ? 1.f : p.scale;
-        void* dst_base = which == 0 ? p.dv : p.dk;
+      const int which = wg;  // warpgroup 0: dV, warpgroup 1: dK
+      const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_base;
+      const float mul = which == 0 ? 1.f : p.scale;
+      void* dst_base = which == 0 ? p.dv : p.dk;
+      if (!p.dkv_accumulate) {
+        // bf16 out through shared memory, so that the global stores are whole rows: each warp
+        // stages its 32 key rows in the K / V tiles (every MMA that read them has completed), then
+        // consecutive lanes store consecutive 16-byte pieces of a row
+        constexpr int UPR = D / 8;  // 16-byte units per row
+        const uint32_t stg = smem_u32(sm + L::kK) + (uint32_t)(wg * 4 + quarter) * (32 * D * 2);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tsrc + c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = any ? __uint_as_float(o[u4 * 8 + e]) * mul : 0.f;
+            const int unit = c / 8 + u4;
+            st_shared_v4(stg + lane * (D * 2) + ((unit ^ (lane & (UPR - 1))) << 4), pack_bf16x2(x[0], x[1]),
+                         pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+          }
+        }
+        __syncwarp();
+        constexpr int RPI = 32 / UPR;  // rows per store instruction
+        const int sub = lane / UPR, unit = lane % UPR;
+#pragma unroll
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int lr = i * RPI + sub;
+          const int kr = quarter * 32 + lr;
+          const bool sec = t.split1 && kr >= t.split1;
+          const bool valid = sec ? kr - t.split1 < t.rows1 : kr < t.rows;
+          uint32_t v4[4];
+          ld_shared_v4(stg + lr * (D * 2) + ((unit ^ (lr & (UPR - 1))) << 4), v4);
+          if (valid) {
+            const int64_t kg = sec ? (int64_t)t.row1 + (kr - t.split1) : (int64_t)t.row0 + kr;
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(dst_base) + kg * p.dkv_stride_t +
+                                 (int64_t)kvh * p.dkv_stride_h + unit * 8;
+            *reinterpret_cast<uint4*>(dst) = make_uint4(v4[0], v4[1], v4[2], v4[3]);
+          }
+        }
+      } else {
         const int64_t off = (int64_t)kglobal * p.dkv_stride_t + (int64_t)kvh * p.dkv_stride_h;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
           tmem_ld32(tsrc + c, o);
           tmem_ld_wait();
-          if (!kvalid) continue;
-          if (p.dkv_accumulate) {
-            if (!any) continue;
-            float* dst = reinterpret_cast<float*>(dst_base) + off + c;
+          if (!kvalid || !any) continue;
+          float* dst = reinterpret_cast<float*>(dst_base) + off + c;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              float4 a = *reinterpret_cast<float4*>(dst + e);
-              a.x += __uint_as_float(o[e]) * mul;
-              a.y += __uint_as_float(o[e + 1]) * mul;
-              a.z += __uint_as_float(o[e + 2]) * mul;
-              a.w += __uint_as_float(o[e + 3]) * mul;
-              *reinterpret_cast<float4*>(dst + e) = a;
-            }
-          } else {
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(dst_base) + off + c;
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              float x[8];
-#pragma unroll
-              for (int q = 0; q < 8; ++q) x[q] = any ? __uint_as_float(o[e + q]) * mul : 0.f;
-              uint4 v = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                                   pack_bf16x2(x[6], x[7]));
-              *reinterpret_cast<uint4*>(dst + e) = v;
-            }
+          for (int e = 0; e < 32; e += 4) {
+            float4 a = *reinterpret_cast<float4*>(dst + e);
+            a.x += __uint_as_float(o[e]) * mul;
+            a.y += __uint_as_float(o[e + 1]) * mul;
+            a.z += __uint_as_float(o[e + 2]) * mul;
+            a.w += __uint_as_float(o[e + 3]) * mul;
+            *reinterpret_cast<float4*>(dst + e) = a;
           }
         }
       }

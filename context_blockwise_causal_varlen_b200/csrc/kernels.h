@@ -83,6 +83,9 @@ struct BwdParams {
   // (deterministic mode); null: fp32 reduce-adds through tm_dq.  Layout: see fixed_index().
   unsigned long long* dq_fixed;
   int64_t dq_fixed_tpad;
+  // > 0: each CTA prefetches into L2 the key and value tile of task blockIdx.x + prefetch_ahead
+  // (the SM count: roughly the task that starts on an SM when this wave's CTAs finish)
+  int32_t prefetch_ahead;
   int* status;
 };
 
