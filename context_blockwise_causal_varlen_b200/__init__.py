@@ -147,6 +147,34 @@ class CachedRingArgs(ctypes.Structure):
     ]
 
 
+class RingStepArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("rank", ctypes.c_int32), ("step", ctypes.c_int32),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n_local", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("num_docs", ctypes.c_int32), ("cu_seqlens", c_i32p), ("cp", ctypes.c_int32), ("layout", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("window", ctypes.c_int32),
+        ("out_acc", ctypes.c_void_p), ("lse_acc", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("dout", ctypes.c_void_p), ("out_merged", ctypes.c_void_p), ("lse_merged", ctypes.c_void_p),
+        ("dq_acc", ctypes.c_void_p), ("dk_acc", ctypes.c_void_p), ("dv_acc", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class DiagArgs(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", ctypes.c_uint32), ("abi_version", ctypes.c_uint32),
+        ("q", ctypes.c_void_p), ("cache_k", ctypes.POINTER(ctypes.c_void_p)),
+        ("cache_v", ctypes.POINTER(ctypes.c_void_p)), ("num_blocks", ctypes.c_int32), ("total", ctypes.c_int64),
+        ("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("out0", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("dout", ctypes.c_void_p), ("out_merged", ctypes.c_void_p), ("lse_merged", ctypes.c_void_p),
+        ("dq0", ctypes.c_void_p), ("dq", ctypes.c_void_p), ("dcache_k", ctypes.POINTER(ctypes.c_void_p)),
+        ("dcache_v", ctypes.POINTER(ctypes.c_void_p)),
+    ]
+
+
 class RowRun(ctypes.Structure):
     _fields_ = [("doc", ctypes.c_int32), ("row0", ctypes.c_int32), ("rows", ctypes.c_int32), ("pos0", ctypes.c_int32),
                 ("local0", ctypes.c_int32)]
@@ -168,7 +196,9 @@ EXPORTS = [
     "cbv_zigzag_ring_bwd", "cbv_block_bwd_workspace_size", "cbv_attn_block_bwd",
     "cbv_kvp_workspace_size", "cbv_kvp_segmented_prefill", "cbv_decode_workspace_size", "cbv_varlen_decode",
     "cbv_noalloc_scratch_bytes", "cbv_zigzag_ring_fwd_noalloc", "cbv_noalloc_read_status",
-    "cbv_debug_ring_fwd_stalled",
+    "cbv_debug_ring_fwd_stalled", "cbv_ring_step_fwd_workspace_size", "cbv_ring_step_fwd",
+    "cbv_ring_step_bwd_workspace_size", "cbv_ring_step_bwd", "cbv_cached_diag_merge", "cbv_cached_diag_grad",
+    "cbv_convert_f32_bf16", "cbv_swap_leading_axes",
     "cbv_cached_ring_fwd_workspace_size", "cbv_cached_ring_fwd", "cbv_cached_ring_bwd_workspace_size",
     "cbv_cached_ring_bwd",
 ]
@@ -203,6 +233,15 @@ def _declare(L):
     L.cbv_zigzag_ring_fwd_noalloc.argtypes = [ctypes.POINTER(RingArgs), ctypes.c_void_p]
     L.cbv_noalloc_read_status.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
     L.cbv_debug_ring_fwd_stalled.argtypes = [ctypes.POINTER(RingArgs), ctypes.c_uint64, ctypes.c_void_p]
+    for name in ("fwd", "bwd"):
+        getattr(L, f"cbv_ring_step_{name}_workspace_size").argtypes = [ctypes.POINTER(RingStepArgs)]
+        getattr(L, f"cbv_ring_step_{name}_workspace_size").restype = ctypes.c_size_t
+        getattr(L, f"cbv_ring_step_{name}").argtypes = [ctypes.POINTER(RingStepArgs), ctypes.c_void_p]
+    L.cbv_cached_diag_merge.argtypes = [ctypes.POINTER(DiagArgs), ctypes.c_void_p]
+    L.cbv_cached_diag_grad.argtypes = [ctypes.POINTER(DiagArgs), ctypes.c_void_p]
+    L.cbv_convert_f32_bf16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p]
+    L.cbv_swap_leading_axes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int64, ctypes.c_void_p]
     L.cbv_attn_merge.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                  ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]
 
@@ -670,3 +709,127 @@ def varlen_decode(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, validate=None
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
     _check(lib().cbv_varlen_decode(ctypes.byref(a), _stream(q.device)))
     return out
+
+
+# ----------------------------------------------------------------------------- ring steps on real ranks
+def _step_args(rank, step, q, k, v, cu, cp, scale, window, layout, **tensors):
+    n, H, D = q.shape
+    return RingStepArgs(**_header(RingStepArgs), rank=int(rank), step=int(step), q=_ptr(q), k=_ptr(k), v=_ptr(v),
+                        n_local=n, num_heads=H, num_kv_heads=k.shape[1], head_dim=D, num_docs=len(cu) - 1,
+                        cu_seqlens=_p32(cu), cp=int(cp), layout=_layout(layout), scale=_scale(scale),
+                        window=int(window), **{name: _ptr(t) for name, t in tensors.items()})
+
+
+def ring_step_fwd(rank: int, step: int, q, k, v, cu_seqlens, cp: int, out_acc, lse_acc, out=None, scale=None,
+                  window: int = 0, layout="zigzag"):
+    """One rank's block at one ring step on local buffers (see ``cbv_ring_step_fwd``): merges into the
+    running f32 ``(out_acc [n,H,D], lse_acc [H,n])``; with ``out`` (bf16) also rounds the running out into it."""
+    q, k, v = _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v")
+    n, H, D = q.shape
+    _shape(k, (n, k.shape[1], D), "k")
+    _shape(v, k.shape, "v")
+    _given(out_acc, (n, H, D), torch.float32, q.device, "out_acc")
+    _given(lse_acc, (H, n), torch.float32, q.device, "lse_acc")
+    if out is not None:
+        _given(out, (n, H, D), torch.bfloat16, q.device, "out")
+    cu = _host_i32(cu_seqlens)
+    a = _step_args(rank, step, q, k, v, cu, cp, scale, window, layout, out_acc=out_acc, lse_acc=lse_acc, out=out)
+    ws = _workspace(lib().cbv_ring_step_fwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_ring_step_fwd(ctypes.byref(a), _stream(q.device)))
+    return out_acc, lse_acc
+
+
+def ring_step_bwd(rank: int, step: int, dout, q, k, v, out, lse, cu_seqlens, cp: int, dq_acc, dk_acc, dv_acc,
+                  scale=None, window: int = 0, layout="zigzag"):
+    """One rank's block backward at one ring step, fed this rank's merged ``(out, lse)``: adds into
+    ``dq_acc`` (this rank's rows) and ``dk_acc`` / ``dv_acc`` (the rows of the k/v held at this step)."""
+    dout, q, k, v, out = (_bf16(t, nm) for t, nm in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")))
+    n, H, D = q.shape
+    _shape(k, (n, k.shape[1], D), "k")
+    _shape(v, k.shape, "v")
+    _shape(dout, q.shape, "dout")
+    _shape(out, q.shape, "out")
+    _shape(lse, (H, n), "lse", torch.float32)
+    _given(dq_acc, (n, H, D), torch.float32, q.device, "dq_acc")
+    _given(dk_acc, k.shape, torch.float32, q.device, "dk_acc")
+    _given(dv_acc, k.shape, torch.float32, q.device, "dv_acc")
+    cu = _host_i32(cu_seqlens)
+    a = _step_args(rank, step, q, k, v, cu, cp, scale, window, layout, dout=dout, out_merged=out,
+                   lse_merged=lse.contiguous(), dq_acc=dq_acc, dk_acc=dk_acc, dv_acc=dv_acc)
+    ws = _workspace(lib().cbv_ring_step_bwd_workspace_size(ctypes.byref(a)), q.device)
+    a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
+    _check(lib().cbv_ring_step_bwd(ctypes.byref(a), _stream(q.device)))
+    return dq_acc, dk_acc, dv_acc
+
+
+def _diag_args(q, ck, cv, scale, **tensors):
+    T, H, D = q.shape
+    keep = [_ptr_array(ck), _ptr_array(cv)]
+    a = DiagArgs(**_header(DiagArgs), q=_ptr(q), num_blocks=len(ck), total=T, num_heads=H,
+                 num_kv_heads=ck[0].shape[1], head_dim=D, scale=_scale(scale),
+                 **{name: _ptr(t) for name, t in tensors.items()})
+    a.cache_k = ctypes.cast(keep[0], ctypes.POINTER(ctypes.c_void_p))
+    a.cache_v = ctypes.cast(keep[1], ctypes.POINTER(ctypes.c_void_p))
+    return a, keep
+
+
+def cached_diag_merge(q, cache_k, cache_v, out0, lse, scale=None, out=None):
+    """Merge the per-position cache diagonals (blocks 1..) into block 0's normalised f32 ``out0`` and
+    ``lse`` (updated in place): returns ``(out bf16, lse)``."""
+    q = _bf16(q, "q")
+    ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
+    T, H, D = q.shape
+    _shape(out0, q.shape, "out0", torch.float32)
+    _given(lse, (H, T), torch.float32, q.device, "lse")
+    out = torch.empty_like(q) if out is None else _given(out, q.shape, torch.bfloat16, q.device, "out")
+    a, keep = _diag_args(q, ck, cv, scale, out0=out0.contiguous(), lse=lse, out=out)
+    _check(lib().cbv_cached_diag_merge(ctypes.byref(a), _stream(q.device)))
+    return out, lse
+
+
+def cached_diag_grad(dout, q, cache_k, cache_v, out, lse, dq0, scale=None, dq=None, dcache_k=None, dcache_v=None):
+    """Closed-form gradients of the cache diagonals fed the merged ``(out, lse)``: ``dq = dq0 + diagonal
+    terms`` (bf16) and the gradients of blocks 1.. (lists; entry 0 is None)."""
+    dout, q, out = _bf16(dout, "dout"), _bf16(q, "q"), _bf16(out, "out")
+    ck, cv = _blocks(cache_k, "cache_k"), _blocks(cache_v, "cache_v")
+    T, H, D = q.shape
+    _shape(dq0, q.shape, "dq0", torch.float32)
+    _shape(lse, (H, T), "lse", torch.float32)
+    dq = torch.empty_like(q) if dq is None else _given(dq, q.shape, torch.bfloat16, q.device, "dq")
+    dck = [None] + ([torch.empty_like(b) for b in ck[1:]] if dcache_k is None else list(dcache_k)[1:])
+    dcv = [None] + ([torch.empty_like(b) for b in cv[1:]] if dcache_v is None else list(dcache_v)[1:])
+    a, keep = _diag_args(q, ck, cv, scale, dout=dout, out_merged=out, lse_merged=lse.contiguous(), dq0=dq0.contiguous(),
+                         dq=dq)
+    pk = (ctypes.c_void_p * len(ck))(*[0] + [b.data_ptr() for b in dck[1:]])
+    pv = (ctypes.c_void_p * len(cv))(*[0] + [b.data_ptr() for b in dcv[1:]])
+    a.dcache_k = ctypes.cast(pk, ctypes.POINTER(ctypes.c_void_p))
+    a.dcache_v = ctypes.cast(pv, ctypes.POINTER(ctypes.c_void_p))
+    _check(lib().cbv_cached_diag_grad(ctypes.byref(a), _stream(q.device)))
+    return dq, dck, dcv
+
+
+def convert_f32_bf16(src, dst=None, mul: float = 1.0):
+    """bf16 rounding of an f32 tensor (``cbv_convert_f32_bf16``)."""
+    if not src.is_cuda or src.dtype != torch.float32:
+        raise CbvError(-3, "src must be a CUDA float32 tensor")
+    src = src.contiguous()
+    dst = torch.empty(src.shape, dtype=torch.bfloat16, device=src.device) if dst is None else dst
+    _given(dst, src.shape, torch.bfloat16, src.device, "dst")
+    _check(lib().cbv_convert_f32_bf16(_ptr(src), _ptr(dst), src.numel(), float(mul), _stream(src.device)))
+    return dst
+
+
+def swap_leading_axes(src, dst=None):
+    """``dst[b, a, ...] = src[a, b, ...]`` for a contiguous CUDA tensor of >= 2 dims (``cbv_swap_leading_axes``)."""
+    if not src.is_cuda or src.dim() < 2:
+        raise CbvError(-1, "src must be a CUDA tensor with at least two dimensions")
+    src = src.contiguous()
+    a, b = src.shape[0], src.shape[1]
+    shape = (b, a) + tuple(src.shape[2:])
+    dst = torch.empty(shape, dtype=src.dtype, device=src.device) if dst is None else dst
+    _given(dst, shape, src.dtype, src.device, "dst")
+    row = src[0, 0].numel() * src.element_size() if src.numel() else 0
+    _check(lib().cbv_swap_leading_axes(_ptr(src), _ptr(dst), a, b, row, _stream(src.device)))
+    return dst
+

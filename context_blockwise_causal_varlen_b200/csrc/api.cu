@@ -1135,3 +1135,230 @@ int cbv_cached_ring_bwd(const cbv_cached_ring_args* a, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------ one ring step on real ranks
+namespace {
+
+int ring_step_checks(const cbv_ring_step_args* a) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_ring_step_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if (a->cp < 1) return fail(CBV_ERR_BAD_ARG, "cp must be >= 1");
+  if (a->rank < 0 || a->rank >= a->cp || a->step < 0 || a->step >= a->cp)
+    return fail(CBV_ERR_BAD_ARG, "rank %d / step %d outside [0, %d)", a->rank, a->step, a->cp);
+  if (a->layout != CBV_LAYOUT_ZIGZAG && a->layout != CBV_LAYOUT_CONTIGUOUS) return fail(CBV_ERR_BAD_ARG, "bad layout");
+  if (a->n_local < 0) return fail(CBV_ERR_BAD_SHAPE, "n_local must be >= 0");
+  if ((rc = check_cu(a->cu_seqlens, a->num_docs, a->n_local * a->cp, "cu_seqlens"))) return rc;
+  if ((int64_t)a->cu_seqlens[a->num_docs] != a->n_local * a->cp)
+    return fail(CBV_ERR_BAD_CU_SEQLENS, "cu_seqlens must end at n_local * cp (%lld)", (long long)(a->n_local * a->cp));
+  std::string e = check_divisible(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout);
+  if (!e.empty()) return fail(CBV_ERR_NOT_DIVISIBLE_2CP, "%s", e.c_str());
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  return CBV_OK;
+}
+
+Plan ring_step_fwd_plan(const cbv_ring_step_args* a) {
+  return plan_ring_step_fwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_heads, a->rank,
+                            a->step, kPairRows);
+}
+
+Plan ring_step_bwd_plan(const cbv_ring_step_args* a) {
+  return plan_ring_step_bwd(a->cu_seqlens, a->num_docs, a->cp, (Layout)a->layout, a->window, a->num_kv_heads,
+                            a->rank, a->step, 128);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t cbv_ring_step_fwd_workspace_size(const cbv_ring_step_args* a) {
+  if (ring_step_checks(a)) return 0;
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  carve_plan(c, ring_step_fwd_plan(a));
+  return c.off;
+}
+
+int cbv_ring_step_fwd(const cbv_ring_step_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_ring_step_fwd");
+  int rc = ring_step_checks(a);
+  if (rc) return rc;
+  if (a->n_local == 0) return CBV_OK;
+  if (!a->out_acc || !a->lse_acc) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->out_acc) || !aligned16(a->out)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  Plan plan = ring_step_fwd_plan(a);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, plan);
+  if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
+  FwdParams p{};
+  if ((rc = map_thd(&p.tm_q, a->q, a->n_local, H, D, (int64_t)H * D, D, 128))) return rc;
+  if ((rc = map_thd(&p.tm_k, a->k, a->n_local, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  if ((rc = map_thd(&p.tm_v, a->v, a->n_local, Hkv, D, (int64_t)Hkv * D, D, 128))) return rc;
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)plan.tasks.size();
+  p.num_heads = H;
+  p.heads_per_kv = H / Hkv;
+  p.scale_log2 = resolve_scale(a->scale, D) * kLog2e;
+  p.window = a->window > 0 ? a->window : 0;
+  p.out = a->out_acc;
+  p.out_stride_t = (int64_t)H * D;
+  p.out_stride_h = D;
+  p.lse = a->lse_acc;
+  p.lse_stride_h = a->n_local;
+  p.lse_stride_t = 1;
+  p.out_mode = a->step == 0 ? kOutF32 : kOutMerge;  // every local row takes part in step 0's block
+  p.block_size = 1;
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s))) return rc;
+  const int grid = grid_of(plan.tasks.size(), 1);
+  if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
+  if ((rc = launch_rc(launch_fwd_pingpong(p, D, false, grid, s), "ring step forward launch"))) return rc;
+  if (!a->out) return CBV_OK;
+  return launch_rc(launch_convert_bf16(a->out_acc, a->out, a->n_local * H * D, 1.f, s), "output rounding");
+}
+
+size_t cbv_ring_step_bwd_workspace_size(const cbv_ring_step_args* a) {
+  if (ring_step_checks(a)) return 0;
+  Carve c(nullptr);
+  c.take(kStatusBytes);
+  carve_plan(c, ring_step_bwd_plan(a));
+  c.take((size_t)a->num_heads * pad4(a->n_local) * 2 * sizeof(float));  // {lse * log2e, Delta}
+  return c.off;
+}
+
+int cbv_ring_step_bwd(const cbv_ring_step_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_ring_step_bwd");
+  int rc = ring_step_checks(a);
+  if (rc) return rc;
+  if (a->n_local == 0) return CBV_OK;
+  if (!a->dout || !a->out_merged || !a->lse_merged || !a->dq_acc || !a->dk_acc || !a->dv_acc)
+    return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->dout) || !aligned16(a->out_merged) || !aligned16(a->dq_acc) || !aligned16(a->dk_acc) ||
+      !aligned16(a->dv_acc))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads, Hkv = a->num_kv_heads;
+  Plan plan = ring_step_bwd_plan(a);
+  Carve c(a->workspace);
+  int* status = static_cast<int*>(c.take(kStatusBytes));
+  PlanDev pd = carve_plan(c, plan);
+  const int64_t tp = pad4(a->n_local);
+  float* rows = static_cast<float*>(c.take((size_t)H * tp * 2 * sizeof(float)));
+  if (!a->workspace || a->workspace_bytes < c.off) return fail(CBV_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes", c.off);
+  BwdParams p{};
+  if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, a->dq_acc, a->n_local, a->n_local, H, Hkv, D))) return rc;
+  p.tasks = pd.tasks;
+  p.segs = pd.segs;
+  p.num_tasks = (int)plan.tasks.size();
+  p.num_heads = H;
+  p.num_kv_heads = Hkv;
+  p.heads_per_kv = H / Hkv;
+  p.scale = resolve_scale(a->scale, D);
+  p.scale_log2 = p.scale * kLog2e;
+  p.window = a->window > 0 ? a->window : 0;
+  if ((rc = make_row_map(&p.tm_rows, rows, tp, H))) return rc;
+  p.dk = a->dk_acc;
+  p.dv = a->dv_acc;
+  p.dkv_stride_t = (int64_t)Hkv * D;
+  p.dkv_stride_h = D;
+  p.dkv_accumulate = 1;
+  p.prefetch_ahead = sm_count();
+  p.status = status;
+  if ((rc = zero_status(status, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out_merged, a->lse_merged, a->n_local, tp, H, D, rows, nullptr,
+                                            nullptr, 0, s),
+                      "backward preprocess")))
+    return rc;
+  return launch_rc(launch_bwd(p, D, grid_of(plan.tasks.size(), 1), s), "ring step backward launch");
+}
+
+// ------------------------------------------------------------------------ cache diagonals alone
+static int diag_checks(const cbv_diag_args* a, cbv::CacheBlocks* cb, bool grads) {
+  if (!a) return fail(CBV_ERR_BAD_ARG, "args is NULL");
+  int rc = check_header(a->struct_size, sizeof(cbv_diag_args), a->abi_version);
+  if (rc) return rc;
+  if ((rc = check_heads(a->num_heads, a->num_kv_heads, a->head_dim))) return rc;
+  if (a->num_blocks < 1 || a->num_blocks > cbv::kCacheMaxBlocks)
+    return fail(CBV_ERR_BAD_ARG, "num_blocks must be in [1, %d]", cbv::kCacheMaxBlocks);
+  if (a->total < 0) return fail(CBV_ERR_BAD_SHAPE, "total must be >= 0");
+  *cb = cbv::CacheBlocks{};
+  if (a->num_blocks > 1 && (!a->cache_k || !a->cache_v || (grads && (!a->dcache_k || !a->dcache_v))))
+    return fail(CBV_ERR_BAD_ARG, "NULL cache block array");
+  for (int i = 1; i < a->num_blocks; ++i) {
+    cb->k[i] = a->cache_k[i];
+    cb->v[i] = a->cache_v[i];
+    if (grads) {
+      cb->dk[i] = a->dcache_k[i];
+      cb->dv[i] = a->dcache_v[i];
+    }
+    if (!cb->k[i] || !cb->v[i] || (grads && (!cb->dk[i] || !cb->dv[i]))) return fail(CBV_ERR_BAD_ARG, "NULL cache block %d", i);
+    if (!aligned16(cb->k[i]) || !aligned16(cb->v[i]) || (grads && (!aligned16(cb->dk[i]) || !aligned16(cb->dv[i]))))
+      return fail(CBV_ERR_MISALIGNED, "cache block %d must be 16-byte aligned", i);
+  }
+  return CBV_OK;
+}
+
+int cbv_cached_diag_merge(const cbv_diag_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_cached_diag_merge");
+  cbv::CacheBlocks cb;
+  int rc = diag_checks(a, &cb, false);
+  if (rc) return rc;
+  if (a->total == 0) return CBV_OK;
+  if (!a->q || !a->out0 || !a->lse || !a->out) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->q) || !aligned16(a->out0) || !aligned16(a->out)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads;
+  if (a->num_blocks == 1)
+    return launch_rc(launch_convert_bf16(a->out0, a->out, a->total * H * D, 1.f, s), "output rounding");
+  return launch_rc(cbv::launch_diag_merge(a->q, cb, a->num_blocks, a->total, H, a->num_kv_heads, D,
+                                          resolve_scale(a->scale, D), a->out0, a->lse, a->out, s),
+                   "diagonal merge");
+}
+
+int cbv_cached_diag_grad(const cbv_diag_args* a, void* stream) {
+  NvtxRange nvtx_range("cbv_cached_diag_grad");
+  cbv::CacheBlocks cb;
+  int rc = diag_checks(a, &cb, true);
+  if (rc) return rc;
+  if (a->total == 0) return CBV_OK;
+  if (!a->dq0 || !a->dq || (a->num_blocks > 1 && (!a->q || !a->dout || !a->out_merged || !a->lse_merged)))
+    return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(a->dq0) || !aligned16(a->dq) || !aligned16(a->q) || !aligned16(a->dout) || !aligned16(a->out_merged))
+    return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int D = a->head_dim, H = a->num_heads;
+  if (a->num_blocks == 1) return launch_rc(launch_convert_bf16(a->dq0, a->dq, a->total * H * D, 1.f, s), "dq rounding");
+  return launch_rc(cbv::launch_diag_grad(a->q, cb, a->num_blocks, a->total, H, a->num_kv_heads, D,
+                                         resolve_scale(a->scale, D), a->dout, a->out_merged, a->lse_merged, a->dq0,
+                                         nullptr, a->dq, s),
+                   "diagonal gradients");
+}
+
+// ------------------------------------------------------------------------ layout helpers
+int cbv_convert_f32_bf16(const float* src, void* dst, int64_t n, float mul, void* stream) {
+  if (n < 0 || n % 4) return fail(CBV_ERR_BAD_SHAPE, "n must be a non-negative multiple of 4");
+  if (n == 0) return CBV_OK;
+  if (!src || !dst) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if (!aligned16(src) || !aligned16(dst)) return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+  return launch_rc(launch_convert_bf16(src, dst, n, mul, static_cast<cudaStream_t>(stream)), "conversion");
+}
+
+int cbv_swap_leading_axes(const void* src, void* dst, int64_t a, int64_t b, int64_t row_bytes, void* stream) {
+  if (a < 0 || b < 0 || row_bytes < 0 || row_bytes % 4) return fail(CBV_ERR_BAD_SHAPE, "bad sizes");
+  if (a * b * row_bytes == 0) return CBV_OK;
+  if (!src || !dst) return fail(CBV_ERR_BAD_ARG, "NULL tensor");
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 3) return fail(CBV_ERR_MISALIGNED, "4-byte alignment");
+  const char *s0 = static_cast<const char*>(src), *d0 = static_cast<const char*>(dst);
+  const int64_t n = a * b * row_bytes;
+  if (s0 < d0 + n && d0 < s0 + n) return fail(CBV_ERR_BAD_ARG, "src and dst overlap");
+  return launch_rc(launch_swap01(src, dst, a, b, row_bytes, static_cast<cudaStream_t>(stream)), "axis swap");
+}
+
+}  // extern "C"

@@ -112,6 +112,8 @@ int launch_schedule(void* image_dst, const void* image, size_t bytes, size_t off
 // first_tile + (i - first_task) % ntiles with head (i - first_task) / ntiles.
 int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* tiles, TileTask* tasks, int ntasks,
                         cudaStream_t stream);
+// dst [B][A][row] = src [A][B][row] (row_bytes a multiple of 4; 16-byte moves when aligned).
+int launch_swap01(const void* src, void* dst, int64_t A, int64_t B, int64_t row_bytes, cudaStream_t stream);
 // fp32 [T, H, D] -> bf16, times `mul`.
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream);
 // The two halves of each of `ntasks` split prefill tasks (q tiles of up to 256 rows), whose

@@ -436,6 +436,35 @@ int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* ti
   return launched();
 }
 
+namespace {
+// dst [B][A][row] = src [A][B][row]: the exchange of the leading two axes of an array of rows
+template <typename U>
+__global__ void __launch_bounds__(256) swap01_kernel(const U* __restrict__ src, U* __restrict__ dst, int64_t A,
+                                                     int64_t B, int64_t units) {
+  const int64_t n = A * B * units;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = i % units, ab = i / units;
+    const int64_t a = ab / B, b = ab % B;
+    dst[(b * A + a) * units + u] = src[i];
+  }
+}
+}  // namespace
+
+int launch_swap01(const void* src, void* dst, int64_t A, int64_t B, int64_t row_bytes, cudaStream_t stream) {
+  if (A * B * row_bytes == 0) return 0;
+  const bool v16 = row_bytes % 16 == 0 && reinterpret_cast<uintptr_t>(src) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(dst) % 16 == 0;
+  const int64_t units = row_bytes / (v16 ? 16 : 4);
+  const int64_t blocks = std::min<int64_t>((A * B * units + 255) / 256, 148 * 16);
+  if (v16)
+    swap01_kernel<uint4><<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), A, B,
+                                                     units);
+  else
+    swap01_kernel<uint32_t><<<blocks, 256, 0, stream>>>(static_cast<const uint32_t*>(src),
+                                                        static_cast<uint32_t*>(dst), A, B, units);
+  return launched();
+}
+
 int launch_convert_bf16(const float* src, void* dst, int64_t n, float mul, cudaStream_t stream) {
   if (n == 0) return 0;
   const int64_t n4 = n / 4;  // n is a multiple of the head dim (64 or 128)

@@ -401,6 +401,117 @@ Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
   return plan;
 }
 
+namespace {
+
+// First row of global chunk x of document d in the local sequence of the rank that owns it (its
+// front chunk first, then its back chunk).
+int32_t chunk_local0(const int32_t* cu, int32_t d, int32_t x, int32_t cp, Layout layout) {
+  const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+  const int32_t c = (cu[d + 1] - cu[d]) / nchunk;
+  return cu[d] / cp + ((layout == kZigZag && x >= cp) ? c : 0);
+}
+
+// The chunk pairs of `rank` at `step`, grouped by (document, chunk of side `key`), in order.
+std::vector<std::vector<ChunkPair>> step_groups(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout,
+                                                int32_t window, int32_t rank, int32_t step, bool by_k) {
+  std::map<std::pair<int32_t, int32_t>, size_t> at;
+  std::vector<std::vector<ChunkPair>> out;
+  for (const ChunkPair& p : ring_chunk_pairs(cu, num_docs, cp, layout, window, step)) {
+    if (p.rank != rank) continue;
+    const auto key = std::make_pair(p.doc, by_k ? p.k_chunk : p.q_chunk);
+    auto it = at.find(key);
+    if (it == at.end()) {
+      at[key] = out.size();
+      out.push_back({p});
+    } else {
+      out[it->second].push_back(p);
+    }
+  }
+  return out;
+}
+
+}  // namespace
+
+Plan plan_ring_step_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window,
+                        int32_t heads, int32_t rank, int32_t step, int32_t tile_m) {
+  Plan plan;
+  const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+  for (const auto& g : step_groups(cu, num_docs, cp, layout, window, rank, step, false)) {
+    const int32_t d = g[0].doc, x = g[0].q_chunk;
+    const int32_t c = (cu[d + 1] - cu[d]) / nchunk;
+    const int32_t seg0 = (int32_t)plan.segs.size();
+    for (const ChunkPair& p : g) {
+      Seg s;
+      s.row0 = chunk_local0(cu, d, p.k_chunk, cp, layout);
+      s.rows = c;
+      s.pos0 = cu[d] + p.k_chunk * c;
+      s.flags = (p.causal ? kSegCausal : 0) | (p.k_chunk == g[0].k_chunk ? kSegBlockStart : 0);
+      plan.segs.push_back(s);
+    }
+    coalesce_tail(plan.segs, seg0);
+    const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    for (int32_t t0 = 0; t0 < c; t0 += tile_m) {
+      TileTask t{};
+      t.row0 = chunk_local0(cu, d, x, cp, layout) + t0;
+      t.rows = std::min(tile_m, c - t0);
+      t.pos0 = cu[d] + x * c + t0;
+      t.seg0 = seg0;
+      t.nseg = nseg;
+      t.aux = -1;
+      t.head = d;
+      int64_t w = 0;
+      for (int32_t i = 0; i < nseg; ++i) {
+        const Seg& s = plan.segs[seg0 + i];
+        w += visible_pairs(t.pos0, t.rows, s.pos0, s.rows, s.flags & kSegCausal, window);
+      }
+      t.work = weight(w);
+      plan.tasks.push_back(t);
+    }
+  }
+  expand_heads(plan, heads);
+  return plan;
+}
+
+Plan plan_ring_step_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window,
+                        int32_t kv_heads, int32_t rank, int32_t step, int32_t tile_n) {
+  Plan plan;
+  const int32_t nchunk = layout == kZigZag ? 2 * cp : cp;
+  for (const auto& g : step_groups(cu, num_docs, cp, layout, window, rank, step, true)) {
+    const int32_t d = g[0].doc, y = g[0].k_chunk;
+    const int32_t c = (cu[d + 1] - cu[d]) / nchunk;
+    const int32_t seg0 = (int32_t)plan.segs.size();
+    for (const ChunkPair& p : g) {
+      Seg s;
+      s.row0 = chunk_local0(cu, d, p.q_chunk, cp, layout);
+      s.rows = c;
+      s.pos0 = cu[d] + p.q_chunk * c;
+      s.flags = (p.causal ? kSegCausal : 0) | kSegBlockStart;
+      plan.segs.push_back(s);
+    }
+    coalesce_tail(plan.segs, seg0);
+    const int32_t nseg = (int32_t)plan.segs.size() - seg0;
+    for (int32_t t0 = 0; t0 < c; t0 += tile_n) {
+      TileTask t{};
+      t.row0 = chunk_local0(cu, d, y, cp, layout) + t0;
+      t.rows = std::min(tile_n, c - t0);
+      t.pos0 = cu[d] + y * c + t0;
+      t.seg0 = seg0;
+      t.nseg = nseg;
+      t.aux = -1;
+      t.head = d;
+      int64_t w = 0;
+      for (int32_t i = 0; i < nseg; ++i) {
+        const Seg& s = plan.segs[seg0 + i];
+        w += visible_pairs(s.pos0, s.rows, t.pos0, t.rows, s.flags & kSegCausal, window);
+      }
+      t.work = weight(w);
+      plan.tasks.push_back(t);
+    }
+  }
+  expand_heads(plan, kv_heads);
+  return plan;
+}
+
 Plan plan_block_fwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qbase, const int32_t* kbase,
                     int32_t num_docs, bool causal, int32_t window, int32_t heads, int32_t tile_m) {
   Plan plan;

@@ -113,6 +113,17 @@ Plan plan_ring_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layou
 // that meet the tile's chunk (all blocks), coalesced into runs of adjacent rows.
 Plan plan_ring_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window, int32_t kv_heads,
                    int32_t tile_n);
+// One ring step of one rank on LOCAL buffers, for the ring over real ranks: q rows are rows of
+// `rank`'s local sequence, k rows rows of the local sequence of the step's source rank, and
+// positions stay global, so the masks mean what they mean in the single-GPU ring.
+// Forward: one task per 128-row q tile of every chunk of `rank` that the block touches (per head),
+// segments = the source chunks it meets.  Backward: one task per 128-row k tile of every source
+// chunk the block touches (per kv head), segments = the q chunks of `rank` that meet it.
+Plan plan_ring_step_fwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window,
+                        int32_t heads, int32_t rank, int32_t step, int32_t tile_m);
+Plan plan_ring_step_bwd(const int32_t* cu, int32_t num_docs, int32_t cp, Layout layout, int32_t window,
+                        int32_t kv_heads, int32_t rank, int32_t step, int32_t tile_n);
+
 // One varlen block with explicit per-document positions.
 Plan plan_block_fwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qbase, const int32_t* kbase,
                     int32_t num_docs, bool causal, int32_t window, int32_t heads, int32_t tile_m);

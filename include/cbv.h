@@ -271,6 +271,57 @@ int cbv_zigzag_ring_fwd(const cbv_ring_args* a, void* stream);
 size_t cbv_zigzag_ring_bwd_workspace_size(const cbv_ring_args* a);
 int cbv_zigzag_ring_bwd(const cbv_ring_args* a, void* stream);
 
+/* ========================================================================= one ring step on real ranks
+ * The ring over cp REAL ranks (one process per GPU), as the zig-zag page runs it: RingComm
+ * rotates K/V one rank along per step, and each rank runs one flash block per step against the
+ * K/V it holds (zigzag_ring_flash_attn_varlen_forward; ring_attention.ring_flash_attn_forward for
+ * CBV_LAYOUT_CONTIGUOUS).  These calls are that block on a rank's LOCAL buffers; the exchange is
+ * the caller's (the Python package's ring driver sends over torch.distributed).  At `step`, rank
+ * `rank` holds the k/v of src = (rank - step) mod cp and runs the block of cbv_ring_step /
+ * cbv_plan_zigzag against them.  Local buffers hold a rank's tokens in local order (for every
+ * document its front chunk, then its back chunk: the rows of cbv_rank_tokens); masks use global
+ * positions computed from cu_seqlens, so results equal the single-GPU ring's.
+ * Forward: step 0 writes the rank's running (out_acc, lse_acc); later steps merge into them with
+ * the online-softmax identity in the kernel epilogue; with `out` set, the running out is also
+ * rounded into that bf16 tensor (pass it at the last step).
+ * Backward (zigzag_ring_flash_attn_varlen_backward, the merged-lse identity): the block's
+ * gradients, fed the MERGED out_merged / lse_merged of this rank's rows, are ADDED into dq_acc
+ * (this rank's rows) and into dk_acc / dv_acc, the fp32 accumulators of src's k/v rows that
+ * travel around the ring with k/v and arrive back at their owner after cp hops.
+ * Errors: those of cbv_ring_args, plus rank / step outside [0, cp) -> CBV_ERR_BAD_ARG and
+ * cu_seqlens[num_docs] != n_local * cp -> CBV_ERR_BAD_CU_SEQLENS. */
+typedef struct cbv_ring_step_args {
+  uint32_t struct_size;       /* sizeof(cbv_ring_step_args) */
+  uint32_t abi_version;       /* CBV_ABI_VERSION */
+  int32_t rank, step;
+  const void* q;              /* device bf16 [n_local, num_heads, head_dim]: this rank's local q */
+  const void* k;              /* device bf16 [n_local, num_kv_heads, head_dim]: src's local k (held at this step) */
+  const void* v;
+  int64_t n_local;            /* total / cp */
+  int32_t num_heads, num_kv_heads, head_dim;
+  int32_t num_docs;
+  const int32_t* cu_seqlens;  /* host int32 [num_docs+1], GLOBAL */
+  int32_t cp;                 /* ranks in the ring, >= 1 */
+  int32_t layout;             /* cbv_layout */
+  float scale;
+  int32_t window;
+  float* out_acc;             /* forward: device f32 [n_local, num_heads, head_dim], running out */
+  float* lse_acc;             /* forward: device f32 [num_heads, n_local], running lse */
+  void* out;                  /* forward: NULL, or device bf16 [n_local, num_heads, head_dim] */
+  const void* dout;           /* backward: device bf16 [n_local, num_heads, head_dim] */
+  const void* out_merged;     /* backward: device bf16, this rank's merged forward output */
+  const float* lse_merged;    /* backward: device f32 [num_heads, n_local], this rank's merged lse */
+  float* dq_acc;              /* backward: device f32 [n_local, num_heads, head_dim], += */
+  float* dk_acc;              /* backward: device f32 [n_local, num_kv_heads, head_dim] of src's rows, += */
+  float* dv_acc;
+  void* workspace;
+  size_t workspace_bytes;
+} cbv_ring_step_args;
+size_t cbv_ring_step_fwd_workspace_size(const cbv_ring_step_args* a);
+int cbv_ring_step_fwd(const cbv_ring_step_args* a, void* stream);
+size_t cbv_ring_step_bwd_workspace_size(const cbv_ring_step_args* a);
+int cbv_ring_step_bwd(const cbv_ring_step_args* a, void* stream);
+
 /* ========================================================================= EAGLE-3 cached ring
  * NeMo AutoModel ring_attention, _CachedZigZagRingAttention / cached_zigzag_ring_attention
  * (layout = CBV_LAYOUT_ZIGZAG) and _CachedRingAttention / cached_ring_attention
@@ -319,6 +370,52 @@ size_t cbv_cached_ring_fwd_workspace_size(const cbv_cached_ring_args* a);
 int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream);
 size_t cbv_cached_ring_bwd_workspace_size(const cbv_cached_ring_args* a);
 int cbv_cached_ring_bwd(const cbv_cached_ring_args* a, void* stream);
+
+/* ========================================================================= cache diagonals alone
+ * The per-position diagonals of the EAGLE-3 cache (blocks 1..num_blocks-1, as in
+ * cbv_cached_ring_fwd / _bwd) applied to a block-0 result computed elsewhere: by Ulysses
+ * (ulysses_attention._CachedUlyssesAttention: block 0 over the all-to-all-gathered sequence, the
+ * diagonals merged shard-locally, comm-free) or by any caller.  Rows are independent, so the
+ * tokens may be any slice of a sequence.  With num_blocks == 1 both calls only round.
+ * cbv_cached_diag_merge: out0 is block 0's NORMALISED fp32 output [total, H, D] and lse holds
+ *   block 0's lse [H, total] on entry; the merged lse replaces it and the merged output is
+ *   rounded into out (bf16).
+ * cbv_cached_diag_grad: fed the MERGED out / lse, writes dq = dq0 (block 0's fp32 dq) + the
+ *   diagonal terms (bf16) and the gradients of blocks 1..num_blocks-1 into dcache_k / dcache_v
+ *   (entries 0 are not touched). */
+typedef struct cbv_diag_args {
+  uint32_t struct_size;        /* sizeof(cbv_diag_args) */
+  uint32_t abi_version;        /* CBV_ABI_VERSION */
+  const void* q;               /* device bf16 [total, num_heads, head_dim] */
+  const void* const* cache_k;  /* host array [num_blocks] of device bf16 [total, num_kv_heads, head_dim]; [0] unused */
+  const void* const* cache_v;
+  int32_t num_blocks;          /* 1..8 */
+  int64_t total;
+  int32_t num_heads, num_kv_heads, head_dim;
+  float scale;
+  const float* out0;           /* merge: device f32 [total, num_heads, head_dim], block 0 normalised */
+  float* lse;                  /* merge: device f32 [num_heads, total], block 0's lse in, merged lse out */
+  void* out;                   /* merge: device bf16 [total, num_heads, head_dim] */
+  const void* dout;            /* grad: device bf16 [total, num_heads, head_dim] */
+  const void* out_merged;      /* grad: device bf16, merged output */
+  const float* lse_merged;     /* grad: device f32 [num_heads, total] */
+  const float* dq0;            /* grad: device f32 [total, num_heads, head_dim], block 0's dq */
+  void* dq;                    /* grad: device bf16 [total, num_heads, head_dim] */
+  void* const* dcache_k;       /* grad: host array [num_blocks] of device bf16 outputs; [0] unused */
+  void* const* dcache_v;
+} cbv_diag_args;
+int cbv_cached_diag_merge(const cbv_diag_args* a, void* stream);
+int cbv_cached_diag_grad(const cbv_diag_args* a, void* stream);
+
+/* ========================================================================= layout helpers
+ * cbv_convert_f32_bf16: dst[i] = bf16_rne(src[i] * mul), n elements (n a multiple of 4, both
+ *   16-byte aligned): the finalise of an fp32 accumulator.
+ * cbv_swap_leading_axes: dst [b][a][row] = src [a][b][row] for an array of a * b rows of
+ *   row_bytes bytes (a multiple of 4): the reordering on either side of an all-to-all that turns
+ *   sequence shards into head shards and back (ulysses_attention._gather_seq_scatter_heads,
+ *   _scatter_seq_gather_heads, _gather_lse, _scatter_lse).  src and dst must not overlap. */
+int cbv_convert_f32_bf16(const float* src, void* dst, int64_t n, float mul, void* stream);
+int cbv_swap_leading_axes(const void* src, void* dst, int64_t a, int64_t b, int64_t row_bytes, void* stream);
 
 /* ========================================================================= block backward
  * One block's backward fed the MERGED softmax statistics (zigzag_ring_attention._block_backward;

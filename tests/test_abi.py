@@ -34,7 +34,7 @@ def test_struct_layouts_match_the_c_compiler():
     structs = {"cbv_block_fwd_args": cbv.BlockFwdArgs, "cbv_ring_args": cbv.RingArgs,
                "cbv_block_bwd_args": cbv.BlockBwdArgs, "cbv_kvp_args": cbv.KvpArgs, "cbv_decode_args": cbv.DecodeArgs,
                "cbv_cached_ring_args": cbv.CachedRingArgs, "cbv_ring_block": cbv.RingBlock,
-               "cbv_row_run": cbv.RowRun}
+               "cbv_row_run": cbv.RowRun, "cbv_ring_step_args": cbv.RingStepArgs, "cbv_diag_args": cbv.DiagArgs}
     src = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
     for cname, st in structs.items():
         src.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
@@ -389,4 +389,48 @@ def test_stalled_forward_diagnostic_checks_its_limit_before_any_launch():
     a.schedule = cbv.SCHEDULE_STEPWISE
     assert cbv.STATUS[L.cbv_debug_ring_fwd_stalled(ctypes.byref(a), 1_000_000, None)] == "BAD_ARG"
     assert cbv.launch_count() == n0
+
+
+def _step_args(**kw):
+    cu = kw.pop("cu", np.array([0, 96, 256], np.int32))
+    a = cbv.RingStepArgs(struct_size=ctypes.sizeof(cbv.RingStepArgs), abi_version=cbv.ABI_VERSION, rank=0, step=0,
+                         n_local=int(cu[-1]) // 2, num_heads=2, num_kv_heads=2, head_dim=64, num_docs=len(cu) - 1,
+                         cu_seqlens=cu.ctypes.data_as(cbv.c_i32p), cp=2)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a, cu
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("rank", 2, "BAD_ARG"), ("step", -1, "BAD_ARG"), ("cp", 0, "BAD_ARG"), ("n_local", 100, "BAD_CU_SEQLENS"),
+    ("head_dim", 96, "UNSUPPORTED_HEAD_DIM"), ("num_kv_heads", 3, "GQA_MISMATCH"), ("abi_version", 3, "VERSION"),
+    ("layout", 5, "BAD_ARG"),
+])
+def test_ring_step_argument_errors_are_reported_before_any_launch(field, value, status):
+    a, cu = _step_args(**{field: value})
+    L = cbv.lib()
+    n0 = cbv.launch_count()
+    for fn in (L.cbv_ring_step_fwd, L.cbv_ring_step_bwd):
+        assert cbv.STATUS[fn(ctypes.byref(a), None)] == status
+    assert L.cbv_ring_step_fwd_workspace_size(ctypes.byref(a)) == 0
+    assert cbv.launch_count() == n0
+
+
+def test_ring_step_workspace_sizes_are_reported():
+    a, cu = _step_args()
+    L = cbv.lib()
+    assert L.cbv_ring_step_fwd_workspace_size(ctypes.byref(a)) > 256
+    assert L.cbv_ring_step_bwd_workspace_size(ctypes.byref(a)) > 256
+
+
+def test_diag_and_layout_helper_errors():
+    L = cbv.lib()
+    a = cbv.DiagArgs(struct_size=ctypes.sizeof(cbv.DiagArgs), abi_version=cbv.ABI_VERSION, num_blocks=9, total=4,
+                     num_heads=2, num_kv_heads=2, head_dim=64)
+    assert cbv.STATUS[L.cbv_cached_diag_merge(ctypes.byref(a), None)] == "BAD_ARG"
+    a.num_blocks, a.head_dim = 2, 80
+    assert cbv.STATUS[L.cbv_cached_diag_grad(ctypes.byref(a), None)] == "UNSUPPORTED_HEAD_DIM"
+    assert cbv.STATUS[L.cbv_convert_f32_bf16(None, None, 6, 1.0, None)] == "BAD_SHAPE"
+    assert cbv.STATUS[L.cbv_swap_leading_axes(None, None, 2, 2, 6, None)] == "BAD_SHAPE"
+    assert L.cbv_swap_leading_axes(None, None, 0, 2, 8, None) == 0  # nothing to move
 
