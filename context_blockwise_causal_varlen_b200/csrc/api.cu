@@ -566,8 +566,8 @@ static int kvp_checks(const cbv_kvp_args* a) {
   if (a->q_len < 0 || a->shards < 1 || a->blocks_per_shard < 1 || a->num_blocks < 1)
     return fail(CBV_ERR_BAD_SHAPE, "bad q_len / shards / blocks");
   const int bs = a->block_size;
-  if (bs < 8 || bs > 128 || 128 % bs) return fail(CBV_ERR_BAD_ARG, "block_size must divide 128 and be >= 8");
-  if (a->seg_size <= 0 || a->seg_size % 128) return fail(CBV_ERR_BAD_ARG, "seg_size must be a positive multiple of 128");
+  if (bs < 8 || bs > 128 || 128 % bs) return fail(CBV_ERR_BAD_ARG, "block_size must be a power of two in [8, 128]");
+  if (a->seg_size <= 0) return fail(CBV_ERR_BAD_ARG, "seg_size must be positive");
   if (a->kv_mode != CBV_KV_CONTIGUOUS && a->kv_mode != CBV_KV_ROUND_ROBIN) return fail(CBV_ERR_BAD_ARG, "bad kv_mode");
   if (a->global_q_offset < 0) return fail(CBV_ERR_BAD_ARG, "global_q_offset must be >= 0");
   if (!aligned16(a->q) || !aligned16(a->k_cache) || !aligned16(a->v_cache) || !aligned16(a->out))
@@ -599,10 +599,15 @@ static int kvp_tail_tasks(const Plan& plan) {
   return w >= kMinSplitWork * tail ? tail : 0;
 }
 
+// The segment length the kernel walks: seg_size rounded up to whole 128-key tiles, so that every
+// k tile starts on a page boundary.  The result does not depend on the segment length (the
+// segments are merged by the online-softmax identity), only the order of the merges does.
+static int32_t kvp_segment(int32_t seg_size) { return (int32_t)std::min<int64_t>(((int64_t)seg_size + 127) / 128 * 128, INT32_MAX / 2); }
+
 static size_t kvp_layout(const cbv_kvp_args* a, Plan* plan_out, int* tail_out) {
   const int n_local = a->blocks_per_shard * a->block_size;
-  Plan plan = plan_kvp(a->q_len, a->num_heads, a->shards, n_local, a->seg_size, (KvMode)a->kv_mode, a->block_size,
-                       a->global_q_offset, a->sliding_window, a->shard_out != nullptr, kPairRows);
+  Plan plan = plan_kvp(a->q_len, a->num_heads, a->shards, n_local, kvp_segment(a->seg_size), (KvMode)a->kv_mode,
+                       a->block_size, a->global_q_offset, a->sliding_window, a->shard_out != nullptr, kPairRows);
   const int tail = a->shard_out ? 0 : kvp_tail_tasks(plan);
   Carve c(nullptr);
   c.take(kStatusBytes);

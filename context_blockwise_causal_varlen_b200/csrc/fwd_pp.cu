@@ -369,18 +369,32 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           for (int c = 0; c < BN; ++c)
             if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
         } else if (need_mask) {
-          // round-robin pages: position = page base + offset inside the page (shifts: the
-          // block size is a power of two)
+          // round-robin pages: column c sits at kpos0 + delta(c), delta(c) = (c / bs) * shards * bs
+          // + c % bs, which grows with c, so the columns a row sees are again one range [lo, hi]:
+          // invert delta at the row's two bounds (two divisions per row instead of a position per
+          // score)
           const int lbs = __ffs(p.block_size) - 1;
-          const int32_t page_stride = p.shards << lbs, in_page = p.block_size - 1;
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int32_t kpos = r.kpos0 + (c >> lbs) * page_stride + (c & in_page);
-            bool vis = c < r.nvalid;
-            if (cz) vis = vis && (kpos <= qpos);
-            if (W > 0) vis = vis && (qpos - kpos < W);
-            if (!vis) s[c] = __float_as_uint(-INFINITY);
+          const int32_t bs = p.block_size, page_stride = p.shards << lbs;
+          int32_t hi = r.nvalid - 1, lo = 0;
+          if (cz) {
+            const int32_t x = qpos - r.kpos0;  // largest visible delta
+            if (x < 0) {
+              hi = -1;
+            } else {
+              const int32_t pg = x / page_stride, off = x - pg * page_stride;
+              hi = min(hi, off >= bs ? ((pg + 1) << lbs) - 1 : (pg << lbs) + off);
+            }
           }
+          if (W > 0) {
+            const int32_t x = qpos - W + 1 - r.kpos0;  // smallest visible delta
+            if (x > 0) {
+              const int32_t pg = x / page_stride, off = x - pg * page_stride;
+              lo = max(lo, off >= bs ? (pg + 1) << lbs : (pg << lbs) + off);
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
         }
         // row maximum of the raw scores (the scale is positive, so it commutes)
         // eight independent chains (the max is exact in any order), so the reduction sits on the

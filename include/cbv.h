@@ -464,7 +464,10 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream);
  * softmax: across segments and shards on chip in one launch (shard_out == NULL), or per
  * shard into shard_out / shard_lse for a later cbv_attn_merge (shard_out != NULL).
  * GQA: q head h reads kv head h / (num_heads / num_kv_heads).
- * Requirements: block_size divides 128 and is >= 8; seg_size is a multiple of 128. */
+ * Requirements: block_size is a power of two in [8, 128] (a page is whole 8-row atoms of the
+ * 128-byte-swizzled tiles the tensor cores read, and a 128-key tile is whole pages); seg_size > 0,
+ * rounded up to a multiple of 128 (whole key tiles): a performance parameter only, since the
+ * segments are merged by the online-softmax identity and the result does not depend on it. */
 typedef struct cbv_kvp_args {
   uint32_t struct_size;
   uint32_t abi_version;

@@ -239,7 +239,9 @@ def test_kvp_rejects_bad_block_and_segment_sizes():
                     num_kv_heads=2, head_dim=128, num_blocks=8, block_size=24, shards=2, blocks_per_shard=4,
                     seg_size=512)
     assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"
-    a.block_size, a.seg_size = 32, 100
+    a.block_size, a.seg_size = 32, 0
+    assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"
+    a.block_size, a.seg_size = 4, 512
     assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)] == "BAD_ARG"
 
 

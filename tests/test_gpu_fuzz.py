@@ -130,7 +130,7 @@ def test_random_paged_prefill_matches_oracle(seed):
     hq, hkv = [(4, 1), (8, 2), (4, 4), (12, 3)][int(rng.integers(0, 4))]
     D = int(rng.choice([64, 128]))
     mode = PG.ROUND_ROBIN if rng.random() < 0.6 else PG.CONTIGUOUS
-    seg = int(rng.choice([128, 256, 512]))
+    seg = int(rng.choice([128, 256, 512, 100, 300, 1]))  # any positive length (rounded up to whole key tiles)
     window = int(rng.choice([0, 0, 1 + int(rng.integers(0, 600))]))
     kv_len = R * bps * bs
     S = int(rng.integers(1, min(kv_len, 400) + 1))
