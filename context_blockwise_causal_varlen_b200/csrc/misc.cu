@@ -116,7 +116,14 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (c == 0) rows[h * t_pad + tok] = make_float2(lse[h * total + tok] * 1.4426950408889634f, s);
+  if (c == 0) {
+    // A row that sees no key at all has lse = -inf; it is masked in every block, and storing a
+    // finite value keeps exp2(-inf - lse) at 0 in the backward's masked tiles.  The pad rows
+    // [total, t_pad) are zeroed: a row box may read them.
+    const float l = lse[h * total + tok];
+    rows[h * t_pad + tok] = make_float2(l == -INFINITY ? 0.f : l * 1.4426950408889634f, s);
+    for (int64_t e = total + tok; e < t_pad; e += total) rows[h * t_pad + e] = make_float2(0.f, 0.f);
+  }
 }
 
 __global__ void __launch_bounds__(256) convert_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
