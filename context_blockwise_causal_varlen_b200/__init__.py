@@ -14,7 +14,9 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcbv.so")
+# CBV_LIBRARY=debug selects the bounds-checking build (libcbv_debug.so): its kernels check every row
+# and page index against its tensor, and every call below then also reads the status word back.
+LIB_PATH = os.path.join(_HERE, "libcbv_debug.so" if os.environ.get("CBV_LIBRARY") == "debug" else "libcbv.so")
 ABI_VERSION = 1
 
 ZIGZAG, CONTIGUOUS = 0, 1
@@ -188,7 +190,7 @@ class RingBlock(ctypes.Structure):
 
 
 EXPORTS = [
-    "cbv_last_error_message", "cbv_abi_version", "cbv_read_status", "cbv_launch_count",
+    "cbv_last_error_message", "cbv_abi_version", "cbv_read_status", "cbv_launch_count", "cbv_build_flags",
     "cbv_local_cu_seqlens", "cbv_half_cu_seqlens", "cbv_get_half_index", "cbv_get_half_lse", "cbv_rank_tokens",
     "cbv_rank_pair_counts", "cbv_ring_step", "cbv_plan_zigzag",
     "cbv_block_fwd_workspace_size", "cbv_attn_block_fwd", "cbv_attn_merge",
@@ -208,6 +210,7 @@ def _declare(L):
     L.cbv_last_error_message.restype = ctypes.c_char_p
     L.cbv_abi_version.restype = ctypes.c_int
     L.cbv_launch_count.restype = ctypes.c_size_t
+    L.cbv_build_flags.restype = ctypes.c_int
     L.cbv_read_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
     L.cbv_local_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i32p]
     L.cbv_half_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, c_i32p]
@@ -250,6 +253,22 @@ def _declare(L):
 def _check(rc: int):
     if rc != 0:
         raise CbvError(rc, lib().cbv_last_error_message().decode())
+
+
+def debug_build() -> bool:
+    """True when the loaded library is the bounds-checking build."""
+    return bool(lib().cbv_build_flags() & 1)
+
+
+def _run(fn, args, ws, device):
+    """One library call; in the bounds-checking build, the call's status word is read back (the stream
+    synchronises; not while a CUDA graph is being captured) and a kernel that reported a bad index or gave
+    up a wait raises."""
+    _check(fn(ctypes.byref(args), _stream(device)))
+    if debug_build() and not torch.cuda.is_current_stream_capturing():  # no synchronising inside a capture
+        code = read_status(ws)
+        if code:
+            raise CbvError(-12, f"a kernel reported status 0x{code:x}")
 
 
 def _host_i32(x) -> np.ndarray:
@@ -297,7 +316,10 @@ def _given(t, like_shape, dtype, device, name):
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    # zeroed in the bounds-checking build, whose status check must not read what a call that launched
+    # nothing (an empty problem) left unwritten
+    alloc = torch.zeros if debug_build() else torch.empty
+    return alloc(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def _header(st):
@@ -435,7 +457,7 @@ def zigzag_ring_fwd(q, k, v, cu_seqlens, cp: int, scale=None, window: int = 0, l
                  out=_ptr(out), lse=_ptr(lse))
     ws = _given_workspace(workspace, lib().cbv_zigzag_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_zigzag_ring_fwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_zigzag_ring_fwd, a, ws, q.device)
     return (out, lse, ws) if return_workspace else (out, lse)
 
 
@@ -465,7 +487,7 @@ def zigzag_ring_bwd(dout, q, k, v, out, lse, cu_seqlens, cp: int, scale=None, wi
                  dq=_ptr(dq), dk=_ptr(dk), dv=_ptr(dv))
     ws = _given_workspace(workspace, lib().cbv_zigzag_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_zigzag_ring_bwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_zigzag_ring_bwd, a, ws, q.device)
     return (dq, dk, dv, ws) if return_workspace else (dq, dk, dv)
 
 
@@ -517,7 +539,7 @@ def cached_ring_fwd(q, cache_k, cache_v, cu_seqlens, cp: int, scale=None, window
     a, keep = _cached_args(q, ck, cv, cu, cp, scale, window, layout, max_seqlen, out=out, lse=lse)
     ws = _workspace(lib().cbv_cached_ring_fwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_cached_ring_fwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_cached_ring_fwd, a, ws, q.device)
     return (out, lse, ws) if return_workspace else (out, lse)
 
 
@@ -557,7 +579,7 @@ def cached_ring_bwd(dout, q, cache_k, cache_v, out, lse, cu_seqlens, cp: int, sc
                            deterministic=deterministic, out=out, lse=lse, dout=dout, dq=dq)
     ws = _workspace(lib().cbv_cached_ring_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_cached_ring_bwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_cached_ring_bwd, a, ws, q.device)
     return (dq, dcache_k, dcache_v, ws) if return_workspace else (dq, dcache_k, dcache_v)
 
 
@@ -589,7 +611,7 @@ def attn_block_fwd(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int = 0, sca
                      out_dtype=DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16, out=_ptr(out), lse=_ptr(lse))
     ws = _workspace(lib().cbv_block_fwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_attn_block_fwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_attn_block_fwd, a, ws, q.device)
     return out, lse
 
 
@@ -637,7 +659,7 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
                      dv_acc=_ptr(dv_acc))
     ws = _workspace(lib().cbv_block_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_attn_block_bwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_attn_block_bwd, a, ws, q.device)
     return dq_acc, dk_acc, dv_acc
 
 
@@ -679,7 +701,7 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
         raise CbvError(-4, "q's last dimension must be contiguous")
     ws = _given_workspace(workspace, lib().cbv_kvp_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_kvp_segmented_prefill(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_kvp_segmented_prefill, a, ws, q.device)
     res = [out]
     if return_lse:
         res.append(lse)
@@ -707,7 +729,7 @@ def varlen_decode(q, k, v, cu_seqlens_q, cu_seqlens_k, scale=None, validate=None
         raise CbvError(-9, "cu_seqlens_q and cu_seqlens_k sizes differ")
     ws = _workspace(lib().cbv_decode_workspace_size(ctypes.byref(a)), q.device) if workspace is None else workspace
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_varlen_decode(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_varlen_decode, a, ws, q.device)
     return out
 
 
@@ -736,7 +758,7 @@ def ring_step_fwd(rank: int, step: int, q, k, v, cu_seqlens, cp: int, out_acc, l
     a = _step_args(rank, step, q, k, v, cu, cp, scale, window, layout, out_acc=out_acc, lse_acc=lse_acc, out=out)
     ws = _workspace(lib().cbv_ring_step_fwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_ring_step_fwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_ring_step_fwd, a, ws, q.device)
     return out_acc, lse_acc
 
 
@@ -759,7 +781,7 @@ def ring_step_bwd(rank: int, step: int, dout, q, k, v, out, lse, cu_seqlens, cp:
                    lse_merged=lse.contiguous(), dq_acc=dq_acc, dk_acc=dk_acc, dv_acc=dv_acc)
     ws = _workspace(lib().cbv_ring_step_bwd_workspace_size(ctypes.byref(a)), q.device)
     a.workspace, a.workspace_bytes = _ptr(ws), ws.numel()
-    _check(lib().cbv_ring_step_bwd(ctypes.byref(a), _stream(q.device)))
+    _run(lib().cbv_ring_step_bwd, a, ws, q.device)
     return dq_acc, dk_acc, dv_acc
 
 

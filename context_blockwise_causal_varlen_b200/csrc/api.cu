@@ -256,6 +256,7 @@ FwdParams ring_fwd_params(const cbv_ring_args* a, int* rc) {
   p.lse_stride_h = a->total;
   p.lse_stride_t = 1;
   p.block_size = 1;
+  p.q_rows = p.kv_rows = a->total;
   return p;
 }
 
@@ -271,6 +272,14 @@ const char* cbv_last_error_message(void) { return g_err.c_str(); }
 int cbv_abi_version(void) { return CBV_ABI_VERSION; }
 
 size_t cbv_launch_count(void) { return cbv::launch_count(); }
+
+int cbv_build_flags(void) {
+#ifdef CBV_DEBUG
+  return CBV_BUILD_DEBUG;
+#else
+  return 0;
+#endif
+}
 
 int cbv_read_status(const void* workspace, int* status_out, void* stream) {
   if (!workspace || !status_out) return fail(CBV_ERR_BAD_ARG, "NULL argument");
@@ -448,6 +457,8 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   p.lse_stride_t = 1;
   p.out_mode = a->merge ? kOutMerge : (a->out_dtype == CBV_DTYPE_F32 ? kOutF32 : kOutBf16);
   p.block_size = 1;
+  p.q_rows = a->total_q;
+  p.kv_rows = a->total_k > 0 ? a->total_k : a->total_q;  // without keys the maps describe q
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
@@ -672,6 +683,8 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   p.shards = a->shards;
   p.kv_mode = a->kv_mode;
   p.n_local = a->blocks_per_shard * bs;
+  p.q_rows = a->q_len;
+  p.kv_rows = a->num_blocks;  // pages of the cache
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
@@ -779,6 +792,8 @@ int cbv_varlen_decode(const cbv_decode_args* a, void* stream) {
   p.cu_q = a->cu_seqlens_q;
   p.cu_k = a->cu_seqlens_k;
   p.num_seqs = a->num_seqs;
+  p.total_q = a->total_q;
+  p.total_k = a->total_k;
   p.hq = a->num_heads;
   p.hkv = Hkv;
   p.head_dim = D;
@@ -881,6 +896,7 @@ static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_
   p.dkv_accumulate = 0;
   p.dq_fixed = det ? static_cast<unsigned long long*>(dq_buf) : nullptr;
   p.dq_fixed_tpad = fixed_tpad(a->total);
+  p.q_rows = p.kv_rows = a->total;
   p.prefetch_ahead = sm_count();
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
@@ -961,6 +977,8 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   if ((rc = make_bwd_maps(&p, a->q, a->dout, a->k, a->v, a->dq_acc, a->total_q, a->total_k, H, Hkv, D))) return rc;
   p.dq_fixed = dq_fixed;
   p.dq_fixed_tpad = fixed_tpad(a->total_q);
+  p.q_rows = a->total_q;
+  p.kv_rows = a->total_k;
   p.tasks = pd.tasks;
   p.segs = pd.segs;
   p.num_tasks = (int)plan.tasks.size();
@@ -1218,6 +1236,7 @@ int cbv_ring_step_fwd(const cbv_ring_step_args* a, void* stream) {
   p.lse_stride_t = 1;
   p.out_mode = a->step == 0 ? kOutF32 : kOutMerge;  // every local row takes part in step 0's block
   p.block_size = 1;
+  p.q_rows = p.kv_rows = a->n_local;
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;
@@ -1274,6 +1293,7 @@ int cbv_ring_step_bwd(const cbv_ring_step_args* a, void* stream) {
   p.dkv_stride_h = D;
   p.dkv_accumulate = 1;
   p.prefetch_ahead = sm_count();
+  p.q_rows = p.kv_rows = a->n_local;
   p.status = status;
   if ((rc = zero_status(status, s))) return rc;
   if ((rc = upload_plan(pd, plan, s))) return rc;

@@ -207,13 +207,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_arrive_expect_tx(&bar[bKVFull], 2 * L::kKV);
       for (int h = 0; h < KH; ++h) {
         if (!t.split1) {
-          tma_load_3d(sK + h * 16384, &p.tm_k, &bar[bKVFull], h * 64, kvh, t.row0);
-          tma_load_3d(sV + h * 16384, &p.tm_v, &bar[bKVFull], h * 64, kvh, t.row0);
+          int32_t kr = t.row0;
+          CBV_CHECK_RANGE(kr, 0, p.kv_rows, p.status, kDevBoundsKV);
+          tma_load_3d(sK + h * 16384, &p.tm_k, &bar[bKVFull], h * 64, kvh, kr);
+          tma_load_3d(sV + h * 16384, &p.tm_v, &bar[bKVFull], h * 64, kvh, kr);
         } else {
           // two key ranges: 8-row pieces (1 KB of the 128B-swizzled tile each, so the swizzle
           // pattern stays aligned); every tile row is loaded, from one range or the other
           for (int g = 0; g < BN / 8; ++g) {
-            const int32_t row = g * 8 < t.split1 ? t.row0 + g * 8 : t.row1 + (g * 8 - t.split1);
+            int32_t row = g * 8 < t.split1 ? t.row0 + g * 8 : t.row1 + (g * 8 - t.split1);
+#ifdef CBV_DEBUG
+            // pieces past a range's valid keys may start past the tensor (the copy reads zeros there)
+            if (g * 8 < t.split1 ? g * 8 < t.rows : g * 8 - t.split1 < t.rows1)
+              CBV_CHECK_RANGE(row, 0, p.kv_rows, p.status, kDevBoundsKV);
+#endif
             tma_load_3d(sK + h * 16384 + g * 1024, &p.tm_k8, &bar[bKVFull], h * 64, kvh, row);
             tma_load_3d(sV + h * 16384 + g * 1024, &p.tm_v8, &bar[bKVFull], h * 64, kvh, row);
           }
@@ -229,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!mbar_wait(&bar[bQEmpty + st], ((j / NS) & 1) ^ 1, p.status, kDevTimeoutTmaEmpty)) break;
         uint64_t* full = &bar[bQFull + st];
         mbar_arrive_expect_tx(full, 2 * L::kQT + L::kRowBytes);
+        CBV_CHECK_RANGE(r.q_row, 0, p.q_rows, p.status, kDevBoundsQ);
         for (int h = 0; h < KH; ++h) {
           tma_load_3d(sQ + st * L::kQT + h * 8192, &p.tm_q, full, h * 64, r.head, r.q_row);
           tma_load_3d(sDO + st * L::kQT + h * 8192, &p.tm_do, full, h * 64, r.head, r.q_row);
@@ -329,8 +337,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const bool second = t.split1 && krow >= t.split1;  // this key row belongs to the second range
     const int32_t kpos = second ? t.pos1 + (krow - t.split1) : t.pos0 + krow;
-    const bool kvalid = second ? krow - t.split1 < t.rows1 : krow < t.rows;
+    bool kvalid = second ? krow - t.split1 < t.rows1 : krow < t.rows;
     const int32_t kglobal = second ? t.row1 + (krow - t.split1) : t.row0 + krow;
+#ifdef CBV_DEBUG
+    if (kvalid && (kglobal < 0 || kglobal >= p.kv_rows)) {
+      atomicCAS(p.status, 0, kDevBoundsOut);
+      kvalid = false;
+    }
+#endif
     const int32_t W = p.window;
     const float sl2 = p.scale_log2;
     const uint32_t pt_buf[2] = {smem_u32(sPt), smem_u32(sm + L::kPt1)};
@@ -452,11 +466,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           const int lr = i * RPI + sub;
           const int kr = quarter * 32 + lr;
           const bool sec = t.split1 && kr >= t.split1;
-          const bool valid = sec ? kr - t.split1 < t.rows1 : kr < t.rows;
+          bool valid = sec ? kr - t.split1 < t.rows1 : kr < t.rows;
           uint32_t v4[4];
           ld_shared_v4(stg + lr * (D * 2) + ((unit ^ (lr & (UPR - 1))) << 4), v4);
+          const int64_t kg = sec ? (int64_t)t.row1 + (kr - t.split1) : (int64_t)t.row0 + kr;
+#ifdef CBV_DEBUG
+          if (valid && (kg < 0 || kg >= p.kv_rows)) {
+            atomicCAS(p.status, 0, kDevBoundsOut);
+            valid = false;
+          }
+#endif
           if (valid) {
-            const int64_t kg = sec ? (int64_t)t.row1 + (kr - t.split1) : (int64_t)t.row0 + kr;
             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(dst_base) + kg * p.dkv_stride_t +
                                  (int64_t)kvh * p.dkv_stride_h + unit * 8;
             *reinterpret_cast<uint4*>(dst) = make_uint4(v4[0], v4[1], v4[2], v4[3]);

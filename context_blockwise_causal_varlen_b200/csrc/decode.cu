@@ -77,9 +77,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const __grid_consta
   const uint32_t half_bytes = hpc * L::kHead;
   const uint32_t tile_bytes = (D / 64) * half_bytes;
 
-  const int qrow = __ldg(&p.cu_q[seq]);
-  const int k_start = __ldg(&p.cu_k[seq]);
-  const int k_end = __ldg(&p.cu_k[seq + 1]);
+  int qrow = __ldg(&p.cu_q[seq]);
+  int k_start = __ldg(&p.cu_k[seq]);
+  int k_end = __ldg(&p.cu_k[seq + 1]);
+  // the offsets are read here, not checked on the host (they may change between graph replays): a
+  // sequence whose offsets leave the tensors is reported and skipped
+  const bool bad = qrow < 0 || qrow >= p.total_q || k_start < 0 || k_end > p.total_k || k_end < k_start;
+  if (bad) {
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, kDevBadOffsets);
+    return;
+  }
   const int nkeys = max(0, k_end - k_start);
   const int ntiles = (nkeys + kDecKeys - 1) / kDecKeys;
 

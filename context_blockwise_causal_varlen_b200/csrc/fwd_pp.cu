@@ -199,9 +199,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
       mbar_arrive_expect_tx(&bar[pQFull], (has_b ? 2 : 1) * L::kTile);
-      for (int x = 0; x < (has_b ? 2 : 1); ++x)
-        for (int h = 0; h < QH; ++h)
-          tma_load_3d(sQ + x * L::kTile + h * 16384, &p.tm_q, &bar[pQFull], h * 64, head, t.row0 + x * BM);
+      for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+        int32_t qr = t.row0 + x * BM;
+        CBV_CHECK_RANGE(qr, 0, p.q_rows, p.status, kDevBoundsQ);
+        for (int h = 0; h < QH; ++h) tma_load_3d(sQ + x * L::kTile + h * 16384, &p.tm_q, &bar[pQFull], h * 64, head, qr);
+      }
       KIter it;
       KTile r;
       int i = 0;
@@ -220,13 +222,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           }
           mbar_arrive_expect_tx(full, L::kTile);
           if (!PAGED) {
-            for (int h = 0; h < QH; ++h) tma_load_3d(dst + h * 16384, map, full, h * 64, kvh, r.k_row);
+            int32_t kr = r.k_row;
+            CBV_CHECK_RANGE(kr, 0, p.kv_rows, p.status, kDevBoundsKV);
+            for (int h = 0; h < QH; ++h) tma_load_3d(dst + h * 16384, map, full, h * 64, kvh, kr);
           } else {
             // one box per page of block_size tokens, found through the shard's block table
             const int bs = p.block_size, lbs = __ffs(bs) - 1;
+            int32_t shard = r.shard;
+            CBV_CHECK_RANGE(shard, 0, p.shards, p.status, kDevBoundsPage);
             for (int pg = 0; pg < (BN >> lbs); ++pg) {
               const int blk = min((r.k_row >> lbs) + pg, p.blocks_per_shard - 1);  // k_row: a multiple of 128
-              const int page = __ldg(&p.block_tables[(int64_t)r.shard * p.blocks_per_shard + blk]);
+              int32_t page = __ldg(&p.block_tables[(int64_t)shard * p.blocks_per_shard + blk]);
+              CBV_CHECK_RANGE(page, 0, p.kv_rows, p.status, kDevBoundsPage);
               for (int h = 0; h < QH; ++h) tma_load_4d(dst + h * 16384 + pg * bs * 128, map, full, h * 64, 0, kvh, page);
             }
           }
@@ -486,8 +493,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       const bool has = (l > 0.f) && (m != -INFINITY);
       const float inv_l = (has && lr > 0.f) ? 1.f / lr : 0.f;
       const float lse_b = has ? (m + __log2f(l)) * kLn2 : -INFINITY;
-      const bool valid = trow < t.rows;
+      bool valid = trow < t.rows;
       const int64_t orow = (int64_t)(t.row0 + trow);
+#ifdef CBV_DEBUG
+      if (valid && (orow < 0 || orow >= p.q_rows)) {
+        atomicCAS(p.status, 0, kDevBoundsOut);
+        valid = false;
+      }
+#endif
       const int64_t shard_off = t.aux >= 0 ? (int64_t)t.aux : 0;  // per-shard outputs
       float* lse_ptr = l_base + shard_off * l_sh + (int64_t)head * l_h + orow * l_t;
       float wa = 0.f, wb = 1.f, lse_new = lse_b;

@@ -56,6 +56,9 @@ struct FwdParams {
   // timeout path: no copy or tensor-core operation is ever in flight when the kernel gives up)
   uint64_t wait_limit_ns;
   int32_t withhold_loads;
+  // extents the CBV_DEBUG build checks coordinates against: rows of q / out, rows of k / v (paged:
+  // pages of the cache)
+  int64_t q_rows, kv_rows;
 };
 
 struct BwdParams {
@@ -83,6 +86,7 @@ struct BwdParams {
   // (deterministic mode); null: fp32 reduce-adds through tm_dq.  Layout: see fixed_index().
   unsigned long long* dq_fixed;
   int64_t dq_fixed_tpad;
+  int64_t q_rows, kv_rows;  // extents the CBV_DEBUG build checks rows against
   // > 0: each CTA prefetches into L2 the key and value tile of task blockIdx.x + prefetch_ahead
   // (the SM count: roughly the task that starts on an SM when this wave's CTAs finish)
   int32_t prefetch_ahead;
@@ -167,6 +171,7 @@ struct DecodeParams {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int32_t num_seqs, hq, hkv, head_dim;
+  int64_t total_q, total_k;  // every sequence's offsets are checked against these
   int32_t heads_per_cta;  // kv heads per CTA: 4, 2 or 1, dividing hkv (the TMA box never leaves the tensor)
   float scale_log2;
   int* status;

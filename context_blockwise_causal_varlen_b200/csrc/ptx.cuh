@@ -20,7 +20,30 @@ enum DeviceStatus : int {
   kDevTimeoutMma = 0x103,
   kDevTimeoutSoftmax = 0x104,
   kDevTimeoutEpilogue = 0x105,
+  // a coordinate outside its tensor (checked in CBV_DEBUG builds; decode offsets always)
+  kDevBoundsQ = 0x201,
+  kDevBoundsKV = 0x202,
+  kDevBoundsPage = 0x203,
+  kDevBoundsOut = 0x204,
+  kDevBadOffsets = 0x205,
 };
+
+// Debug builds (CBV_DEBUG) check a row or page index against its extent before the copy or
+// store that uses it; a violation records `code` in the status word and the access goes to the
+// first row instead, so the kernel still ends normally (with wrong values and an error status).
+#ifdef CBV_DEBUG
+#define CBV_CHECK_RANGE(v, lo, hi, status, code)      \
+  do {                                                \
+    if ((v) < (lo) || (v) >= (hi)) {                  \
+      atomicCAS((status), 0, (code));                 \
+      (v) = (lo);                                     \
+    }                                                 \
+  } while (0)
+#else
+#define CBV_CHECK_RANGE(v, lo, hi, status, code) \
+  do {                                           \
+  } while (0)
+#endif
 
 // A stalled wait gives up after this many nanoseconds of device time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

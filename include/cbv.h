@@ -101,6 +101,14 @@ int cbv_read_status(const void* workspace, int* status_out, void* stream);
  * difference across a stretch of calls is exactly what those calls enqueued. */
 size_t cbv_launch_count(void);
 
+/* How the library was built: CBV_BUILD_DEBUG is set in the bounds-checking build (libcbv_debug.so,
+ * compiled with CBV_DEBUG), whose kernels check every row and page index they copy or store
+ * against its tensor and report a violation as a status code 0x201-0x204 (read with
+ * cbv_read_status) instead of touching memory outside the tensor.  The varlen decode checks its
+ * device-side offsets in every build (status 0x205, the sequence is skipped). */
+#define CBV_BUILD_DEBUG 1
+int cbv_build_flags(void);
+
 /* ========================================================================= planner (host only)
  * Integer, exact; all arrays are host memory.  cu_seqlens is GLOBAL, int32 [num_docs+1],
  * natural packed order.  NeMo AutoModel zigzag_ring_attention: module docstring
