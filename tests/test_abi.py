@@ -436,3 +436,13 @@ def test_diag_and_layout_helper_errors():
     assert cbv.STATUS[L.cbv_swap_leading_axes(None, None, 2, 2, 6, None)] == "BAD_SHAPE"
     assert L.cbv_swap_leading_axes(None, None, 0, 2, 8, None) == 0  # nothing to move
 
+
+@pytest.mark.parametrize("seed", range(12))
+def test_block_descriptors_on_random_document_mixes(seed):
+    # random document counts and lengths (multiples of 2 cp, empty documents included) for every cp
+    rng = np.random.default_rng(500 + seed)
+    cp = int(rng.choice([1, 2, 3, 4, 8]))
+    n = int(rng.integers(1, 9))
+    lengths = rng.integers(0, 12, n) * 2 * cp
+    _check_block_descriptors(cu_from_lengths(lengths), cp)
+
