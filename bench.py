@@ -594,23 +594,31 @@ def main():
     pairs = visible_pairs(cu)
     f_fwd, f_bwd = 4 * D * H * pairs, 10 * D * H * pairs
     state = {}
-    ev = {"f0": [], "f1": [], "b1": []}
+    ev = {"f0": [], "f1": [], "b1": [], "kf": [], "kb": []}
+
+    def mark(key):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        ev[key].append(e)
+
+    def kernel_events(key):
+        # the library records this pair around its attention-kernel launch, on the call's stream
+        pair = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        ev[key].append(pair)
+        cbv.set_kernel_events(*pair)
 
     def step(record=False):
         if record:
-            e = torch.cuda.Event(enable_timing=True)
-            e.record()
-            ev["f0"].append(e)
+            mark("f0")
+            kernel_events("kf")
         state["out"], state["lse"] = cbv.zigzag_ring_fwd(q, k, v, cu, cp)
         if record:
-            e = torch.cuda.Event(enable_timing=True)
-            e.record()
-            ev["f1"].append(e)
+            mark("f1")
+            kernel_events("kb")
         state["grads"] = cbv.zigzag_ring_bwd(do, q, k, v, state["out"], state["lse"], cu, cp)
         if record:
-            e = torch.cuda.Event(enable_timing=True)
-            e.record()
-            ev["b1"].append(e)
+            cbv.set_kernel_events()
+            mark("b1")
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -636,6 +644,8 @@ def main():
         dist.barrier()
     fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["f0"], ev["f1"])]))
     bwd_ms = float(np.mean([a.elapsed_time(b) for a, b in zip(ev["f1"], ev["b1"])]))
+    fwd_kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev["kf"]]))
+    bwd_kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in ev["kb"]]))
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     e2e_ms, h2d, d2h = e2e_pipelined(cbv, torch, (q, k, v, do), cu, cp, max(6, args.steps // 2), 2)
@@ -644,7 +654,8 @@ def main():
     value = total_flops / (ms * 1e-3) / 1e12
     if rank == 0:
         # the dominant kernel: the block backward (10 of the 14 flops per pair)
-        dom_ms, dom_flops, dom_name = (bwd_ms, f_bwd, "bwd_kernel") if bwd_ms >= fwd_ms else (fwd_ms, f_fwd, "fwd_pp_kernel")
+        dom_ms, dom_flops, dom_name = ((bwd_kernel_ms, f_bwd, "bwd_kernel") if bwd_kernel_ms >= fwd_kernel_ms
+                                       else (fwd_kernel_ms, f_fwd, "fwd_pp_kernel"))
         achieved = dom_flops / (dom_ms * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -662,9 +673,12 @@ def main():
                          "frac_of_stated_peak": achieved / STATED_PEAKS["bf16_tflops"],
                          "step_frac": value / pk["bf16_tflops"],
                          "step_frac_of_stated_peak": value / STATED_PEAKS["bf16_tflops"],
-                         "note": "duration = CUDA events around the API call on its stream (includes the call's "
-                                 "small helper kernels)"},
-            "phases_ms": {"fwd": fwd_ms, "bwd": bwd_ms},
+                         "duration_ms": dom_ms,
+                         "note": "duration = CUDA events the library records on the call's stream right before "
+                                 "and after the kernel's launch (cbv_set_kernel_events), averaged over the timed "
+                                 "steps"},
+            "phases_ms": {"fwd": fwd_ms, "bwd": bwd_ms, "fwd_kernel": fwd_kernel_ms, "bwd_kernel": bwd_kernel_ms,
+                          "bwd_helpers": bwd_ms - bwd_kernel_ms},
             "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches,

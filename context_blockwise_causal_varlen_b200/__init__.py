@@ -191,6 +191,7 @@ class RingBlock(ctypes.Structure):
 
 EXPORTS = [
     "cbv_last_error_message", "cbv_abi_version", "cbv_read_status", "cbv_launch_count", "cbv_build_flags",
+    "cbv_set_kernel_events",
     "cbv_local_cu_seqlens", "cbv_half_cu_seqlens", "cbv_get_half_index", "cbv_get_half_lse", "cbv_rank_tokens",
     "cbv_rank_pair_counts", "cbv_ring_step", "cbv_plan_zigzag",
     "cbv_block_fwd_workspace_size", "cbv_attn_block_fwd", "cbv_attn_merge",
@@ -211,6 +212,7 @@ def _declare(L):
     L.cbv_abi_version.restype = ctypes.c_int
     L.cbv_launch_count.restype = ctypes.c_size_t
     L.cbv_build_flags.restype = ctypes.c_int
+    L.cbv_set_kernel_events.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     L.cbv_read_status.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]
     L.cbv_local_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, c_i32p]
     L.cbv_half_cu_seqlens.argtypes = [c_i32p, ctypes.c_int32, ctypes.c_int32, c_i32p]
@@ -339,6 +341,21 @@ def _layout(layout) -> int:
 def launch_count() -> int:
     """Kernels the library has launched from this thread so far (diagnostic)."""
     return int(lib().cbv_launch_count())
+
+
+def set_kernel_events(start=None, stop=None) -> None:
+    """Measurement hook for this thread: ``torch.cuda.Event`` ``start`` / ``stop`` are recorded
+    right before and after every attention-kernel launch (forward, backward, decode) until
+    cleared with ``set_kernel_events()``.  Events not yet recorded are recorded once on the
+    current stream first, which creates them."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if not ev.cuda_event:
+            ev.record()
+        return ctypes.c_void_p(ev.cuda_event)
+
+    _check(lib().cbv_set_kernel_events(handle(start), handle(stop)))
 
 
 def read_status(workspace: torch.Tensor) -> int:

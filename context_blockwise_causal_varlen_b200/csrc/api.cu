@@ -273,6 +273,11 @@ int cbv_abi_version(void) { return CBV_ABI_VERSION; }
 
 size_t cbv_launch_count(void) { return cbv::launch_count(); }
 
+int cbv_set_kernel_events(void* start_event, void* stop_event) {
+  cbv::set_kernel_events(static_cast<cudaEvent_t>(start_event), static_cast<cudaEvent_t>(stop_event));
+  return CBV_OK;
+}
+
 int cbv_build_flags(void) {
 #ifdef CBV_DEBUG
   return CBV_BUILD_DEBUG;

@@ -575,7 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
       ++j;
     }
-    if (lane == 0) bulk_wait_group<0>();
+    // the staging buffers must outlive only the reads of the last reduces; their additions into the
+    // accumulator are complete when the grid is, before any later kernel on the stream reads it
+    if (lane == 0) bulk_wait_group_read<0>();
   }
 
   tc_fence_before();
@@ -589,8 +591,11 @@ int launch_bwd_t(const BwdParams& p, int grid, cudaStream_t stream) {
   const uint32_t smem = BwdSmem<D>::kDynamic;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
+  if (const int ev = kernel_event_start(stream)) return ev;
   kern<<<grid, kThreads, smem, stream>>>(p);
-  return launched();
+  const int rc = launched();
+  if (rc) return rc;
+  return kernel_event_stop(stream);
 }
 
 }  // namespace

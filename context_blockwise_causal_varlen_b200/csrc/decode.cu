@@ -282,8 +282,11 @@ int launch_decode_t(const DecodeParams& p, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
   dim3 grid(p.num_seqs, p.hkv / p.heads_per_cta);
+  if (const int ev = kernel_event_start(stream)) return ev;
   kern<<<grid, kDecThreads, smem, stream>>>(p);
-  return launched();
+  const int rc = launched();
+  if (rc) return rc;
+  return kernel_event_stop(stream);
 }
 
 }  // namespace

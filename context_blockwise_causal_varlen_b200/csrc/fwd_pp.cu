@@ -593,8 +593,11 @@ int launch_pp_t(const FwdParams& p, int grid, cudaStream_t stream) {
   const uint32_t smem = PPSmem<D>::kDynamic;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return (int)e;
+  if (const int ev = kernel_event_start(stream)) return ev;
   kern<<<grid, kThreads, smem, stream>>>(p);
-  return launched();
+  const int rc = launched();
+  if (rc) return rc;
+  return kernel_event_stop(stream);
 }
 
 }  // namespace

@@ -13,6 +13,12 @@ namespace cbv {
 // the calling thread (cbv_launch_count) and returns the launch's error code.
 int launched();
 size_t launch_count();
+// Measurement hook (cbv_set_kernel_events): when set for the calling thread, the attention kernels
+// (forward, backward, decode) record the start event on their stream right before their launch and
+// the stop event right after it.  Both return the record's error code (0 when no hook is set).
+void set_kernel_events(cudaEvent_t start, cudaEvent_t stop);
+int kernel_event_start(cudaStream_t stream);
+int kernel_event_stop(cudaStream_t stream);
 
 // Output modes of the forward kernel's epilogue.
 enum OutMode : int32_t {

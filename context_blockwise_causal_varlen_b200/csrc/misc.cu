@@ -386,7 +386,17 @@ int launch_convert_bf16_transposed(const float* src, void* dst, int H, int64_t S
 
 namespace {
 thread_local size_t g_launches = 0;
+thread_local cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;
 }
+
+void set_kernel_events(cudaEvent_t start, cudaEvent_t stop) {
+  g_ev_start = start;
+  g_ev_stop = stop;
+}
+
+int kernel_event_start(cudaStream_t stream) { return g_ev_start ? (int)cudaEventRecord(g_ev_start, stream) : 0; }
+
+int kernel_event_stop(cudaStream_t stream) { return g_ev_stop ? (int)cudaEventRecord(g_ev_stop, stream) : 0; }
 
 int launched() {
   ++g_launches;

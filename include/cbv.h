@@ -101,6 +101,16 @@ int cbv_read_status(const void* workspace, int* status_out, void* stream);
  * difference across a stretch of calls is exactly what those calls enqueued. */
 size_t cbv_launch_count(void);
 
+/* Measurement hook, per calling thread.  While set, every launch of an attention kernel (the
+ * forward kernel of the ring, block, cached and paged forwards, the backward kernel, the decode
+ * kernel) records `start_event` on the call's stream right before the launch and `stop_event`
+ * right after it, so cudaEventElapsedTime gives that kernel's device time without the call's
+ * helper kernels.  In a call that launches several attention kernels (the stepwise schedule)
+ * the events bracket the last one.  The events are caller-owned cudaEvent_t handles; NULL, NULL
+ * clears the hook.  Returns CBV_OK; a failed record makes the call that launched return
+ * CBV_ERR_CUDA. */
+int cbv_set_kernel_events(void* start_event, void* stop_event);
+
 /* How the library was built: CBV_BUILD_DEBUG is set in the bounds-checking build (libcbv_debug.so,
  * compiled with CBV_DEBUG), whose kernels check every row and page index they copy or store
  * against its tensor and report a violation as a status code 0x201-0x204 (read with

@@ -143,3 +143,31 @@ def test_each_call_launches_its_schedule_upload_and_kernels():
     n2 = cbv.launch_count()
     sync()
     assert n1 - n0 == 2 and n2 - n1 == 4
+
+
+def test_kernel_events_bracket_the_attention_kernels_only():
+    # the measurement hook records the caller's events around the attention kernel of each call:
+    # they lie inside events taken around the whole call, and clearing the hook stops the records
+    cu, q, k, v, do = _case(7, [2048, 1024], 4, 4, 128)
+    args = (dev(q), dev(k), dev(v), cu, 2)
+    out, lse = cbv.zigzag_ring_fwd(*args)
+    sync()
+    call = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    kern = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for fn in (lambda: cbv.zigzag_ring_fwd(*args),
+               lambda: cbv.zigzag_ring_bwd(dev(do), dev(q), dev(k), dev(v), out, lse, cu, 2)):
+        cbv.set_kernel_events(*kern)
+        call[0].record()
+        fn()
+        call[1].record()
+        cbv.set_kernel_events()
+        sync()
+        whole, inner = call[0].elapsed_time(call[1]), kern[0].elapsed_time(kern[1])
+        assert 0 < inner <= whole
+        assert call[0].elapsed_time(kern[0]) >= 0 and kern[1].elapsed_time(call[1]) >= 0
+    # cleared: a further call records nothing, so the stop event stays before it
+    mark = torch.cuda.Event(enable_timing=True)
+    mark.record()
+    cbv.zigzag_ring_fwd(*args)
+    sync()
+    assert kern[1].elapsed_time(mark) >= 0
