@@ -388,27 +388,38 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[bSFree]);
+        bool skip = false;  // no row of this warp sees any of its 32 q columns
         if (r.need_mask) {
           // this key row sees the q columns [lo, hi] (positions are linear in the column).  The
           // others get a score of -inf and then the same arithmetic as visible ones: every
           // {lse * log2e, Delta} the row box delivers is finite (rows with no visible key store 0,
-          // pad rows are zero, past the tensor the box reads zeros), so P and dS come out 0
+          // pad rows are zero, past the tensor the box reads zeros), so P and dS come out 0.
+          // A warp whose rows all see every column skips the mask, one whose rows see none skips
+          // the arithmetic too (its P and dS are zeros).
           int32_t hi = kvalid ? r.nvalid - 1 : -1, lo = 0;
           if (r.causal || W > 0) lo = max(lo, kpos - r.qpos0);
           if (W > 0) hi = min(hi, kpos + W - 1 - r.qpos0);
           lo -= c0;
           hi -= c0;
+          skip = __all_sync(0xffffffffu, hi < 0 || lo > 31 || hi < lo);
+          if (!skip && !__all_sync(0xffffffffu, lo <= 0 && hi >= 31)) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 32; ++c)
+              if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
+          }
         }
+        if (skip) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float2 r0 = lrow[c], r1 = lrow[c + 1];
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -r0.x));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -r1.x));
-          pp[c / 2] = pack_bf16x2(p0, p1);
-          pd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - r0.y), p1 * (__uint_as_float(dp[c + 1]) - r1.y));
+          for (int c = 0; c < 16; ++c) pp[c] = pd[c] = 0u;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float2 r0 = lrow[c], r1 = lrow[c + 1];
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -r0.x));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -r1.x));
+            pp[c / 2] = pack_bf16x2(p0, p1);
+            pd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - r0.y), p1 * (__uint_as_float(dp[c + 1]) - r1.y));
+          }
         }
       }
       // buffer j & 1 was last read by the UMMAs of q tile j - 2
