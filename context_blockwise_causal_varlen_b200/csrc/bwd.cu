@@ -16,10 +16,11 @@
 // Warps: 0 TMA producer (q, dO, lse*log2e and Delta rows of a 3-stage ring),
 // 1 UMMA issuer (+ TMEM owner; the whole warp runs the loop, one elected lane issues), 2-9 P / dS in two warpgroups that split the 64
 // q columns (one key row per thread) and then the dV / dK epilogue, 10-13 dQ readout.
-// TMEM columns: S^T [0,64), dP^T [64,128), dQ^T [128,192), V [192, 192+D/2), dV [256,256+D),
-// dK [384,384+D).  V sits in TMEM (copied once from shared memory) as the A operand of
-// dP^T = V dO^T, so that product reads only dO from shared memory: the five UMMAs of a
-// q tile are limited by shared-memory bandwidth, and this one then needs a third of it.
+// TMEM columns: S^T [0,64), dP^T [64,128), dQ^T [128,192), P^T [192,256) (two buffers of 32 columns,
+// bf16 pairs), dV [256,256+D), dK [384,384+D).  P^T goes from the softmax warps' registers straight
+// into TMEM as the A operand of dV = P^T dO: a store to shared memory would have to complete before
+// the hand-off to the UMMA issuer, and those stores, not the UMMAs' operand reads, are what the
+// shared memory spends its time on.  dS^T still goes to shared memory: it is also dQ^T's B operand.
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -98,23 +99,17 @@ template <int D>
 struct BwdSmem {
   static constexpr uint32_t kKV = BN * D * 2;   // K or V tile (128 x D)
   static constexpr uint32_t kQT = BM * D * 2;   // a q / dO tile (64 x D)
-  static constexpr uint32_t kPT = BN * BM * 2;  // P^T or dS^T (128 x 64)
+  static constexpr uint32_t kPT = BN * BM * 2;  // dS^T (128 x 64)
   static constexpr uint32_t kRowBytes = kRowPairs * 8;  // bytes one row box delivers
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kKV;
   static constexpr uint32_t kQ = kV + kKV;            // NS stages
   static constexpr uint32_t kDO = kQ + NS * kQT;      // NS stages
-  static constexpr uint32_t kPt = kDO + NS * kQT;
-  static constexpr uint32_t kDSt = kPt + kPT;
+  static constexpr uint32_t kDSt = kDO + NS * kQT;       // dS^T, two buffers (q tile j uses j & 1)
+  static constexpr uint32_t kDSt1 = kDSt + kPT;
   static constexpr uint32_t kDQBuf = kDQRows * D * 4;     // fp32 staging buffer: 4 warps x [16][D/4]
-  static constexpr uint32_t kDQ = kDSt + kPT;              // two staging buffers
-  // P^T / dS^T are double-buffered.  The second pair lives in the V tile when it fits
-  // there (V is read from shared memory only once, to copy it into TMEM).
-  static constexpr bool kPdsInV = kKV >= 2 * kPT;
-  static constexpr uint32_t kX = kDQ + 2 * kDQBuf;         // second P^T / dS^T pair when not in V
-  static constexpr uint32_t kPt1 = kPdsInV ? kV : kX;
-  static constexpr uint32_t kDSt1 = kPt1 + kPT;
-  static constexpr uint32_t kRow = kX + (kPdsInV ? 0 : 2 * kPT);  // per stage: lse*log2e and Delta slots
+  static constexpr uint32_t kDQ = kDSt1 + kPT;            // two staging buffers
+  static constexpr uint32_t kRow = kDQ + 2 * kDQBuf;      // per stage: lse*log2e and Delta slots
   static constexpr uint32_t kBars = kRow + NS * kRowSlot * 4;
   static constexpr uint32_t kEnd = kBars + 256;
   static constexpr uint32_t kDynamic = (kEnd + 1024) < 120 * 1024 ? 120 * 1024 : (kEnd + 1024);
@@ -131,7 +126,7 @@ enum BBar {
   bPtFree = 11,  // +P^T / dS^T buffer (2)
   bDQFull = 13,
   bDQFree = 14,
-  bVTmem = 15,
+  bUnused15 = 15,
   bAccDone = 16,
   bBNum = 17
 };
@@ -147,7 +142,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* sV = sm + L::kV;
   uint8_t* sQ = sm + L::kQ;
   uint8_t* sDO = sm + L::kDO;
-  uint8_t* sPt = sm + L::kPt;
   uint8_t* sDSt = sm + L::kDSt;
   float* sDQ = reinterpret_cast<float*>(sm + L::kDQ);
   float* sRow = reinterpret_cast<float*>(sm + L::kRow);  // [stage][66 pairs {lse*log2e, Delta}]
@@ -167,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
     mbar_init(&bar[bDQFull], 1);
     mbar_init(&bar[bDQFree], 4);
-    mbar_init(&bar[bVTmem], 4);
     mbar_init(&bar[bSFull], 1);
     mbar_init(&bar[bSFree], 8);
     mbar_init(&bar[bPFull], 8);
@@ -184,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 64, tDQ = tmem + 128, tV = tmem + 192, tDV = tmem + 256, tDK = tmem + 384;
+  const uint32_t tS = tmem, tDP = tmem + 64, tDQ = tmem + 128, tPt = tmem + 192, tDV = tmem + 256, tDK = tmem + 384;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -256,8 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);        // K as K-major A (S^T)
       const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);    // K^T as MN-major A (dQ^T)
       // P^T / dS^T buffer b of 2 (q tile j uses buffer j & 1)
-      const uint64_t dPt[2] = {sdesc_sw128(smem_u32(sPt), 16, 1024),       // P^T, K-major A (dV)
-                               sdesc_sw128(smem_u32(sm + L::kPt1), 16, 1024)};
+      const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);        // V as K-major A (dP^T)
       const uint64_t dDSt[2] = {sdesc_sw128(smem_u32(sDSt), 16, 1024),     // dS^T, K-major A (dK)
                                 sdesc_sw128(smem_u32(sm + L::kDSt1), 16, 1024)};
       const uint64_t dDSt_mn[2] = {sdesc_sw128(smem_u32(sDSt), 16384, 1024),  // dS^T, MN-major B (dQ^T)
@@ -268,7 +260,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 8192, 1024);    // q as MN-major B (dK)
       const uint64_t dO_mn = sdesc_sw128(smem_u32(sDO), 8192, 1024);   // dO as MN-major B (dV)
       bool ok = mbar_wait_warp(&bar[bKVFull], 0, p.status, kDevTimeoutMma);
-      ok = ok && mbar_wait_warp(&bar[bVTmem], 0, p.status, kDevTimeoutMma);
       tc_fence_after();
       auto issue_sdp = [&](int j) -> bool {
         const int st = j % NS;
@@ -281,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           const uint32_t ao = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t bb = (kk >> 2) * 8192 + (kk & 3) * 32;
           umma_bf16_ss(tS, sdesc_add(dK_k, ao), sdesc_add(bq, bb), id_st, kk > 0);
-          umma_bf16_ts(tDP, tV + kk * 8, sdesc_add(bo, bb), id_st, kk > 0);
+          umma_bf16_ss(tDP, sdesc_add(dV_k, ao), sdesc_add(bo, bb), id_st, kk > 0);
         }
         umma_commit(&bar[bSFull]);
         return true;
@@ -304,12 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!mbar_wait_warp(&bar[bPFull + pb], (j >> 1) & 1, p.status, kDevTimeoutMma)) { ok = false; break; }
         tc_fence_after();
         const uint64_t omn = sdesc_add(dO_mn, st * L::kQT), qmn = sdesc_add(dQ_mn, st * L::kQT);
-        const uint64_t apt = pb ? dPt[1] : dPt[0], ads = pb ? dDSt[1] : dDSt[0];
+        const uint64_t ads = pb ? dDSt[1] : dDSt[0];
         const uint64_t bds = pb ? dDSt_mn[1] : dDSt_mn[0];
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16_ss(tDV, sdesc_add(apt, kk * 32), sdesc_add(omn, kk * 2048), id_kv, acc);
+          umma_bf16_ts(tDV, tPt + pb * 32 + kk * 8, sdesc_add(omn, kk * 2048), id_kv, acc);
           umma_bf16_ss(tDK, sdesc_add(ads, kk * 32), sdesc_add(qmn, kk * 2048), id_kv, acc);
         }
         if (!mbar_wait_warp(&bar[bDQFree], (j & 1) ^ 1, p.status, kDevTimeoutMma)) { ok = false; break; }
@@ -347,27 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 #endif
     const int32_t W = p.window;
     const float sl2 = p.scale_log2;
-    const uint32_t pt_buf[2] = {smem_u32(sPt), smem_u32(sm + L::kPt1)};
     const uint32_t ds_buf[2] = {smem_u32(sDSt), smem_u32(sm + L::kDSt1)};
     bool ok = true;
-    if (wg == 0) {
-      // V rows (this thread's key) from the swizzled tile into TMEM, as the A operand of dP^T
-      ok = mbar_wait_warp(&bar[bKVFull], 0, p.status, kDevTimeoutSoftmax);
-      if (ok) {
-        const uint32_t vrow = smem_u32(sV);
-#pragma unroll
-        for (int h = 0; h < KH; ++h) {
-          uint32_t vals[32];
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) ld_shared_v4(vrow + h * 16384 + sw128_offset(krow, ch), vals + ch * 4);
-          tmem_st32(tV + lane_base + h * 32, vals);
-        }
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[bVTmem]);
-    }
     QIter it;
     QTile r;
     int j = 0;
@@ -428,13 +400,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         ok = false;
         break;
       }
-      const uint32_t pt_row = pb ? pt_buf[1] : pt_buf[0], ds_row = pb ? ds_buf[1] : ds_buf[0];
+      // P^T: this key row's 32 q columns as 16 bf16 pairs, columns [c0 / 2, c0 / 2 + 16) of the buffer
+      tmem_st16(tPt + lane_base + pb * 32 + (c0 >> 1), pp);
+      const uint32_t ds_row = pb ? ds_buf[1] : ds_buf[0];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int chunk = (c0 >> 3) + ch;
-        st_shared_v4(pt_row + sw128_offset(krow, chunk), pp[ch * 4], pp[ch * 4 + 1], pp[ch * 4 + 2], pp[ch * 4 + 3]);
-        st_shared_v4(ds_row + sw128_offset(krow, chunk), pd[ch * 4], pd[ch * 4 + 1], pd[ch * 4 + 2], pd[ch * 4 + 3]);
-      }
+      for (int ch = 0; ch < 4; ++ch)
+        st_shared_v4(ds_row + sw128_offset(krow, (c0 >> 3) + ch), pd[ch * 4], pd[ch * 4 + 1], pd[ch * 4 + 2],
+                     pd[ch * 4 + 3]);
+      tmem_st_wait();
+      tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[bPFull + pb]);
