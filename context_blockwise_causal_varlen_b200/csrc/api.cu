@@ -170,16 +170,20 @@ PlanDev carve_plan(Carve& c, const Plan& p) {
 }
 
 // Uploads the compact schedule inside kernel launch parameters (no copy engine, no host wait)
-// and expands the task list on the device.
-int upload_plan(const PlanDev& d, const Plan& p, cudaStream_t s) {
-  if (p.tasks.empty()) return CBV_OK;
-  std::vector<unsigned char> img(d.image_bytes, 0);
-  memcpy(img.data(), p.groups.data(), p.groups.size() * sizeof(PlanGroup));
-  memcpy(img.data() + d.off_tiles, p.tiles.data(), p.tiles.size() * sizeof(TileTask));
-  memcpy(img.data() + d.off_segs, p.segs.data(), p.segs.size() * sizeof(Seg));
-  const int e = launch_schedule(d.image, img.data(), img.size(), d.off_tiles, (int)p.groups.size(), d.tasks,
-                                (int)p.tasks.size(), s);
-  return e ? cuda_fail(e, "uploading the schedule") : CBV_OK;
+// and expands the task list on the device.  With `status`, the call's status word is cleared
+// too: by the schedule launch itself when it is a single one, else by a memset.
+int upload_plan(const PlanDev& d, const Plan& p, cudaStream_t s, int* status = nullptr) {
+  bool cleared = false;
+  if (!p.tasks.empty()) {
+    std::vector<unsigned char> img(d.image_bytes, 0);
+    memcpy(img.data(), p.groups.data(), p.groups.size() * sizeof(PlanGroup));
+    memcpy(img.data() + d.off_tiles, p.tiles.data(), p.tiles.size() * sizeof(TileTask));
+    memcpy(img.data() + d.off_segs, p.segs.data(), p.segs.size() * sizeof(Seg));
+    const int e = launch_schedule(d.image, img.data(), img.size(), d.off_tiles, (int)p.groups.size(), d.tasks,
+                                  (int)p.tasks.size(), status, s, &cleared);
+    if (e) return cuda_fail(e, "uploading the schedule");
+  }
+  return status && !cleared ? zero_status(status, s) : CBV_OK;
 }
 
 int launch_rc(int e, const char* what) { return e == 0 ? CBV_OK : cuda_fail(e, what); }
@@ -465,8 +469,7 @@ int cbv_attn_block_fwd(const cbv_block_fwd_args* a, void* stream) {
   p.q_rows = a->total_q;
   p.kv_rows = a->total_k > 0 ? a->total_k : a->total_q;  // without keys the maps describe q
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s, status))) return rc;
   const int grid = grid_of(plan.tasks.size(), 1);
   if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
   return launch_rc(launch_fwd_pingpong(p, D, false, grid, s), "block forward launch");
@@ -538,11 +541,10 @@ int cbv::ring_fwd_run(const cbv_ring_args* a, const RingFwdLayout& L, void* work
   p.status = status;
   p.wait_limit_ns = wait_limit_ns;
   p.withhold_loads = withhold_loads;
-  if ((rc = zero_status(status, s))) return rc;
   const int D = a->head_dim, H = a->num_heads;
   if (a->schedule == CBV_SCHEDULE_FUSED) {
     PlanDev pd = carve_plan(c, L.fused);
-    if ((rc = upload_plan(pd, L.fused, s))) return rc;
+    if ((rc = upload_plan(pd, L.fused, s, status))) return rc;
     p.tasks = pd.tasks;
     p.segs = pd.segs;
     p.num_tasks = (int)L.fused.tasks.size();
@@ -550,6 +552,7 @@ int cbv::ring_fwd_run(const cbv_ring_args* a, const RingFwdLayout& L, void* work
     p.out_mode = kOutBf16;
     return launch_rc(launch_fwd_pingpong(p, D, false, grid_of(L.fused.tasks.size(), 1), s), "ring forward launch");
   }
+  if ((rc = zero_status(status, s))) return rc;
   std::vector<PlanDev> pds;
   for (auto& pl : L.steps) {
     pds.push_back(carve_plan(c, pl));
@@ -691,8 +694,7 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   p.q_rows = a->q_len;
   p.kv_rows = a->num_blocks;  // pages of the cache
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s, status))) return rc;
   const int grid = grid_of(plan.tasks.size(), 1);
   if (!a->shard_out) {
     p.out = a->out;
@@ -904,8 +906,7 @@ static int ring_bwd_core(const cbv_ring_args* a, cudaStream_t s, float** dq_acc_
   p.q_rows = p.kv_rows = a->total;
   p.prefetch_ahead = sm_count();
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s, status))) return rc;
   if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total, tp, H, D, rows,
                                             det ? nullptr : static_cast<float*>(dq_buf), det ? dq_buf : nullptr,
                                             det ? dq_bytes : 0, s),
@@ -1001,8 +1002,7 @@ int cbv_attn_block_bwd(const cbv_block_bwd_args* a, void* stream) {
   p.dkv_accumulate = 1;
   p.prefetch_ahead = sm_count();
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s, status))) return rc;
   if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out, a->lse, a->total_q, tp, H, D, rows, nullptr, dq_fixed,
                                             fix_bytes, s),
                       "backward preprocess")))
@@ -1120,8 +1120,7 @@ int cbv_cached_ring_fwd(const cbv_cached_ring_args* a, void* stream) {
   FwdParams p = ring_fwd_params(&r, &rc);
   if (rc) return rc;
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, L.fused, s))) return rc;
+  if ((rc = upload_plan(pd, L.fused, s, status))) return rc;
   p.tasks = pd.tasks;
   p.segs = pd.segs;
   p.num_tasks = (int)L.fused.tasks.size();
@@ -1243,8 +1242,7 @@ int cbv_ring_step_fwd(const cbv_ring_step_args* a, void* stream) {
   p.block_size = 1;
   p.q_rows = p.kv_rows = a->n_local;
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s, status))) return rc;
   const int grid = grid_of(plan.tasks.size(), 1);
   if (grid < 0) return fail(CBV_ERR_BAD_SHAPE, "too many tiles");
   if ((rc = launch_rc(launch_fwd_pingpong(p, D, false, grid, s), "ring step forward launch"))) return rc;
@@ -1300,8 +1298,7 @@ int cbv_ring_step_bwd(const cbv_ring_step_args* a, void* stream) {
   p.prefetch_ahead = sm_count();
   p.q_rows = p.kv_rows = a->n_local;
   p.status = status;
-  if ((rc = zero_status(status, s))) return rc;
-  if ((rc = upload_plan(pd, plan, s))) return rc;
+  if ((rc = upload_plan(pd, plan, s, status))) return rc;
   if ((rc = launch_rc(launch_bwd_preprocess(a->dout, a->out_merged, a->lse_merged, a->n_local, tp, H, D, rows, nullptr,
                                             nullptr, 0, s),
                       "backward preprocess")))

@@ -115,9 +115,11 @@ int launch_bwd_preprocess(const void* dout, const void* out, const float* lse, i
 // transfer on the copy engine; this neither blocks nor queues.  dst 16-byte aligned.
 int launch_inline_copy(void* dst, const void* src, size_t bytes, cudaStream_t stream);
 // A schedule image (groups at 0, tiles at off_tiles, then segments) written to image_dst and
-// expanded into `tasks`: one launch when the image fits one payload, else copy + expansion.
+// expanded into `tasks`: one launch when the image fits one payload, else copy + expansion.  The
+// single launch also clears *status (when non-null) and sets *status_cleared; otherwise the caller
+// must clear it.
 int launch_schedule(void* image_dst, const void* image, size_t bytes, size_t off_tiles, int ngroups, TileTask* tasks,
-                    int ntasks, cudaStream_t stream);
+                    int ntasks, int* status, cudaStream_t stream, bool* status_cleared);
 // The task list from its compact form (plan.h: PlanGroup): task i of group g is tile
 // first_tile + (i - first_task) % ntiles with head (i - first_task) / ntiles.
 int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* tiles, TileTask* tasks, int ntasks,

@@ -203,19 +203,25 @@ __global__ void __launch_bounds__(256) inline_copy_kernel(const __grid_constant_
 
 // The usual case, a schedule image that fits one payload: one launch both writes the image to
 // the workspace (block 0) and expands the task list, reading the groups and tiles straight from
-// its own parameters.
+// its own parameters; it also clears the call's status word.  The payload comes in three sizes,
+// so that a small schedule does not pay for uploading 30 KB of launch parameters.
+template <int kBytes>
 struct ScheduleChunk {
   uint4* dst;                // the image's place in the workspace
   TileTask* tasks;           // the expanded task list
+  int* status;               // cleared by the first thread (may be null)
   uint32_t n16;              // image size, 16-byte words
   uint32_t off_tiles;        // byte offset of the tiles in the image (the groups start at 0)
   int32_t ngroups, ntasks;
-  uint4 data[kInlineBytes / 16];
+  uint4 data[kBytes / 16];
 };
 
-__global__ void __launch_bounds__(256) schedule_kernel(const __grid_constant__ ScheduleChunk c) {
-  if (blockIdx.x == 0)
+template <int kBytes>
+__global__ void __launch_bounds__(256) schedule_kernel(const __grid_constant__ ScheduleChunk<kBytes> c) {
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0 && c.status) *c.status = 0;
     for (uint32_t i = threadIdx.x; i < c.n16; i += blockDim.x) c.dst[i] = c.data[i];
+  }
   const PlanGroup* groups = reinterpret_cast<const PlanGroup*>(c.data);
   const TileTask* tiles = reinterpret_cast<const TileTask*>(reinterpret_cast<const unsigned char*>(c.data) + c.off_tiles);
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < c.ntasks; i += gridDim.x * blockDim.x) {
@@ -231,6 +237,23 @@ __global__ void __launch_bounds__(256) schedule_kernel(const __grid_constant__ S
     t.head = local / g.ntiles;
     c.tasks[i] = t;
   }
+}
+
+template <int kBytes>
+int launch_schedule_t(void* image_dst, const void* image, size_t bytes, size_t off_tiles, int ngroups, TileTask* tasks,
+                      int ntasks, int* status, cudaStream_t stream) {
+  ScheduleChunk<kBytes> c;
+  c.dst = static_cast<uint4*>(image_dst);
+  c.tasks = tasks;
+  c.status = status;
+  c.n16 = (uint32_t)(bytes / 16);
+  c.off_tiles = (uint32_t)off_tiles;
+  c.ngroups = ngroups;
+  c.ntasks = ntasks;
+  memcpy(c.data, image, bytes);
+  const int blocks = std::min((ntasks + 255) / 256, 148 * 4);
+  schedule_kernel<kBytes><<<blocks, 256, 0, stream>>>(c);
+  return launched();
 }
 
 __global__ void __launch_bounds__(256) expand_tasks_kernel(const PlanGroup* __restrict__ groups, int ngroups,
@@ -423,7 +446,8 @@ int launch_inline_copy(void* dst, const void* src, size_t bytes, cudaStream_t st
 }
 
 int launch_schedule(void* image_dst, const void* image, size_t bytes, size_t off_tiles, int ngroups, TileTask* tasks,
-                    int ntasks, cudaStream_t stream) {
+                    int ntasks, int* status, cudaStream_t stream, bool* status_cleared) {
+  *status_cleared = false;
   if (ntasks == 0 || ngroups == 0) return 0;
   if (bytes > (size_t)kInlineBytes || bytes % 16) {  // larger images: copy in pieces, then expand
     int e = launch_inline_copy(image_dst, image, bytes, stream);
@@ -432,17 +456,10 @@ int launch_schedule(void* image_dst, const void* image, size_t bytes, size_t off
                                reinterpret_cast<const TileTask*>(static_cast<unsigned char*>(image_dst) + off_tiles),
                                tasks, ntasks, stream);
   }
-  ScheduleChunk c;
-  c.dst = static_cast<uint4*>(image_dst);
-  c.tasks = tasks;
-  c.n16 = (uint32_t)(bytes / 16);
-  c.off_tiles = (uint32_t)off_tiles;
-  c.ngroups = ngroups;
-  c.ntasks = ntasks;
-  memcpy(c.data, image, bytes);
-  const int blocks = std::min((ntasks + 255) / 256, 148 * 4);
-  schedule_kernel<<<blocks, 256, 0, stream>>>(c);
-  return launched();
+  *status_cleared = status != nullptr;
+  if (bytes <= 2048) return launch_schedule_t<2048>(image_dst, image, bytes, off_tiles, ngroups, tasks, ntasks, status, stream);
+  if (bytes <= 8192) return launch_schedule_t<8192>(image_dst, image, bytes, off_tiles, ngroups, tasks, ntasks, status, stream);
+  return launch_schedule_t<kInlineBytes>(image_dst, image, bytes, off_tiles, ngroups, tasks, ntasks, status, stream);
 }
 
 int launch_expand_tasks(const PlanGroup* groups, int ngroups, const TileTask* tiles, TileTask* tasks, int ntasks,
