@@ -130,7 +130,8 @@ enum PBar {
   pPFull = 11,   // +tile
   pPVDone = 13,  // +tile
   pODone = 15,
-  pNum = 16
+  pPHalf = 16,   // +tile: the first 64 columns of P are in TMEM (pPFull: all 128)
+  pNum = 18
 };
 
 template <int D, bool PAGED>
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
       mbar_init(&bar[pVEmpty + s], 1);
       mbar_init(&bar[pSFull + s], 1);
       mbar_init(&bar[pPFull + s], 4);
+      mbar_init(&bar[pPHalf + s], 4);
       mbar_init(&bar[pPVDone + s], 1);
     }
     mbar_init(&bar[pODone], 1);
@@ -270,13 +272,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         }
         umma_commit(&bar[pSFull + x]);
       };
-      // PV_x of k tile i (V stage i & 1); `first` starts O_x afresh
-      auto issue_pv = [&](int x, int i, bool first) {
+      // PV_x of k tile i (V stage i & 1); `first` starts O_x afresh.  The first 64 keys' half runs
+      // as soon as the softmax has stored that half of P (parity ph of pPHalf), the rest once all
+      // of P is in (the caller has waited for pPFull); returns false if the half's wait gave up.
+      auto issue_pv_half = [&](int x, int i, bool first, int half_i) {
         const uint64_t dv = sdesc_add(dV0, (i & 1) * L::kTile);
         const uint32_t tp = tmem + x * 128, to = tmem + 256 + x * D;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int k4 = 0; k4 < BN / 32; ++k4) {
+          const int kk = half_i * (BN / 32) + k4;
           umma_bf16_ts(to, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc_o, (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int x, int i, bool first) {
+        issue_pv_half(x, i, first, 1);
         umma_commit(&bar[pPVDone + x]);
       };
       if (!has_b) {
@@ -293,6 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           const int x = i & 1;
           const uint32_t ph = (i >> 1) & 1;  // half x's own tile count, and stage x's load count
           if (!mbar_wait_warp(&bar[pVFull + x], ph, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
+          if (!mbar_wait_warp(&bar[pPHalf + x], ph, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv_half(x, i, i < 2, 0);
           if (!mbar_wait_warp(&bar[pPFull + x], ph, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
           tc_fence_after();
           issue_pv(x, i, i < 2);
@@ -318,6 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         const int st = i & 1;
         if (!mbar_wait_warp(&bar[pVFull + st], (i >> 1) & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
         for (int x = 0; x < ntile && ok; ++x) {
+          if (!mbar_wait_warp(&bar[pPHalf + x], i & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv_half(x, i, i == 0, 0);
           if (!mbar_wait_warp(&bar[pPFull + x], i & 1, p.status, kDevTimeoutMma, lim)) { ok = false; break; }
           tc_fence_after();
           issue_pv(x, i, i == 0);
@@ -426,8 +441,39 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         const float msub = (m_use == -INFINITY) ? 0.f : m_use;
         float rowsum = 0.f, rowsum_r = 0.f;
         uint32_t pk[BN / 2];
+        // P in two halves of 64 keys: the first goes to TMEM (and its PV starts) while the second
+        // is being formed
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
+        for (int c = 0; c < BN / 2; c += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -msub));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -msub));
+          const uint32_t pb = pack_bf16x2(p0, p1);
+          rowsum += p0 + p1;
+          rowsum_r = add_bf16x2_f32(rowsum_r, pb);
+          pk[c / 2] = pb;
+        }
+        // PV of the previous k tile must be done: O is rescaled and P overwrites its input
+        if (i > 0 && !mbar_wait_warp(&bar[pPVDone + x], (i - 1) & 1, p.status, kDevTimeoutSoftmax, lim)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // 16 columns at a time: half of the scores are still held in registers here
+#pragma unroll 1
+          for (int c = 0; c < D; c += 16) {
+            uint32_t o[16];
+            tmem_ld16(tO + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(tO + c, o);
+          }
+        }
+        tmem_st32(tS, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[pPHalf + x]);
+#pragma unroll
+        for (int c = BN / 2; c < BN; c += 2) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -msub));
           const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -msub));
           const uint32_t pb = pack_bf16x2(p0, p1);
@@ -438,21 +484,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
         l = l * alpha + rowsum;
         lr = lr * alpha + rowsum_r;
         m = m_use;
-        // PV of the previous k tile must be done: O is rescaled and P overwrites its input
-        if (i > 0 && !mbar_wait_warp(&bar[pPVDone + x], (i - 1) & 1, p.status, kDevTimeoutSoftmax, lim)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale_o)) {
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + c, o);
-          }
-        }
-        tmem_st32(tS, pk);
         tmem_st32(tS + 32, pk + 32);
         tmem_st_wait();
         tc_fence_before();
