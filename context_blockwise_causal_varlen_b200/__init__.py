@@ -119,6 +119,7 @@ class KvpArgs(ctypes.Structure):
         ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("shard_out", ctypes.c_void_p),
         ("shard_lse", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("shard_base", ctypes.c_int32), ("total_shards", ctypes.c_int32),
     ]
 
 
@@ -683,9 +684,10 @@ def attn_block_bwd(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, scale=No
 def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_ROBIN, seg_size: int = 512,
                           scale=None, global_q_offset: int = 0, sliding_window: int = 0, per_shard: bool = False,
                           return_lse: bool = True, tp_out: bool = False, out=None, lse=None, shard_out=None,
-                          shard_lse=None, workspace=None):
+                          shard_lse=None, workspace=None, shard_base: int = 0, total_shards: int = 0):
     """Paged KV-parallel prefill; q ``[HQ, S, D]`` -> ``out [HQ, S, D]`` (``[HQ, D, S]`` with ``tp_out``)
-    (+ lse, + per-shard partials)."""
+    (+ lse, + per-shard partials).  ``block_tables`` are shards ``shard_base ..`` of ``total_shards``
+    (0: all of them): key positions follow the global shard index."""
     if not q.is_cuda or q.dtype != torch.bfloat16:
         raise CbvError(-3, "q must be a CUDA bfloat16 tensor")
     k_cache, v_cache = _bf16(k_cache, "k_cache"), _bf16(v_cache, "v_cache")
@@ -713,7 +715,8 @@ def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_RO
                 kv_mode=int(kv_mode), seg_size=int(seg_size), scale=_scale(scale),
                 global_q_offset=int(global_q_offset), sliding_window=int(sliding_window), tp_out=int(bool(tp_out)),
                 out=_ptr(out),
-                lse=_ptr(lse), shard_out=_ptr(so), shard_lse=_ptr(sl))
+                lse=_ptr(lse), shard_out=_ptr(so), shard_lse=_ptr(sl), shard_base=int(shard_base),
+                total_shards=int(total_shards))
     if q.stride(2) != 1:
         raise CbvError(-4, "q's last dimension must be contiguous")
     ws = _given_workspace(workspace, lib().cbv_kvp_workspace_size(ctypes.byref(a)), q.device)

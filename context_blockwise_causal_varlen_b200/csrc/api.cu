@@ -593,6 +593,10 @@ static int kvp_checks(const cbv_kvp_args* a) {
     return fail(CBV_ERR_MISALIGNED, "tensors must be 16-byte aligned");
   if ((a->q_stride_token % 8) || (a->q_stride_head % 8)) return fail(CBV_ERR_MISALIGNED, "q strides must be multiples of 8 elements");
   if ((a->shard_out == nullptr) != (a->shard_lse == nullptr)) return fail(CBV_ERR_BAD_ARG, "shard_out and shard_lse go together");
+  if (a->shard_base < 0 || a->total_shards < 0 ||
+      (int64_t)a->shard_base + a->shards > (a->total_shards ? (int64_t)a->total_shards : (int64_t)a->shards))
+    return fail(CBV_ERR_BAD_ARG, "shards %d from shard_base %d exceed total_shards %d", a->shards, a->shard_base,
+                a->total_shards);
   return CBV_OK;
 }
 
@@ -626,7 +630,8 @@ static int32_t kvp_segment(int32_t seg_size) { return (int32_t)std::min<int64_t>
 static size_t kvp_layout(const cbv_kvp_args* a, Plan* plan_out, int* tail_out) {
   const int n_local = a->blocks_per_shard * a->block_size;
   Plan plan = plan_kvp(a->q_len, a->num_heads, a->shards, n_local, kvp_segment(a->seg_size), (KvMode)a->kv_mode,
-                       a->block_size, a->global_q_offset, a->sliding_window, a->shard_out != nullptr, kPairRows);
+                       a->block_size, a->global_q_offset, a->sliding_window, a->shard_out != nullptr, kPairRows,
+                       a->shard_base, a->total_shards);
   const int tail = a->shard_out ? 0 : kvp_tail_tasks(plan);
   Carve c(nullptr);
   c.take(kStatusBytes);
@@ -689,6 +694,8 @@ int cbv_kvp_segmented_prefill(const cbv_kvp_args* a, void* stream) {
   p.blocks_per_shard = a->blocks_per_shard;
   p.block_size = bs;
   p.shards = a->shards;
+  p.shard_base = a->shard_base;
+  p.total_shards = a->total_shards ? a->total_shards : a->shards;
   p.kv_mode = a->kv_mode;
   p.n_local = a->blocks_per_shard * bs;
   p.q_rows = a->q_len;

@@ -51,14 +51,15 @@ struct KIter {
   Seg seg;
 };
 
-// global position of shard-local token t of a paged KV cache (block_size is a power of two:
-// the call accepts only divisors of 128)
+// global position of shard-local token t of the call's shard `shard` of a paged KV cache (its global
+// index is shard_base + shard of total_shards; block_size is a power of two: the call accepts only
+// divisors of 128)
 __device__ __forceinline__ int32_t kvp_position(const FwdParams& p, int32_t shard, int32_t t) {
   if (p.kv_mode == kKvRoundRobin) {
     const int lbs = __ffs(p.block_size) - 1;
-    return ((((t >> lbs) * p.shards + shard)) << lbs) + (t & (p.block_size - 1));
+    return ((((t >> lbs) * p.total_shards + p.shard_base + shard)) << lbs) + (t & (p.block_size - 1));
   }
-  return shard * p.n_local + t;
+  return (p.shard_base + shard) * p.n_local + t;
 }
 
 // k tiles that at least one row of q positions [qp0, qp1] can see.  Every role runs
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           // invert delta at the row's two bounds (two divisions per row instead of a position per
           // score)
           const int lbs = __ffs(p.block_size) - 1;
-          const int32_t bs = p.block_size, page_stride = p.shards << lbs;
+          const int32_t bs = p.block_size, page_stride = p.total_shards << lbs;
           int32_t hi = r.nvalid - 1, lo = 0;
           if (cz) {
             const int32_t x = qpos - r.kpos0;  // largest visible delta

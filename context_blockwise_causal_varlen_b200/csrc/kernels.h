@@ -56,6 +56,7 @@ struct FwdParams {
   // paged KV
   const int32_t* block_tables;  // [shards, blocks_per_shard]
   int32_t blocks_per_shard, block_size, shards, kv_mode, n_local;
+  int32_t shard_base, total_shards;  // the call's shard s is shard shard_base + s of total_shards (positions)
   int* status;  // device status word (0 = ok)
   // diagnostics: every wait gives up after wait_limit_ns (0 = the default limit); with
   // withhold_loads the producer issues no copy at all, so every wait runs out (the test of the

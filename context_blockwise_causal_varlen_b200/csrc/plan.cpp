@@ -569,8 +569,14 @@ Plan plan_block_bwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qba
 }
 
 Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int32_t seg_size, KvMode mode,
-              int32_t block_size, int32_t global_q_offset, int32_t window, bool per_shard, int32_t tile_m) {
+              int32_t block_size, int32_t global_q_offset, int32_t window, bool per_shard, int32_t tile_m,
+              int32_t shard_base, int32_t total_shards) {
   Plan plan;
+  if (total_shards <= 0) total_shards = shards;
+  // key position of local token t of the call's shard r (its global index is shard_base + r)
+  auto kpos = [&](int32_t r, int64_t t) {
+    return kvp_position(shard_base + r, t, n_local, block_size, total_shards, mode);
+  };
   const int64_t q_lo = global_q_offset, q_hi = (int64_t)global_q_offset + q_len - 1;
   std::vector<int32_t> shard_seg0(shards), shard_nseg(shards);
   for (int32_t r = 0; r < shards; ++r) {
@@ -578,8 +584,8 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
     bool first = true;
     for (int32_t s0 = 0; s0 < n_local; s0 += seg_size) {
       const int32_t rows = std::min(seg_size, n_local - s0);
-      const int64_t kmin = kvp_position(r, s0, n_local, block_size, shards, mode);
-      const int64_t kmax = kvp_position(r, s0 + rows - 1, n_local, block_size, shards, mode);
+      const int64_t kmin = kpos(r, s0);
+      const int64_t kmax = kpos(r, s0 + rows - 1);
       // drop segments no query can see (causal: kmin > last q; window: kmax too old for the first q)
       if (kmin > q_hi) continue;
       if (window > 0 && q_lo - kmax >= window && q_hi - kmax >= window) continue;
@@ -600,10 +606,11 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
       t.nseg = per_shard ? shard_nseg[r] : (int32_t)plan.segs.size();
       t.aux = per_shard ? r : -1;
       t.head = 0;
-      // weight: visible keys of the tile (every key position below the tile is one page of some shard)
+      // weight: visible keys of the tile (every key position below the tile is one page of some shard;
+      // this call holds shards / total_shards of them)
       int64_t lo = window > 0 ? std::max<int64_t>(0, pos0 - window + 1) : 0;
       int64_t span = (int64_t)pos0 + rows - lo;
-      t.work = weight((int64_t)rows * span / (per_shard ? shards : 1));
+      t.work = weight((int64_t)rows * span * shards / total_shards / (per_shard ? shards : 1));
       // where to cut the segment list for two halves of about equal work: count the 128-key
       // tiles of each segment this tile sees (the kernel's own skip rule)
       int64_t total = 0;
@@ -614,8 +621,8 @@ Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int
         int64_t n = 0;
         for (int32_t c0 = 0; c0 < g.rows; c0 += 128) {
           const int32_t nv = std::min(128, g.rows - c0);
-          const int64_t kp0 = kvp_position(r, g.row0 + c0, n_local, block_size, shards, mode);
-          const int64_t kp1 = kvp_position(r, g.row0 + c0 + nv - 1, n_local, block_size, shards, mode);
+          const int64_t kp0 = kpos(r, g.row0 + c0);
+          const int64_t kp1 = kpos(r, g.row0 + c0 + nv - 1);
           if (kp0 > (int64_t)pos0 + rows - 1) continue;
           if (window > 0 && kp1 < (int64_t)pos0 - window + 1) continue;
           ++n;

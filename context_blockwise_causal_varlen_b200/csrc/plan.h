@@ -131,8 +131,11 @@ Plan plan_block_bwd(const int32_t* cu_q, const int32_t* cu_k, const int32_t* qba
                     int32_t num_docs, bool causal, int32_t window, int32_t kv_heads, int32_t tile_n);
 // Paged KV-parallel prefill: one task per 128-row q tile per q head; segments = seg_size
 // pieces of every shard's local KV (or of one shard when per_shard is set, one task per shard).
+// The call's shards are shards shard_base .. shard_base + shards - 1 of total_shards (positions
+// follow the global index).
 Plan plan_kvp(int32_t q_len, int32_t heads, int32_t shards, int32_t n_local, int32_t seg_size, KvMode mode,
-              int32_t block_size, int32_t global_q_offset, int32_t window, bool per_shard, int32_t tile_m);
+              int32_t block_size, int32_t global_q_offset, int32_t window, bool per_shard, int32_t tile_m,
+              int32_t shard_base = 0, int32_t total_shards = 0);
 
 // Global position of shard-local token t (paged prefill).
 inline int64_t kvp_position(int32_t shard, int64_t t, int32_t n_local, int32_t block_size, int32_t shards, KvMode mode) {

@@ -21,6 +21,13 @@ per-position cache diagonals merge into it shard-locally.  The backward gathers
 dout, q, k, v and the MERGED out/lse the same way and runs block 0's backward
 against the merged statistics; the diagonals' gradients are closed-form and local.
 
+KV-parallel prefill (NKI attention_kv_parallel_segmented_cte: every shard attends its own
+paged KV, the shards' partial (out, lse) merge by the log-sum-exp identity).  Every rank
+holds the pages of its own shards and the whole q; it computes its shards' partials
+(``cbv_kvp_segmented_prefill`` with ``shard_base`` / ``total_shards``, so that key
+positions follow the global shard index), the partials are all-gathered, and every rank
+merges all of them in shard order.
+
 Every arithmetic step runs in libcbv.so; torch.distributed moves the data (NCCL on
 GPUs; with ``via_host=True`` the tensors travel through host memory, which lets a
 gloo group carry the exchange).  No kernel of one rank ever waits on another rank.
@@ -30,8 +37,9 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (attn_block_bwd, attn_block_fwd, cached_diag_grad, cached_diag_merge, convert_f32_bf16,
-               ring_step_bwd, ring_step_fwd, swap_leading_axes)
+from . import (KV_ROUND_ROBIN, attn_block_bwd, attn_block_fwd, attn_merge, cached_diag_grad, cached_diag_merge,
+               convert_f32_bf16, kvp_segmented_prefill as _kvp_prefill, ring_step_bwd, ring_step_fwd,
+               swap_leading_axes)
 
 
 class RingComm:
@@ -250,3 +258,40 @@ class _Ops:
     @staticmethod
     def finish(x):
         return convert_f32_bf16(x)
+
+
+# ----------------------------------------------------------------------------- KV-parallel prefill
+def _all_gather(x: torch.Tensor, group, via_host: bool) -> list[torch.Tensor]:
+    world = dist.get_world_size(group)
+    src = x.detach().to("cpu") if via_host else x.contiguous()
+    parts = [torch.empty_like(src) for _ in range(world)]
+    dist.all_gather(parts, src, group=group)
+    return [t.to(x.device) for t in parts] if via_host else parts
+
+
+def kvp_segmented_prefill(q, k_cache, v_cache, block_tables, kv_mode=KV_ROUND_ROBIN, seg_size: int = 512,
+                          scale=None, global_q_offset: int = 0, sliding_window: int = 0, group=None,
+                          via_host: bool = False, partial=None, merge=attn_merge, finish=convert_f32_bf16):
+    """KV-parallel prefill with the shards on the ranks of ``group``.  Rank r holds the pages of shards
+    ``r*n .. r*n + n - 1`` (``block_tables`` ``[n, blocks]`` into its own page pool ``k_cache`` /
+    ``v_cache``; ``n`` the same on every rank) and the whole ``q [HQ, S, D]``.  Returns the same
+    ``(out bf16 [HQ, S, D], lse f32 [HQ, S])`` on every rank.  ``partial(shard_base, total_shards)``
+    computes this rank's ``(shard_out f32 [n, HQ, S, D], shard_lse f32 [n, HQ, S])`` (default: the
+    paged prefill kernel); ``merge`` is the online-softmax merge (default: ``attn_merge``)."""
+    world, r = dist.get_world_size(group), dist.get_rank(group)
+    n = block_tables.shape[0]
+    HQ, S, D = q.shape
+    if partial is None:
+        def partial(shard_base, total_shards):
+            res = _kvp_prefill(q, k_cache, v_cache, block_tables, kv_mode, seg_size, scale, global_q_offset,
+                               sliding_window, per_shard=True, return_lse=False, shard_base=shard_base,
+                               total_shards=total_shards)
+            return res[1], res[2]
+    so, sl = partial(r * n, world * n)
+    outs = torch.cat(_all_gather(so, group, via_host))  # [world * n, HQ, S, D], in global shard order
+    lses = torch.cat(_all_gather(sl, group, via_host))
+    out, lse = outs[0].clone(), lses[0].clone()
+    # one (row, head) pair per merge row: [HQ * S, 1, D] outputs, [1, HQ * S] lse
+    for i in range(1, outs.shape[0]):
+        merge(out.view(HQ * S, 1, D), lse.view(1, HQ * S), outs[i].view(HQ * S, 1, D), lses[i].view(1, HQ * S))
+    return finish(out), lse

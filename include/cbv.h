@@ -509,6 +509,13 @@ typedef struct cbv_kvp_args {
   float* shard_lse;           /* with shard_out: device f32 [shards, num_heads, q_len] */
   void* workspace;
   size_t workspace_bytes;
+  /* This call's block tables are shards shard_base .. shard_base + shards - 1 of total_shards
+   * (0: total_shards = shards, shard_base = 0).  Key positions follow the global shard index, so a
+   * process that holds only its own shards' pages computes their partials, which merge with the
+   * other processes' ones by the log-sum-exp identity (the KV-parallel prefill over real ranks).
+   * Requires 0 <= shard_base and shard_base + shards <= total_shards. */
+  int32_t shard_base;
+  int32_t total_shards;
 } cbv_kvp_args;
 /* Workspace bytes for a call with these arguments on the current device.  The size depends on
  * the device's SM count: when the last wave of the prefill's tasks would fill at most half the

@@ -356,11 +356,24 @@ def _kvp_args(**kw):
     ("shards", 0, "BAD_SHAPE"),
     ("num_kv_heads", 3, "GQA_MISMATCH"),
     ("workspace", None, "WORKSPACE_TOO_SMALL"),
+    ("shard_base", -1, "BAD_ARG"),
+    ("total_shards", 1, "BAD_ARG"),   # the call's two shards do not fit in one
+    ("shard_base", 1, "BAD_ARG"),     # shards 1 and 2 of two (total_shards 0: the call's own count)
 ])
 def test_prefill_argument_errors(field, value, status):
     a = _kvp_args(**{field: value})
     rc = cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(a), None)
     assert cbv.STATUS[rc] == status, cbv.lib().cbv_last_error_message()
+
+
+def test_prefill_shard_range_within_the_total():
+    # shards 2 and 3 of four pass the checks (the call then stops at the missing workspace); 3 and 4 do not
+    ok = _kvp_args(shard_base=2, total_shards=4)
+    assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(ok), None)] == "WORKSPACE_TOO_SMALL"
+    assert cbv.lib().cbv_kvp_workspace_size(ctypes.byref(ok)) > 0
+    bad = _kvp_args(shard_base=3, total_shards=4)
+    assert cbv.STATUS[cbv.lib().cbv_kvp_segmented_prefill(ctypes.byref(bad), None)] == "BAD_ARG"
+    assert cbv.lib().cbv_kvp_workspace_size(ctypes.byref(bad)) == 0
 
 
 @pytest.mark.parametrize("field,value,status", [

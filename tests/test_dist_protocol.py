@@ -1,4 +1,4 @@
-"""The multi-rank drivers (ring over real ranks, Ulysses) with two gloo ranks on CPU.
+"""The multi-rank drivers (ring over real ranks, Ulysses, KV-parallel prefill) with two gloo ranks on CPU.
 
 The exchange code under test is the package's own: ``RingComm`` (send to rank+1,
 receive from rank-1, commit / wait), the ring forward and backward with the dK/dV
@@ -242,3 +242,69 @@ def test_ulysses_over_two_ranks_equals_the_joint_softmax(case):
     np.testing.assert_allclose(dck, rk, atol=1e-9)
     np.testing.assert_allclose(dcv, rv, atol=1e-9)
     assert out.shape == (S, H, D) and n * world == S
+
+
+# ----------------------------------------------------------------------------- KV-parallel prefill
+def _kvp_inputs():
+    from oracle import paged as PG
+    from synth import block_permutation
+
+    R, bps, bs, hq, hkv, D, S = 4, 2, 8, 2, 1, 8, 24
+    g = streams(7, 4)
+    q = normal_bf16(g[0], (hq, S, D)).astype(np.float64)
+    kc = normal_bf16(g[1], (R * bps, hkv, bs, D)).astype(np.float64)
+    vc = normal_bf16(g[2], (R * bps, hkv, bs, D)).astype(np.float64)
+    bt = PG.shard_block_tables(block_permutation(g[3], R * bps), R, PG.ROUND_ROBIN)
+    return q, kc, vc, bt, R * bps * bs - S - 3
+
+
+def _kvp_worker(rank, world, port, res):
+    from context_blockwise_causal_varlen_b200 import dist as cdist
+    from oracle import paged as PG
+    from oracle.attention import attention_fwd_masked
+
+    _init(rank, world, port)
+    try:
+        q, kc, vc, bt, gqo = _kvp_inputs()
+        n, bs, R = 2, 8, bt.shape[0]
+        mine = bt[rank * n:(rank + 1) * n]
+
+        def partial(shard_base, total_shards):
+            # the shards' partials from the oracle, at their GLOBAL positions (shard_base + i of total_shards)
+            so, sl = [], []
+            for i in range(n):
+                kpos = PG.local_to_global_positions(shard_base + i, mine.shape[1] * bs, bs, total_shards,
+                                                    PG.ROUND_ROBIN)
+                mask = PG._mask(gqo + np.arange(q.shape[1]), kpos, 10)
+                o, l = attention_fwd_masked(q.transpose(1, 0, 2), PG.gather_shard_kv(kc, mine[i], bs),
+                                            PG.gather_shard_kv(vc, mine[i], bs), mask, 0.3)
+                so.append(o.transpose(1, 0, 2))
+                sl.append(l)
+            return torch.from_numpy(np.stack(so)), torch.from_numpy(np.stack(sl))
+
+        def merge(out, lse, bo, bl):
+            no, nl, _ = A.update_out_and_lse(_np(out), _np(lse), _np(bo), _np(bl))
+            out.copy_(torch.from_numpy(no))
+            lse.copy_(torch.from_numpy(nl))
+
+        out, lse = cdist.kvp_segmented_prefill(torch.from_numpy(q), None, None, torch.from_numpy(mine),
+                                               partial=partial, merge=merge, finish=lambda x: x)
+        res[rank] = (_np(out), _np(lse))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_kvp_prefill_over_two_ranks_equals_the_whole_context():
+    from oracle import paged as PG
+
+    world, port = 2, _free_port()
+    with mp.Manager() as m:
+        res = m.dict()
+        mp.spawn(_kvp_worker, args=(world, port, res), nprocs=world, join=True)
+        res = dict(res)
+    q, kc, vc, bt, gqo = _kvp_inputs()
+    K, V = PG.global_kv(kc, vc, bt, 8, PG.ROUND_ROBIN)
+    ro, rl = PG.prefill_full(q, K, V, 0.3, gqo, window=10)
+    for r in range(world):
+        np.testing.assert_allclose(res[r][0], ro, atol=1e-12)
+        np.testing.assert_allclose(res[r][1], rl, atol=1e-12)

@@ -4,9 +4,9 @@
 ranks simulated in one process: every rank's k/v visits every other rank in ring
 order, the running (out, lse) is merged on the GPU, and the backward adds into the
 owner's dK/dV directly (the accumulators' travel is the driver's and is covered by the
-multi-process tests).  (2) The package's drivers with two processes that share this
-GPU, over gloo with the tensors staged through host memory: no kernel of one process
-waits on the other.  (3) The Ulysses building blocks: the axis swap and the diagonal
+multi-process tests).  (2) The package's drivers (ring, Ulysses, KV-parallel prefill)
+with two processes that share this GPU, over gloo with the tensors staged through host
+memory: no kernel of one process waits on the other.  (3) The Ulysses building blocks: the axis swap and the diagonal
 merge / gradients on their own.
 """
 import datetime
@@ -111,6 +111,16 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
+def _kvp_case():
+    from oracle import paged as PG
+    from synth import block_permutation, streams
+
+    R, bps, bs, hq, hkv, D, S = 4, 4, 32, 4, 2, 128, 160
+    q, kc, vc = gen(85, (hq, S, D), (R * bps, hkv, bs, D), (R * bps, hkv, bs, D))
+    perm = block_permutation(streams(185, 1)[0], R * bps)
+    return q, kc, vc, PG.shard_block_tables(perm, R, PG.ROUND_ROBIN), R * bps * bs - S - 5
+
+
 def _dist_worker(rank, world, port, res):
     from context_blockwise_causal_varlen_b200 import dist as cdist
 
@@ -139,12 +149,21 @@ def _dist_worker(rank, world, port, res):
         g = cdist.ulysses_bwd(dev(do2[sl]), dev(q2[sl]), lck, lcv, o2, l2, cu2, scale=0.1, via_host=True)
         torch.cuda.synchronize()
         uly = (host(o2), host(l2), host(g[0]), [host(x) for x in g[1]], [host(x) for x in g[2]])
-        res[rank] = (ring, uly)
+        # KV-parallel prefill: rank r holds the pages of shards 2r, 2r + 1 of 4 in a pool of its own
+        q3, kc, vc, bt, gqo = _kvp_case()
+        mine = bt[2 * rank:2 * rank + 2]
+        pages = np.unique(mine)
+        remap = {int(pg): i for i, pg in enumerate(pages)}
+        local_bt = torch.tensor([[remap[int(pg)] for pg in row] for row in mine], dtype=torch.int32)
+        o3, l3 = cdist.kvp_segmented_prefill(dev(q3), dev(kc[pages]), dev(vc[pages]), local_bt, seg_size=128, scale=0.1,
+                                             global_q_offset=gqo, sliding_window=400, via_host=True)
+        torch.cuda.synchronize()
+        res[rank] = (ring, uly, (host(o3), host(l3)))
     finally:
         dist.destroy_process_group()
 
 
-def test_ring_and_ulysses_drivers_with_two_processes_on_this_gpu():
+def test_ring_ulysses_and_prefill_drivers_with_two_processes_on_this_gpu():
     world, port = 2, _free_port()
     ctx = mp.get_context("spawn")
     with ctx.Manager() as m:
@@ -184,6 +203,16 @@ def test_ring_and_ulysses_drivers_with_two_processes_on_this_gpu():
     check_rel(dq2, rq, what="ulysses dq")
     check_rel(dck, rk, what="ulysses dcache_k")
     check_rel(dcv, rv, what="ulysses dcache_v")
+    # KV-parallel prefill: every rank returns the whole result, the same on both
+    from oracle import paged as PG
+
+    q3, kc, vc, bt, gqo = _kvp_case()
+    K, V = PG.global_kv(f64(kc), f64(vc), bt, 32, PG.ROUND_ROBIN)
+    ro, rl = PG.prefill_full(f64(q3), K, V, 0.1, gqo, window=400)
+    for r in range(world):
+        check_out(res[r][2][0], ro, what=f"prefill out on rank {r}")
+        check_lse(res[r][2][1], rl, what=f"prefill lse on rank {r}")
+    assert np.array_equal(res[0][2][0], res[1][2][0]) and np.array_equal(res[0][2][1], res[1][2][1])
 
 
 # ----------------------------------------------------------------------------- Ulysses building blocks

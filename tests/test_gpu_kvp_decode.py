@@ -65,6 +65,41 @@ def test_kvp_per_shard_partials_and_their_merge():
         check_lse(host(sl[r]), shards[r][1], what=f"shard {r} lse")
 
 
+@pytest.mark.parametrize("mode,window", [(PG.ROUND_ROBIN, 0), (PG.CONTIGUOUS, 0), (PG.ROUND_ROBIN, 500)])
+def test_kvp_shards_split_over_calls_give_the_same_partials(mode, window):
+    # a call that holds only some of the shards (shard_base / total_shards, as a process that holds only
+    # its own pages would) computes exactly the partials the whole call computes for them, and the
+    # partials of two calls merge to the full result
+    R, bps, bs, hq, hkv, D, S = 4, 4, 32, 4, 2, 128, 200
+    q, kc, vc, perm = _paged(23, R, bps, bs, hq, hkv, D, S)
+    bt = PG.shard_block_tables(perm, R, mode)
+    gqo = R * bps * bs - S - 9
+    kv_mode = cbv.KV_ROUND_ROBIN if mode == PG.ROUND_ROBIN else cbv.KV_CONTIGUOUS
+    kw = dict(kv_mode=kv_mode, seg_size=128, scale=0.1, global_q_offset=gqo, sliding_window=window,
+              per_shard=True, return_lse=True)
+    _, _, so_all, sl_all = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt), **kw)
+    parts = []
+    for base in (0, 2):
+        (so_, sob), (sl_, slb) = guarded((2, hq, S, D), torch.float32), guarded((2, hq, S), torch.float32)
+        out, lse, so, sl = cbv.kvp_segmented_prefill(dev(q), dev(kc), dev(vc), torch.from_numpy(bt[base:base + 2]),
+                                                     shard_base=base, total_shards=R, shard_out=so_, shard_lse=sl_,
+                                                     **kw)
+        sync()
+        check_guards(so_, sob, what="shard_out")
+        check_guards(sl_, slb, what="shard_lse")
+        assert torch.equal(so, so_all[base:base + 2]) and torch.equal(sl, sl_all[base:base + 2])
+        parts.append((out, lse))
+    K, V = PG.global_kv(f64(kc), f64(vc), bt, bs, mode)
+    ro, rl = PG.prefill_full(f64(q), K, V, 0.1, gqo, window=window)
+    # the two calls' merged halves (each over its own shards) merge to the whole result
+    o32 = parts[0][0].float().reshape(hq * S, 1, D).contiguous()
+    l32 = parts[0][1].reshape(1, hq * S).contiguous()
+    cbv.attn_merge(o32, l32, parts[1][0].reshape(hq * S, 1, D), parts[1][1].reshape(1, hq * S))
+    sync()
+    check_lse(host(l32.reshape(hq, S)), rl)
+    np.testing.assert_allclose(host(o32.reshape(hq, S, D)), ro, atol=2e-2)
+
+
 def test_kvp_segment_size_does_not_change_the_result():
     R, bps, bs, hq, hkv, D, S = 2, 16, 16, 4, 2, 64, 256
     q, kc, vc, perm = _paged(22, R, bps, bs, hq, hkv, D, S)
