@@ -122,8 +122,8 @@ enum BBar {
   bQEmpty = 4,   // +stage (NS)
   bSFull = 7,
   bSFree = 8,
-  bPFull = 9,    // +P^T / dS^T buffer (2)
-  bPtFree = 11,  // +P^T / dS^T buffer (2)
+  bPFull = 9,    // +buffer (2): P^T (TMEM) and dS^T (shared memory) written
+  bPtFree = 11,  // +buffer (2): the UMMAs that read P^T / dS^T buffer b have completed
   bDQFull = 13,
   bDQFree = 14,
   bUnused15 = 15,
@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       // base descriptors, built once; per-instruction offsets are compile-time constants
       const uint64_t dK_k = sdesc_sw128(smem_u32(sK), 16, 1024);        // K as K-major A (S^T)
       const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024);    // K^T as MN-major A (dQ^T)
-      // P^T / dS^T buffer b of 2 (q tile j uses buffer j & 1)
       const uint64_t dV_k = sdesc_sw128(smem_u32(sV), 16, 1024);        // V as K-major A (dP^T)
+      // dS^T buffer b of 2 (q tile j uses buffer j & 1; P^T's buffer b is TMEM columns tPt + 32 b)
       const uint64_t dDSt[2] = {sdesc_sw128(smem_u32(sDSt), 16, 1024),     // dS^T, K-major A (dK)
                                 sdesc_sw128(smem_u32(sm + L::kDSt1), 16, 1024)};
       const uint64_t dDSt_mn[2] = {sdesc_sw128(smem_u32(sDSt), 16384, 1024),  // dS^T, MN-major B (dQ^T)
