@@ -37,6 +37,23 @@ constexpr int kThreads = 320;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: keep a stale max while it is within 2^8
 
+// Scores outside the columns [lo, hi] of this thread's row set to -inf, 32 columns at a time: a
+// chunk that every row of the warp sees whole is skipped, the others are tested column by column.
+// On a window's edge tile most chunks are whole for all 32 rows of a warp.  (A separate branch
+// that cleared the chunks no row sees pushed the kernel's scores into local memory.)  The warp
+// must be converged.
+template <int N>
+__device__ __forceinline__ void mask_outside(uint32_t (&s)[N], int32_t lo, int32_t hi) {
+#pragma unroll
+  for (int c0 = 0; c0 < N; c0 += 32) {
+    if (!__all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31)) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (c0 + e < lo || c0 + e > hi) s[c0 + e] = __float_as_uint(-INFINITY);
+    }
+  }
+}
+
 struct KTile {
   int32_t k_row;   // first row (non-paged: tensor row; paged: shard-local token)
   int32_t kpos0;   // position of column 0 (paged: position of the tile's first token)
@@ -388,9 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
           int32_t hi = r.nvalid - 1, lo = 0;
           if (cz) hi = min(hi, qpos - r.kpos0);
           if (W > 0) lo = max(lo, qpos - W + 1 - r.kpos0);
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
+          mask_outside(s, lo, hi);
         } else if (need_mask) {
           // round-robin pages: column c sits at kpos0 + delta(c), delta(c) = (c / bs) * shards * bs
           // + c % bs, which grows with c, so the columns a row sees are again one range [lo, hi]:
@@ -415,9 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_pp_kernel(const __grid_consta
               lo = max(lo, off >= bs ? (pg + 1) << lbs : (pg << lbs) + off);
             }
           }
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < lo || c > hi) s[c] = __float_as_uint(-INFINITY);
+          mask_outside(s, lo, hi);
         }
         // row maximum of the raw scores (the scale is positive, so it commutes)
         // eight independent chains (the max is exact in any order), so the reduction sits on the
