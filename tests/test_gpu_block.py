@@ -30,6 +30,24 @@ def test_block_forward_default_positions(lq, lk, causal, window, D):
         check_lse(host(lse), rl)
 
 
+@pytest.mark.parametrize("offset", [0, 5])
+@pytest.mark.parametrize("window", [31, 32, 33, 96, 128, 129])
+def test_window_edges_on_and_beside_every_32_column_boundary(window, offset):
+    # the forward masks 32 score columns at a time and skips the chunks that every row of a warp
+    # sees whole: windows whose lower edge falls just before, on and just after a chunk boundary,
+    # and queries shifted by a few positions against the keys, so the edges pass through every lane
+    L, H, D = 384, 2, 128
+    q, k, v = gen(30 + window + offset, (L, H, D), (L, H, D), (L, H, D))
+    qpos, kpos = offset + np.arange(L), np.arange(L)
+    ro, rl = A.attention_fwd(f64(q), f64(k), f64(v), [0, L], [0, L], 0.1, causal=True, window=window, qpos=qpos,
+                             kpos=kpos)
+    out, lse = cbv.attn_block_fwd(dev(q), dev(k), dev(v), [0, L], [0, L], scale=0.1, causal=True, window=window,
+                                  q_pos_base=[offset], k_pos_base=[0])
+    sync()
+    check_out(host(out), ro)
+    check_lse(host(lse), rl)
+
+
 def test_blocks_merged_in_place_equal_full_attention():
     # one document split into three key blocks with explicit global positions,
     # merged into a running pair by the fused epilogue in a scrambled order
