@@ -106,9 +106,11 @@ size_t cbv_launch_count(void);
  * kernel) records `start_event` on the call's stream right before the launch and `stop_event`
  * right after it, so cudaEventElapsedTime gives that kernel's device time without the call's
  * helper kernels.  In a call that launches several attention kernels (the stepwise schedule)
- * the events bracket the last one.  The events are caller-owned cudaEvent_t handles; NULL, NULL
- * clears the hook.  Returns CBV_OK; a failed record makes the call that launched return
- * CBV_ERR_CUDA. */
+ * the events bracket the last one.  The records are stream operations between launches and add
+ * to the time of the steps they sit in, so a throughput measurement should time steps without
+ * the hook and use it in a separate pass.  The events are caller-owned cudaEvent_t handles;
+ * NULL, NULL clears the hook.  Returns CBV_OK; a failed record makes the call that launched
+ * return CBV_ERR_CUDA. */
 int cbv_set_kernel_events(void* start_event, void* stop_event);
 
 /* How the library was built: CBV_BUILD_DEBUG is set in the bounds-checking build (libcbv_debug.so,
